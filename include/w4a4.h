@@ -39,7 +39,7 @@
  *   - Entry points return a W4A4_* status and never abort or print.  On an
  *     argument error nothing is launched.
  *   - Shapes: M >= 0 (M == 0 is a no-op), N and K multiples of 128,
- *     K <= 131072.  Device pointers 16-byte aligned; leading dimensions
+ *     K <= 65536.  Device pointers 16-byte aligned; leading dimensions
  *     multiples of 8 elements.
  */
 #ifndef W4A4_H
@@ -196,8 +196,9 @@ int w4a4_select_channels(const uint16_t* Xcal, int Mc, int K, int ldx, int nS,
 /*
  * Synchronize `stream`, then read and clear the library's device error word.
  * Returns W4A4_OK, W4A4_ERR_DEVICE_TIMEOUT (a kernel's bounded wait expired
- * and the kernel returned early; its outputs are undefined) or
- * W4A4_ERR_CUDA.
+ * and the kernel returned early; its outputs are undefined),
+ * W4A4_ERR_INVALID_ARG (a channel index in a device-side S was outside
+ * [0,K); it was replaced by channel 0) or W4A4_ERR_CUDA.
  */
 int w4a4_device_status(void* stream);
 

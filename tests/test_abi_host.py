@@ -1,0 +1,116 @@
+"""Host-side checks of the C-ABI library that need no GPU: it loads, exports
+every entry point the header declares, and rejects bad arguments before
+touching a device."""
+import ctypes as C
+import os
+import re
+
+import pytest
+
+import w4a4_quantized_gemm_token_b200 as w4
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "w4a4.h")
+
+
+@pytest.fixture(scope="module")
+def L():
+    from w4a4_quantized_gemm_token_b200 import build
+    build.build()
+    return w4.lib()
+
+
+def declared():
+    text = open(HEADER).read()
+    return sorted(set(re.findall(r"^\s*(?:int|size_t|void|const char\*)\s+(w4a4_\w+)\s*\(", text, re.M)))
+
+
+def test_header_lists_entry_points():
+    names = declared()
+    assert set(names) == set(w4.EXPORTS), names
+
+
+def test_every_declared_symbol_exported(L):
+    for name in declared():
+        assert hasattr(L, name), name
+
+
+def test_status_strings(L):
+    assert w4.status_string(w4.OK) == "ok"
+    assert "timed out" in w4.status_string(w4.ERR_DEVICE_TIMEOUT)
+    assert w4.status_string(99) == "unknown status"
+
+
+def test_qtensor_bytes(L):
+    c, s, t = w4.qtensor_bytes(w4.NVFP4, 200, 1024, w4.SCALE_TOKEN)
+    assert (c, s, t) == (200 * 512, 256 * 64, 800)
+    c, s, t = w4.qtensor_bytes(w4.NVFP4, 200, 1024, w4.SCALE_TENSOR)
+    assert t == 8
+    c, s, t = w4.qtensor_bytes(w4.MXFP4, 1, 256, 0)
+    assert (c, s, t) == (128, 128 * 8, 0)
+    c, s, t = w4.qtensor_bytes(w4.INT4, 130, 384, 0)
+    assert (c, s, t) == (130 * 192, 3 * 256 * 4, 0)
+    with pytest.raises(w4.W4A4Error):
+        w4.qtensor_bytes(w4.NVFP4, 4, 100, 0)
+    with pytest.raises(w4.W4A4Error):
+        w4.qtensor_bytes(7, 4, 128, 0)
+
+
+def test_workspace_sizes(L):
+    assert w4.linear_workspace(4096, 10240, 8192, w4.NVFP4) >= 4096 * 4096 + 4096 * 512
+    assert w4.linear_workspace(16, 10240, 8192, w4.NVFP4) >= 16 * 10240 * 4
+    assert w4.linear_workspace(16, 100, 8192, w4.NVFP4) == 0        # N not a multiple of 128
+    assert w4.linear_workspace(16, 256, 8192, w4.NVFP4, 100) == 0   # nS not a multiple of 128
+
+
+def _qt(fmt, rows, cols, mode=0, codes=16, scales=16, s2=16):
+    return w4.QTensorStruct(fmt, rows, cols, w4.GROUP[fmt], mode, 0, codes, scales, s2)
+
+
+def test_argument_errors_before_any_device_work(L):
+    q = _qt(w4.NVFP4, 4, 256, w4.SCALE_TOKEN)
+    ref = C.byref(q)
+    # bad K, bad group, bad format, rows mismatch: all rejected on the host
+    assert L.w4a4_quantize_act(C.c_void_p(16), 4, 100, 128, 0, 16, 1, None, ref, None) == w4.ERR_INVALID_ARG
+    assert L.w4a4_quantize_act(C.c_void_p(16), 4, 256, 256, 0, 32, 1, None, ref, None) == w4.ERR_INVALID_ARG
+    assert L.w4a4_quantize_act(C.c_void_p(16), 5, 256, 256, 0, 16, 1, None, ref, None) == w4.ERR_INVALID_ARG
+    assert L.w4a4_quantize_act(C.c_void_p(16), 4, 256, 200, 0, 16, 1, None, ref, None) == w4.ERR_INVALID_ARG
+    # misaligned X
+    assert L.w4a4_quantize_act(C.c_void_p(18), 4, 256, 256, 0, 16, 1, None, ref, None) == w4.ERR_MISALIGNED
+    # M == 0 is a no-op
+    q0 = _qt(w4.NVFP4, 0, 256, w4.SCALE_TOKEN)
+    assert L.w4a4_quantize_act(None, 0, 256, 256, 0, 16, 1, None, C.byref(q0), None) == w4.OK
+    # gemm: format mismatch, K mismatch, N not a multiple of 128
+    a = _qt(w4.NVFP4, 4, 256, w4.SCALE_TOKEN)
+    b = _qt(w4.MXFP4, 256, 256)
+    assert L.w4a4_gemm(C.byref(a), C.byref(b), C.c_void_p(16), 256, None) == w4.ERR_INVALID_ARG
+    b = _qt(w4.NVFP4, 256, 512, w4.SCALE_TENSOR)
+    assert L.w4a4_gemm(C.byref(a), C.byref(b), C.c_void_p(16), 256, None) == w4.ERR_INVALID_ARG
+    b = _qt(w4.NVFP4, 200, 256, w4.SCALE_TENSOR)
+    assert L.w4a4_gemm(C.byref(a), C.byref(b), C.c_void_p(16), 256, None) == w4.ERR_INVALID_ARG
+    # NVFP4 weights must carry a tensor scale
+    b = _qt(w4.NVFP4, 256, 256, w4.SCALE_TOKEN)
+    assert L.w4a4_gemm(C.byref(a), C.byref(b), C.c_void_p(16), 256, None) == w4.ERR_INVALID_ARG
+    # linear: workspace too small, residual channels with a non-NVFP4 weight
+    W = _qt(w4.NVFP4, 256, 256, w4.SCALE_TENSOR)
+    assert L.w4a4_linear(C.c_void_p(16), 4, 256, 256, C.byref(W), 1, None, 0, C.c_void_p(16), 256,
+                         C.c_void_p(256), 16, None) == w4.ERR_WORKSPACE
+    Wm = _qt(w4.MXFP4, 256, 384)
+    assert L.w4a4_linear(C.c_void_p(16), 4, 256, 256, C.byref(Wm), 1, C.c_void_p(16), 128, C.c_void_p(16), 256,
+                         C.c_void_p(256), 1 << 20, None) == w4.ERR_INVALID_ARG
+    # S with nS not a multiple of 128
+    assert L.w4a4_augment_residual(C.c_void_p(16), 4, 256, 256, C.c_void_p(16), 64, ref, None) == w4.ERR_INVALID_ARG
+    # channel selection: workspace too small
+    assert L.w4a4_select_channels(C.c_void_p(16), 4, 256, 256, 16, C.c_void_p(16), C.c_void_p(16), 8,
+                                  None) == w4.ERR_WORKSPACE
+
+
+def test_no_device_means_error_not_fallback(L):
+    """With valid arguments but no usable GPU the library reports an error
+    instead of computing anything on the host."""
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("a GPU is present")
+    q = _qt(w4.NVFP4, 4, 256, w4.SCALE_TOKEN)
+    rc = L.w4a4_quantize_act(C.c_void_p(16), 4, 256, 256, 0, 16, 1, None, C.byref(q), None)
+    assert rc in (w4.ERR_CUDA, w4.ERR_ARCH)

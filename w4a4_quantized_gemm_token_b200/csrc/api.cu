@@ -1,0 +1,417 @@
+// C-ABI of the W4A4 library: argument checks, tensor-map set-up and dispatch
+// to the kernels.  The library allocates no device memory; its only state is
+// a per-device property cache, the driver entry point of the tensor-map
+// encoder and the debug settings of w4a4_debug_set().
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "../../include/w4a4.h"
+#include "kernels.h"
+#include "ptx.cuh"
+
+using namespace w4a4;
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+constexpr int kMaxK = 65536;
+
+struct DevInfo {
+    bool init = false;
+    bool ok = false;
+    int num_sms = 0;
+};
+DevInfo g_dev[kMaxDevices];
+std::mutex g_mu;
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+
+int g_skip_k_tile = -1;
+unsigned long long g_wait_limit_ns = 2000000000ull;
+
+int device_check(int* num_sms) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return W4A4_ERR_CUDA;
+    std::lock_guard<std::mutex> lk(g_mu);
+    DevInfo& d = g_dev[dev];
+    if (!d.init) {
+        int major = 0, minor = 0, sms = 0;
+        if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+            return W4A4_ERR_CUDA;
+        d.ok = (major == 10 && minor == 0);
+        d.num_sms = sms;
+        d.init = true;
+    }
+    if (!d.ok) return W4A4_ERR_ARCH;
+    if (!g_encode) {
+        void* fn = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) != cudaSuccess ||
+            q != cudaDriverEntryPointSuccess || !fn)
+            return W4A4_ERR_CUDA;
+        g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+    }
+    if (num_sms) *num_sms = d.num_sms;
+    return W4A4_OK;
+}
+
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
+inline int pad128(int x) { return (x + 127) / 128 * 128; }
+inline size_t align256(size_t x) { return (x + 255) / 256 * 256; }
+
+int group_of(int fmt) { return fmt == W4A4_NVFP4 ? 16 : fmt == W4A4_MXFP4 ? 32 : fmt == W4A4_INT4 ? 128 : -1; }
+
+// 2-D byte tensor map over codes[rows][row_bytes] with a box of box_x bytes x box_y rows.
+int make_map(CUtensorMap* map, const void* base, int rows, int row_bytes, int box_x, int box_y, bool swizzle128) {
+    cuuint64_t dims[2] = {(cuuint64_t)row_bytes, (cuuint64_t)rows};
+    cuuint64_t strides[1] = {(cuuint64_t)row_bytes};
+    cuuint32_t box[2] = {(cuuint32_t)box_x, (cuuint32_t)box_y};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, estr,
+                          CU_TENSOR_MAP_INTERLEAVE_NONE,
+                          swizzle128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
+                          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? W4A4_OK : W4A4_ERR_CUDA;
+}
+
+int check_qtensor(const w4a4_qtensor* q) {
+    if (!q || !q->codes || !q->scales) return W4A4_ERR_INVALID_ARG;
+    if (q->format < 0 || q->format > 2 || q->group != group_of(q->format) || q->reserved != 0)
+        return W4A4_ERR_INVALID_ARG;
+    if (q->rows < 0 || q->cols < 128 || q->cols % 128 || q->cols > kMaxK + 32768) return W4A4_ERR_INVALID_ARG;
+    if (q->format == W4A4_NVFP4) {
+        if (!q->s2) return W4A4_ERR_INVALID_ARG;
+        if (q->scale_mode != W4A4_SCALE_TENSOR && q->scale_mode != W4A4_SCALE_TOKEN) return W4A4_ERR_INVALID_ARG;
+    }
+    if (!aligned16(q->codes) || !aligned16(q->scales) || (q->s2 && (reinterpret_cast<uintptr_t>(q->s2) & 3)))
+        return W4A4_ERR_MISALIGNED;
+    return W4A4_OK;
+}
+
+cudaStream_t as_stream(void* s) { return reinterpret_cast<cudaStream_t>(s); }
+
+int cuda_status(cudaError_t e) { return e == cudaSuccess ? W4A4_OK : W4A4_ERR_CUDA; }
+
+// Quantize rows [0, M) of X into the first K columns of q (q->cols >= K).
+int quantize_rows(const uint16_t* X, int M, int K, int ldx, const int32_t* S, int K_src, const float* static_s2,
+                  w4a4_qtensor* q, int num_sms, cudaStream_t st) {
+    QuantArgs a{};
+    a.X = X;
+    a.M = M;
+    a.K = K;
+    a.K_src = K_src;
+    a.ldx = ldx;
+    a.S = S;
+    a.codes = static_cast<uint8_t*>(q->codes);
+    a.ldc = q->cols / 2;
+    a.sf = static_cast<uint8_t*>(q->scales);
+    a.sf_col_atoms = q->cols / q->group / 4;
+    a.sfi = static_cast<float*>(q->scales);
+    a.sfi_ld = pad128(q->rows);
+    a.mode = q->scale_mode;
+    a.static_s2 = static_s2;
+    a.s2_out = q->s2;
+    a.tensor_amax = nullptr;
+    if (q->format == W4A4_NVFP4 && q->scale_mode == W4A4_SCALE_TENSOR && !static_s2) {
+        // dynamic tensor scale: amax pass into s2[1], then the quantizer reads it
+        cudaError_t e = cudaMemsetAsync(q->s2 + 1, 0, sizeof(float), st);
+        if (e == cudaSuccess) e = launch_amax(X, M, K_src, ldx, q->s2 + 1, num_sms, st);
+        if (e != cudaSuccess) return W4A4_ERR_CUDA;
+        a.tensor_amax = q->s2 + 1;
+    }
+    return cuda_status(launch_quant(q->format, S != nullptr, a, pad128(M), st));
+}
+
+int check_S_args(const int32_t* S, int nS, int K) {
+    if (nS < 0 || (nS > 0 && (!S || nS % 128 || nS > K))) return W4A4_ERR_INVALID_ARG;
+    if (nS == 0 && S) return W4A4_ERR_INVALID_ARG;
+    return W4A4_OK;
+}
+
+struct GemmSetup {
+    CUtensorMap ta, tb;
+    GemmArgs g;
+};
+
+// Fill tensor maps and arguments for A (activations) x B (weights).
+int setup_gemm(const w4a4_qtensor* A, const w4a4_qtensor* B, uint16_t* Y, int ldy, bool decode, GemmSetup* s) {
+    GemmArgs& g = s->g;
+    std::memset(&g, 0, sizeof(g));
+    g.M = A->rows;
+    g.N = B->rows;
+    g.K = A->cols;
+    g.sfa = static_cast<const uint8_t*>(A->scales);
+    g.sfb = static_cast<const uint8_t*>(B->scales);
+    g.sf_col_atoms = A->format == W4A4_INT4 ? 0 : A->cols / A->group / 4;
+    g.sfa_ld = pad128(A->rows);
+    g.sfb_ld = pad128(B->rows);
+    g.s2a = A->s2;
+    g.s2a_per_row = A->scale_mode == W4A4_SCALE_TOKEN ? 1 : 0;
+    g.s2b = B->s2;
+    g.Y = Y;
+    g.ldy = ldy;
+    g.skip_k_tile = g_skip_k_tile;
+    g.wait_limit_ns = g_wait_limit_ns;
+    const int row_bytes = A->cols / 2;
+    int rc;
+    if (A->format == W4A4_INT4) {
+        rc = make_map(&s->ta, A->codes, A->rows, row_bytes, 64, 128, false);
+        if (rc == W4A4_OK) rc = make_map(&s->tb, B->codes, B->rows, row_bytes, 64, kBN_I4, false);
+    } else if (!decode) {
+        rc = make_map(&s->ta, A->codes, A->rows, row_bytes, 128, kBM, true);
+        if (rc == W4A4_OK) rc = make_map(&s->tb, B->codes, B->rows, row_bytes, 128, kBN, true);
+    } else {
+        // weights take the MMA's M side (box of 128 rows), tokens its N side (16 rows)
+        rc = make_map(&s->ta, B->codes, B->rows, row_bytes, 128, kBM, true);
+        if (rc == W4A4_OK) rc = make_map(&s->tb, A->codes, A->rows, row_bytes, 128, kBN_DEC, true);
+    }
+    return rc;
+}
+
+// Split-K factor of the small-M variant: enough CTAs to cover every SM.
+void decode_split(int N, int K, int num_sms, int* splits, int* kps) {
+    const int KT = (K + kBK_FP4 - 1) / kBK_FP4;
+    const int ntiles = (N + kBM - 1) / kBM;
+    int want = (num_sms + ntiles - 1) / ntiles;
+    if (want < 1) want = 1;
+    if (want > KT) want = KT;
+    int per = (KT + want - 1) / want;
+    *kps = per;
+    *splits = (KT + per - 1) / per;
+}
+
+int run_gemm(const w4a4_qtensor* A, const w4a4_qtensor* B, uint16_t* Y, int ldy, float* partial, int num_sms,
+             bool pdl, cudaStream_t st) {
+    const bool decode = A->format != W4A4_INT4 && partial != nullptr;
+    GemmSetup s;
+    int rc = setup_gemm(A, B, Y, ldy, decode, &s);
+    if (rc != W4A4_OK) return rc;
+    cudaError_t e;
+    if (A->format == W4A4_INT4) {
+        e = launch_gemm_int4(s.ta, s.tb, s.g, num_sms, pdl, st);
+    } else if (decode) {
+        decode_split(s.g.N, s.g.K, num_sms, &s.g.splits, &s.g.k_tiles_per_split);
+        s.g.partial = partial;
+        e = launch_gemm_fp4_decode(A->format == W4A4_NVFP4, s.ta, s.tb, s.g, pdl, st);
+    } else {
+        e = launch_gemm_fp4(A->format == W4A4_NVFP4, s.ta, s.tb, s.g, num_sms, pdl, st);
+    }
+    return cuda_status(e);
+}
+
+// Workspace layout of w4a4_linear: quantized activation (codes, scales, s2),
+// then the split-K partial sums of the small-M variant.
+struct WsLayout {
+    size_t codes, scales, s2, partial, total;
+};
+
+WsLayout ws_layout(int M, int N, int K, int fmt, int nS) {
+    WsLayout w{};
+    const int cols = K + nS;
+    size_t cb = 0, sb = 0, s2b = 0;
+    w4a4_qtensor_bytes(fmt, M, cols, W4A4_SCALE_TOKEN, &cb, &sb, &s2b);
+    if (s2b < 8) s2b = 8;
+    w.codes = 0;
+    w.scales = align256(cb);
+    w.s2 = w.scales + align256(sb);
+    w.partial = w.s2 + align256(s2b);
+    size_t pb = 0;
+    if (fmt != W4A4_INT4 && M <= 16) {
+        const int KT = (cols + kBK_FP4 - 1) / kBK_FP4;
+        pb = (size_t)KT * M * N * sizeof(float);  // upper bound on splits x M x N
+    }
+    w.total = w.partial + align256(pb);
+    return w;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* w4a4_status_string(int status) {
+    switch (status) {
+        case W4A4_OK: return "ok";
+        case W4A4_ERR_INVALID_ARG: return "invalid argument";
+        case W4A4_ERR_MISALIGNED: return "misaligned pointer or leading dimension";
+        case W4A4_ERR_WORKSPACE: return "workspace missing or too small";
+        case W4A4_ERR_ARCH: return "device is not sm_100";
+        case W4A4_ERR_CUDA: return "CUDA error";
+        case W4A4_ERR_DEVICE_TIMEOUT: return "in-kernel wait timed out";
+        default: return "unknown status";
+    }
+}
+
+int w4a4_qtensor_bytes(int format, int rows, int cols, int scale_mode, size_t* codes_bytes, size_t* scales_bytes,
+                       size_t* s2_bytes) {
+    const int g = group_of(format);
+    if (g < 0 || rows < 0 || cols < 0 || cols % 128) return W4A4_ERR_INVALID_ARG;
+    size_t c = (size_t)rows * (cols / 2);
+    size_t s = format == W4A4_INT4 ? (size_t)(cols / 128) * pad128(rows) * sizeof(float)
+                                   : (size_t)pad128(rows) * (cols / g);
+    size_t t = 0;
+    if (format == W4A4_NVFP4) t = scale_mode == W4A4_SCALE_TOKEN ? (size_t)(rows > 0 ? rows : 1) * 4 : 8;
+    if (codes_bytes) *codes_bytes = c;
+    if (scales_bytes) *scales_bytes = s;
+    if (s2_bytes) *s2_bytes = t;
+    return W4A4_OK;
+}
+
+int w4a4_quantize_act(const uint16_t* X, int M, int K, int ldx, int format, int group, int scale_mode,
+                      const float* static_s2, w4a4_qtensor* out, void* stream) {
+    if (M < 0 || K < 128 || K % 128 || K > kMaxK || ldx < K) return W4A4_ERR_INVALID_ARG;
+    if (group_of(format) != group) return W4A4_ERR_INVALID_ARG;
+    int rc = check_qtensor(out);
+    if (rc != W4A4_OK) return rc;
+    if (out->format != format || out->group != group || out->rows != M || out->cols < K ||
+        (format == W4A4_NVFP4 && out->scale_mode != scale_mode))
+        return W4A4_ERR_INVALID_ARG;
+    if (format != W4A4_NVFP4 && static_s2) return W4A4_ERR_INVALID_ARG;
+    if (M == 0) return W4A4_OK;
+    if (!X) return W4A4_ERR_INVALID_ARG;
+    if (!aligned16(X) || ldx % 8) return W4A4_ERR_MISALIGNED;
+    int sms = 0;
+    rc = device_check(&sms);
+    if (rc != W4A4_OK) return rc;
+    return quantize_rows(X, M, K, ldx, nullptr, K, static_s2, out, sms, as_stream(stream));
+}
+
+int w4a4_quantize_weight(const uint16_t* W, int N, int K, int ldw, int format, int group, const int32_t* S, int nS,
+                         w4a4_qtensor* out, void* stream) {
+    if (N < 0 || K < 128 || K % 128 || K > kMaxK || ldw < K) return W4A4_ERR_INVALID_ARG;
+    if (group_of(format) != group) return W4A4_ERR_INVALID_ARG;
+    int rc = check_S_args(S, nS, K);
+    if (rc != W4A4_OK) return rc;
+    rc = check_qtensor(out);
+    if (rc != W4A4_OK) return rc;
+    if (out->format != format || out->rows != N || out->cols != K + nS) return W4A4_ERR_INVALID_ARG;
+    if (format == W4A4_NVFP4 && out->scale_mode != W4A4_SCALE_TENSOR) return W4A4_ERR_INVALID_ARG;
+    if (N == 0) return W4A4_OK;
+    if (!W) return W4A4_ERR_INVALID_ARG;
+    if (!aligned16(W) || ldw % 8) return W4A4_ERR_MISALIGNED;
+    int sms = 0;
+    rc = device_check(&sms);
+    if (rc != W4A4_OK) return rc;
+    return quantize_rows(W, N, K + nS, ldw, nS ? S : nullptr, K, nullptr, out, sms, as_stream(stream));
+}
+
+int w4a4_gemm(const w4a4_qtensor* A, const w4a4_qtensor* B, uint16_t* Y, int ldy, void* stream) {
+    int rc = check_qtensor(A);
+    if (rc == W4A4_OK) rc = check_qtensor(B);
+    if (rc != W4A4_OK) return rc;
+    if (A->format != B->format || A->cols != B->cols || B->rows < 128 || B->rows % 128 || ldy < B->rows)
+        return W4A4_ERR_INVALID_ARG;
+    if (A->format == W4A4_NVFP4 && B->scale_mode != W4A4_SCALE_TENSOR) return W4A4_ERR_INVALID_ARG;
+    if (A->rows == 0) return W4A4_OK;
+    if (!Y) return W4A4_ERR_INVALID_ARG;
+    if (!aligned16(Y) || ldy % 8) return W4A4_ERR_MISALIGNED;
+    int sms = 0;
+    rc = device_check(&sms);
+    if (rc != W4A4_OK) return rc;
+    return run_gemm(A, B, Y, ldy, nullptr, sms, false, as_stream(stream));
+}
+
+size_t w4a4_linear_workspace(int M, int N, int K, int format, int nS) {
+    if (M < 0 || N < 128 || N % 128 || K < 128 || K % 128 || group_of(format) < 0 || nS < 0 || nS % 128)
+        return 0;
+    return ws_layout(M, N, K, format, nS).total;
+}
+
+int w4a4_linear(const uint16_t* X, int M, int K, int ldx, const w4a4_qtensor* Wq, int scale_mode, const int32_t* S,
+                int nS, uint16_t* Y, int ldy, void* ws, size_t ws_bytes, void* stream) {
+    int rc = check_qtensor(Wq);
+    if (rc != W4A4_OK) return rc;
+    const int fmt = Wq->format;
+    if (M < 0 || K < 128 || K % 128 || K > kMaxK || ldx < K) return W4A4_ERR_INVALID_ARG;
+    rc = check_S_args(S, nS, K);
+    if (rc != W4A4_OK) return rc;
+    if (nS && fmt != W4A4_NVFP4) return W4A4_ERR_INVALID_ARG;
+    if (Wq->cols != K + nS || Wq->rows < 128 || Wq->rows % 128 || ldy < Wq->rows) return W4A4_ERR_INVALID_ARG;
+    if (fmt == W4A4_NVFP4 && (Wq->scale_mode != W4A4_SCALE_TENSOR ||
+                              (scale_mode != W4A4_SCALE_TENSOR && scale_mode != W4A4_SCALE_TOKEN)))
+        return W4A4_ERR_INVALID_ARG;
+    if (M == 0) return W4A4_OK;
+    if (!X || !Y) return W4A4_ERR_INVALID_ARG;
+    if (!aligned16(X) || ldx % 8 || !aligned16(Y) || ldy % 8) return W4A4_ERR_MISALIGNED;
+    const int N = Wq->rows;
+    const WsLayout L = ws_layout(M, N, K, fmt, nS);
+    if (!ws || ws_bytes < L.total) return W4A4_ERR_WORKSPACE;
+    if (reinterpret_cast<uintptr_t>(ws) & 255) return W4A4_ERR_MISALIGNED;
+    int sms = 0;
+    rc = device_check(&sms);
+    if (rc != W4A4_OK) return rc;
+    cudaStream_t st = as_stream(stream);
+    uint8_t* base = static_cast<uint8_t*>(ws);
+    w4a4_qtensor xq{};
+    xq.format = fmt;
+    xq.rows = M;
+    xq.cols = K + nS;
+    xq.group = group_of(fmt);
+    xq.scale_mode = fmt == W4A4_NVFP4 ? scale_mode : 0;
+    xq.codes = base + L.codes;
+    xq.scales = base + L.scales;
+    xq.s2 = reinterpret_cast<float*>(base + L.s2);
+    rc = quantize_rows(X, M, K, ldx, nullptr, K, nullptr, &xq, sms, st);
+    if (rc != W4A4_OK) return rc;
+    if (nS) {
+        ResidualArgs r{X, M, K, ldx, pad128(M), S, nS, static_cast<uint8_t*>(xq.codes), xq.cols / 2,
+                       static_cast<uint8_t*>(xq.scales), xq.cols / 16 / 4, xq.s2, xq.scale_mode};
+        if (launch_residual(r, st) != cudaSuccess) return W4A4_ERR_CUDA;
+    }
+    float* partial = (fmt != W4A4_INT4 && M <= 16) ? reinterpret_cast<float*>(base + L.partial) : nullptr;
+    return run_gemm(&xq, Wq, Y, ldy, partial, sms, true, st);
+}
+
+int w4a4_augment_residual(const uint16_t* X, int M, int K, int ldx, const int32_t* S, int nS, w4a4_qtensor* Xaug,
+                          void* stream) {
+    if (M < 0 || K < 128 || K % 128 || K > kMaxK || ldx < K || nS <= 0) return W4A4_ERR_INVALID_ARG;
+    int rc = check_S_args(S, nS, K);
+    if (rc == W4A4_OK) rc = check_qtensor(Xaug);
+    if (rc != W4A4_OK) return rc;
+    if (Xaug->format != W4A4_NVFP4 || Xaug->rows != M || Xaug->cols != K + nS) return W4A4_ERR_INVALID_ARG;
+    if (M == 0) return W4A4_OK;
+    if (!X) return W4A4_ERR_INVALID_ARG;
+    if (!aligned16(X) || ldx % 8) return W4A4_ERR_MISALIGNED;
+    rc = device_check(nullptr);
+    if (rc != W4A4_OK) return rc;
+    ResidualArgs r{X, M, K, ldx, pad128(M), S, nS, static_cast<uint8_t*>(Xaug->codes), Xaug->cols / 2,
+                   static_cast<uint8_t*>(Xaug->scales), Xaug->cols / 16 / 4, Xaug->s2, Xaug->scale_mode};
+    return cuda_status(launch_residual(r, as_stream(stream)));
+}
+
+int w4a4_select_channels(const uint16_t* Xcal, int Mc, int K, int ldx, int nS, int32_t* S_out, void* ws,
+                         size_t ws_bytes, void* stream) {
+    if (Mc < 1 || K < 1 || ldx < K || nS < 0 || nS > K || !Xcal || (nS > 0 && !S_out)) return W4A4_ERR_INVALID_ARG;
+    if (!ws || ws_bytes < (size_t)K * 8) return W4A4_ERR_WORKSPACE;
+    if (reinterpret_cast<uintptr_t>(ws) & 15) return W4A4_ERR_MISALIGNED;
+    int rc = device_check(nullptr);
+    if (rc != W4A4_OK) return rc;
+    if (nS == 0) return W4A4_OK;
+    float* amax = static_cast<float*>(ws);
+    int* sel = reinterpret_cast<int*>(static_cast<uint8_t*>(ws) + (size_t)K * 4);
+    return cuda_status(launch_select(Xcal, Mc, K, ldx, nS, S_out, amax, sel, as_stream(stream)));
+}
+
+int w4a4_device_status(void* stream) {
+    if (cudaStreamSynchronize(as_stream(stream)) != cudaSuccess) return W4A4_ERR_CUDA;
+    int v = 0;
+    if (cudaMemcpyFromSymbol(&v, g_error_word, sizeof(int)) != cudaSuccess) return W4A4_ERR_CUDA;
+    if (v != 0) {
+        const int zero = 0;
+        if (cudaMemcpyToSymbol(g_error_word, &zero, sizeof(int)) != cudaSuccess) return W4A4_ERR_CUDA;
+        return v == kErrTimeout ? W4A4_ERR_DEVICE_TIMEOUT : v == kErrBadIndex ? W4A4_ERR_INVALID_ARG : W4A4_ERR_CUDA;
+    }
+    return W4A4_OK;
+}
+
+void w4a4_debug_set(int skip_k_tile, unsigned long long wait_limit_ns) {
+    g_skip_k_tile = skip_k_tile < 0 ? -1 : skip_k_tile;
+    g_wait_limit_ns = wait_limit_ns ? wait_limit_ns : 2000000000ull;
+}
+
+}  // extern "C"

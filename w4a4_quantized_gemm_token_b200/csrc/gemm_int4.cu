@@ -1,0 +1,264 @@
+// INT4-g128 W4A4 GEMM on the sm_100a 8-bit integer MMA (tcgen05.mma kind::i8).
+//
+// sm_100's tensor cores have no 4-bit integer kind, so the packed nibbles are
+// widened to int8 in shared memory.  Per 128-element K group g the MMA
+// produces the exact int32 partial sum P_g[m,n] = sum_{k in g} qa qw into one
+// of two TMEM buffers; CUDA-core warps rescale it,
+//     acc[m,n] += float(P_g[m,n]) * (sa[m,g] * sw[n,g])    (FP32),
+// and at the end round acc to bf16.  This per-group rescale on the CUDA cores
+// is the cost the APEX4 paragraph ("Depth Registers..." thelatestinai page,
+// para 2) analyses through the tensor-core / CUDA-core throughput ratio.
+//
+// One CTA per 128 x 128 output tile, 14 warps:
+//   warp 0 lane 0   TMA producer: packed codes of A and B (64-byte rows).
+//   warp 1          TMEM owner; lane 0 issues 4 MMAs (K=32) per group.
+//   warps 2..5      unpack: nibbles -> int8, written in the 128-byte swizzled
+//                   K-major layout the MMA reads.
+//   warps 6..13     rescale + epilogue: warp w reads TMEM lane quarter w%4,
+//                   columns [64*((w-6)/4), +64).
+#include <cstdint>
+#include <cuda_bf16.h>
+
+#include "kernels.h"
+#include "ptx.cuh"
+
+namespace w4a4 {
+
+namespace i4 {
+constexpr int STAGES = 4;
+constexpr int PK_BYTES = 128 * 64;      // packed 128 rows x 128 nibbles
+constexpr int UN_BYTES = 128 * 128;     // unpacked 128 rows x 128 int8
+constexpr int STAGE = 2 * UN_BYTES + 2 * PK_BYTES;  // unpacked A, B, then packed A, B
+constexpr int SB_OFF = STAGES * STAGE;              // 2 x 128 floats of B scales
+constexpr int BAR_OFF = SB_OFF + 2 * 128 * 4;
+constexpr int SMEM = BAR_OFF + 512 + 1024;
+constexpr int THREADS = 14 * 32;
+constexpr int TMEM_COLS = 256;                      // two int32 buffers of 128 columns
+}  // namespace i4
+
+// Sign-extend the 8 nibbles of w (element i in nibble i) into 8 int8 bytes,
+// returned as two words (elements 0-3, 4-7).
+__device__ __forceinline__ void widen8(uint32_t w, uint32_t& o0, uint32_t& o1) {
+    uint32_t lo = w & 0x0F0F0F0Fu;          // elements 0,2,4,6
+    uint32_t hi = (w >> 4) & 0x0F0F0F0Fu;   // elements 1,3,5,7
+    // per byte: n in [0,15] -> ((n ^ 8) + 0x78) ^ 0x80 = n - 16*(n >= 8), no carries between bytes
+    lo = ((lo ^ 0x08080808u) + 0x78787878u) ^ 0x80808080u;
+    hi = ((hi ^ 0x08080808u) + 0x78787878u) ^ 0x80808080u;
+    o0 = __byte_perm(lo, hi, 0x5140);  // e0 e1 e2 e3
+    o1 = __byte_perm(lo, hi, 0x7362);  // e4 e5 e6 e7
+}
+
+__device__ __forceinline__ void named_bar(int id, int n) { asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory"); }
+
+__global__ void __launch_bounds__(i4::THREADS, 1)
+    gemm_int4_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB, GemmArgs g) {
+    using namespace i4;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    float* sb_smem = reinterpret_cast<float*>(smem + SB_OFF);
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem + BAR_OFF);
+    uint64_t* conv = full + STAGES;
+    uint64_t* empty = conv + STAGES;
+    uint64_t* accf = empty + STAGES;    // [2]
+    uint64_t* tfree = accf + 2;         // [2]
+    uint64_t* drain = tfree + 2;
+    uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(drain + 1);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int G = g.K / 128;
+    const uint64_t limit = g.wait_limit_ns;
+    // grouped raster over (m tile, n tile)
+    const int num_m = (g.M + 127) / 128, num_n = (g.N + kBN_I4 - 1) / kBN_I4;
+    const int GR = 8, per_group = GR * num_n;
+    const int grp = blockIdx.x / per_group, first = grp * GR, gsz = min(GR, num_m - first);
+    const int in = blockIdx.x - grp * per_group;
+    const int m_tile = first + in % gsz, n_tile = in / gsz;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < STAGES; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&conv[s], 4);
+            mbar_init(&empty[s], 1);
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&accf[b], 1);
+            mbar_init(&tfree[b], 8);
+        }
+        mbar_init(drain, 1);
+        *abort_flag = 0;
+        fence_mbar_init();
+    }
+    if (warp == 0 && lane == 0) {
+        tma_prefetch_desc(&tmA);
+        tma_prefetch_desc(&tmB);
+    }
+    if (warp == 1) {
+        tmem_alloc(tmem_holder, TMEM_COLS);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_holder;
+    pdl_wait();
+
+    if (warp == 0) {
+        if (lane == 0) {
+            int gi = 0;
+            for (; gi < G; ++gi) {
+                const int s = gi % STAGES, n = gi / STAGES;
+                if (gi >= STAGES && !mbar_wait(&empty[s], (n - 1) & 1, limit, abort_flag)) break;
+                if (gi == g.skip_k_tile) continue;
+                uint8_t* st = smem + s * STAGE;
+                mbar_arrive_expect_tx(&full[s], 2 * PK_BYTES);
+                tma_load_2d(st + 2 * UN_BYTES, &tmA, gi * 64, m_tile * 128, &full[s]);
+                tma_load_2d(st + 2 * UN_BYTES + PK_BYTES, &tmB, gi * 64, n_tile * kBN_I4, &full[s]);
+            }
+            if (*abort_flag)
+                for (int j = max(0, gi - STAGES); j < gi; ++j)
+                    if (j != g.skip_k_tile) {
+                        const uint64_t t0 = globaltimer();
+                        while (!mbar_try_wait(&full[j % STAGES], (j / STAGES) & 1) && globaltimer() - t0 < 100000000ull) {
+                        }
+                    }
+        }
+    } else if (warp == 1) {
+        if (lane == 0) {
+            bool ok = true;
+            for (int gi = 0; gi < G; ++gi) {
+                const int s = gi % STAGES, n = gi / STAGES, buf = gi & 1;
+                if (!mbar_wait(&conv[s], n & 1, limit, abort_flag)) { ok = false; break; }
+                if (gi >= 2 && !mbar_wait(&tfree[buf], ((gi >> 1) - 1) & 1, limit, abort_flag)) { ok = false; break; }
+                tc_fence_after();
+                const uint32_t sA = smem_u32(smem + s * STAGE), sB = sA + UN_BYTES;
+#pragma unroll
+                for (int j = 0; j < 4; ++j)
+                    mma_i8(tmem + buf * 128, desc_kmajor_sw128(sA + 32 * j), desc_kmajor_sw128(sB + 32 * j),
+                           idesc_i8(128, kBN_I4), j > 0 ? 1u : 0u);
+                tc_commit(&empty[s]);
+                tc_commit(&accf[buf]);
+            }
+            if (!ok) {
+                tc_commit(drain);
+                const uint64_t t0 = globaltimer();
+                while (!mbar_try_wait(drain, 0) && globaltimer() - t0 < 100000000ull) {
+                }
+            }
+        }
+    } else if (warp < 6) {
+        // ------------------------------ unpack ------------------------------
+        const int uw = warp - 2;  // 0..3
+        for (int gi = 0; gi < G; ++gi) {
+            const int s = gi % STAGES, n = gi / STAGES;
+            if (!mbar_wait(&full[s], n & 1, limit, abort_flag)) break;
+            uint8_t* st = smem + s * STAGE;
+            // each warp pass: 8 rows x 64 packed bytes; lane -> row r0 + lane/4, segment lane%4
+#pragma unroll
+            for (int op = 0; op < 2; ++op) {  // A then B
+                const uint8_t* pk = st + 2 * UN_BYTES + op * PK_BYTES;
+                uint8_t* un = st + op * UN_BYTES;
+#pragma unroll
+                for (int pass = 0; pass < 4; ++pass) {
+                    const int row = (uw * 4 + pass) * 8 + (lane >> 2);
+                    const int seg = lane & 3;
+                    const uint4 w = *reinterpret_cast<const uint4*>(pk + row * 64 + seg * 16);
+                    uint32_t o[8];
+                    widen8(w.x, o[0], o[1]);
+                    widen8(w.y, o[2], o[3]);
+                    widen8(w.z, o[4], o[5]);
+                    widen8(w.w, o[6], o[7]);
+                    // 16-byte chunk c of the 128-byte row lands at chunk c ^ (row % 8)
+                    const int c0 = 2 * seg, c1 = 2 * seg + 1;
+                    *reinterpret_cast<uint4*>(un + row * 128 + ((c0 ^ (row & 7)) << 4)) = make_uint4(o[0], o[1], o[2], o[3]);
+                    *reinterpret_cast<uint4*>(un + row * 128 + ((c1 ^ (row & 7)) << 4)) = make_uint4(o[4], o[5], o[6], o[7]);
+                }
+            }
+            fence_proxy_async_smem();  // generic-proxy writes -> visible to the tensor core
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&conv[s]);
+        }
+    } else {
+        // ------------------------------ rescale + epilogue ------------------------------
+        const int q = warp & 3, half = (warp - 6) >> 2;
+        const int rt = (warp - 6) * 32 + lane;  // 0..255
+        const int row = q * 32 + lane;
+        const int m = m_tile * 128 + row;
+        const int ncol0 = n_tile * kBN_I4 + 64 * half;
+        const float* sfa = reinterpret_cast<const float*>(g.sfa);
+        const float* sfb = reinterpret_cast<const float*>(g.sfb);
+        float acc[64];
+#pragma unroll
+        for (int i = 0; i < 64; ++i) acc[i] = 0.0f;
+        // After a failed wait the loop keeps running (without waiting or reading
+        // TMEM) so that every rescale thread passes the same named barriers.
+        bool ok = true;
+        for (int gi = 0; gi < G; ++gi) {
+            const int buf = gi & 1;
+            float* sbb = sb_smem + buf * 128;
+            if (rt < 128) sbb[rt] = sfb[(size_t)gi * g.sfb_ld + n_tile * kBN_I4 + rt];
+            const float sa = sfa[(size_t)gi * g.sfa_ld + min(m, g.sfa_ld - 1)];
+            named_bar(1, 256);
+            if (ok) ok = mbar_wait(&accf[buf], (gi >> 1) & 1, limit, abort_flag);
+            if (!ok) continue;
+            tc_fence_after();
+#pragma unroll
+            for (int ch = 0; ch < 2; ++ch) {
+                uint32_t r[32];
+                tmem_ld_32x32b_x32(tmem + ((uint32_t)(q * 32) << 16) + buf * 128 + 64 * half + 32 * ch, r);
+                tmem_ld_wait();
+#pragma unroll
+                for (int i = 0; i < 32; ++i) {
+                    const float sc = __fmul_rn(sa, sbb[64 * half + 32 * ch + i]);
+                    acc[32 * ch + i] = __fmaf_rn(__int2float_rn((int)r[i]), sc, acc[32 * ch + i]);
+                }
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&tfree[buf]);
+        }
+        if (ok && m < g.M && ncol0 < g.N) {
+            uint16_t* dst = g.Y + (size_t)m * g.ldy + ncol0;
+#pragma unroll
+            for (int v = 0; v < 8; ++v) {
+                uint32_t pk[4];
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    __nv_bfloat162 h = __floats2bfloat162_rn(acc[8 * v + 2 * e], acc[8 * v + 2 * e + 1]);
+                    pk[e] = *reinterpret_cast<uint32_t*>(&h);
+                }
+                *reinterpret_cast<uint4*>(dst + 8 * v) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+            }
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem, i4::TMEM_COLS);
+    }
+}
+
+cudaError_t launch_gemm_int4(const CUtensorMap& tmA, const CUtensorMap& tmB, const GemmArgs& g, int /*num_sms*/,
+                             bool pdl, cudaStream_t st) {
+    static bool attr_set = false;
+    if (!attr_set) {
+        cudaError_t e = cudaFuncSetAttribute(gemm_int4_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, i4::SMEM);
+        if (e != cudaSuccess) return e;
+        attr_set = true;
+    }
+    const int tiles = ((g.M + 127) / 128) * ((g.N + kBN_I4 - 1) / kBN_I4);
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(tiles);
+    cfg.blockDim = dim3(i4::THREADS);
+    cfg.dynamicSmemBytes = i4::SMEM;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = pdl ? 1 : 0;
+    return cudaLaunchKernelEx(&cfg, gemm_int4_kernel, tmA, tmB, g);
+}
+
+}  // namespace w4a4

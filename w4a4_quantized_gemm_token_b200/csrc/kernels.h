@@ -1,0 +1,90 @@
+// Internal interface between the C-ABI layer (api.cu) and the kernels.
+#pragma once
+#include <cstddef>
+#include <cstdint>
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+namespace w4a4 {
+
+enum { FMT_NVFP4 = 0, FMT_MXFP4 = 1, FMT_INT4 = 2 };
+
+struct QuantArgs {
+    const uint16_t* X;       // bf16 [rows][ldx]
+    int M;                   // live rows
+    int K;                   // columns to quantize (chunks of 16)
+    int K_src;               // gather: columns >= K_src come from S (weights only)
+    int ldx;
+    const int32_t* S;        // gather map (weights only)
+    uint8_t* codes;          // [M][ldc]
+    int ldc;                 // bytes per codes row (= cols/2)
+    uint8_t* sf;             // NVFP4/MXFP4 scales, MMA layout
+    int sf_col_atoms;        // (cols / group) / 4
+    float* sfi;              // INT4 scales [cols/128][sfi_ld]
+    int sfi_ld;              // pad128(rows)
+    int mode;                // NVFP4: 0 tensor, 1 token
+    const float* static_s2;  // nullable
+    float* s2_out;           // NVFP4 s2 ([1] or [M])
+    const float* tensor_amax;  // NVFP4 tensor mode without static s2
+};
+
+struct ResidualArgs {
+    const uint16_t* X;
+    int M, K, ldx, rows_pad;
+    const int32_t* S;
+    int nS;
+    uint8_t* codes;  // augmented codes [M][ldc]
+    int ldc;
+    uint8_t* sf;     // augmented scales, MMA layout
+    int sf_col_atoms;
+    const float* s2;
+    int mode;
+};
+
+struct GemmArgs {
+    int M, N, K;               // K = quantized columns (augmented included)
+    const uint8_t* sfa;        // FP4 scales of A (MMA layout) / INT4: float [K/128][lda_s]
+    const uint8_t* sfb;
+    int sf_col_atoms;          // FP4: (K/group)/4
+    int sfa_ld, sfb_ld;        // INT4: pad128(M), pad128(N)
+    const float* s2a;          // NVFP4 alpha parts (nullable for MXFP4)
+    int s2a_per_row;
+    const float* s2b;
+    uint16_t* Y;
+    int ldy;
+    float* partial;            // split-K partial sums (decode variant)
+    int splits;                // split-K factor (decode variant)
+    int k_tiles_per_split;
+    int skip_k_tile;           // debug: never load this k-tile (-1 = off)
+    unsigned long long wait_limit_ns;
+};
+
+cudaError_t launch_quant(int fmt, bool gather, const QuantArgs& a, int rows_pad, cudaStream_t st);
+cudaError_t launch_amax(const uint16_t* X, int M, int K, int ldx, float* out, int num_sms, cudaStream_t st);
+cudaError_t launch_residual(const ResidualArgs& a, cudaStream_t st);
+cudaError_t launch_select(const uint16_t* X, int Mc, int K, int ldx, int nS, int32_t* S, float* amax, int* sel,
+                          cudaStream_t st);
+
+// FP4 block-scaled GEMM (NVFP4 when nvfp4, else MXFP4).  tmA/tmB: byte tensor
+// maps of the codes with a 128-byte swizzle and boxes of 128 x 128 (A) and
+// 128 x bn (B) bytes.  pdl: launched as a programmatic dependent.
+cudaError_t launch_gemm_fp4(bool nvfp4, const CUtensorMap& tmA, const CUtensorMap& tmB, const GemmArgs& g,
+                            int num_sms, bool pdl, cudaStream_t st);
+// Small-M variant: weights take the MMA's M side (128 rows per tile), the
+// tokens its N side (16), K is split across CTAs; FP32 partial sums go to
+// g.partial [splits][M][N] and a second kernel reduces them into Y.
+cudaError_t launch_gemm_fp4_decode(bool nvfp4, const CUtensorMap& tmW, const CUtensorMap& tmX, const GemmArgs& g,
+                                   bool pdl, cudaStream_t st);
+// INT4-g128 GEMM on the 8-bit integer MMA with per-group FP32 rescaling.
+cudaError_t launch_gemm_int4(const CUtensorMap& tmA, const CUtensorMap& tmB, const GemmArgs& g, int num_sms,
+                             bool pdl, cudaStream_t st);
+
+// Tile shapes (shared with the host-side tensor-map set-up).
+constexpr int kBM = 128;          // rows of A per tile
+constexpr int kBN = 256;          // rows of B per tile (FP4)
+constexpr int kBK_FP4 = 256;      // K elements per pipeline stage (128 bytes of codes)
+constexpr int kBN_DEC = 16;       // token tile of the decode variant
+constexpr int kBN_I4 = 128;       // rows of B per tile (INT4)
+constexpr int kBK_I4 = 128;       // K elements per stage (one INT4 group)
+
+}  // namespace w4a4

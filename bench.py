@@ -1,0 +1,448 @@
+"""Benchmark of the W4A4 quantized linear layer on B200.
+
+One step = the five linears of one Llama-2-70B decoder layer (qkv 8192->10240,
+o 8192->8192, w1/w3 8192->28672, w2 28672->8192) at M tokens, each a fused
+W4A4 linear: per-token NVFP4 quantization of the bf16 activations followed by
+the block-scaled NVFP4 GEMM against NVFP4 weights quantized once beforehand.
+Metric: TFLOPS (2*M*N*K summed over the layer / time), whole job.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+With N > 1 (launched by torchrun) every rank runs its own replica on its own
+tokens ("weak" scaling, no collective).  Also measured in the same run and
+reported under "rows": the activation quantizer (GB/s), the small-M decode
+variant (GB/s), the INT4-g128 path (Qwen2.5-7B shapes, TOPS), the residual
+augmentation (Qwen2.5-3B shapes) and MXFP4.  `--impl reference` times the C
+oracle on the host cores on a bounded sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from w4a4_quantized_gemm_token_b200 import synth  # noqa: E402
+
+LLAMA = synth.SHAPES["llama2_70b"]
+PEAKS_FILE = os.path.join(ROOT, "MEASURED_PEAKS.json")
+FP4_PER_BF16 = 4.0        # nominal dense FP4 / BF16 tensor throughput (9 / 2.25 PFLOP/s)
+INT8_PER_BF16 = 2.0       # nominal dense INT8 / BF16 (4.5 / 2.25)
+
+
+def peaks():
+    try:
+        p = json.load(open(PEAKS_FILE))
+        return {"hbm": float(p["hbm_gbs"]), "bf16": float(p["bf16_tflops"]),
+                "bf16_sustained": float(p.get("bf16_tflops_sustained", p["bf16_tflops"])), "src": "measured"}
+    except Exception:
+        return {"hbm": 6650.0, "bf16": 1590.0, "bf16_sustained": 1400.0, "src": "fallback"}
+
+
+# ----------------------------------------------------------------------------------------------
+# clocks sampled during the timed region
+# ----------------------------------------------------------------------------------------------
+class ClockSampler:
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        try:
+            fd, self.path = tempfile.mkstemp(suffix=".csv")
+            os.close(fd)
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.index), "--query-gpu=" + self.QUERY,
+                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                         stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        rows = []
+        for line in open(self.path):
+            f = [x.strip() for x in line.split(",")]
+            if len(f) >= 9:
+                rows.append(f)
+        os.unlink(self.path)
+        if not rows:
+            return None
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].lower() == "active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": reasons, "samples": len(rows)}
+
+
+# ----------------------------------------------------------------------------------------------
+# the reference arm and the CPU baseline: the oracle on a bounded sample
+# ----------------------------------------------------------------------------------------------
+_ORACLE_W = {}
+
+
+def oracle_sample(M_rows: int, n_cols: int):
+    """Time the C oracle (as it stands, one host thread) on the layer's five
+    linears for `M_rows` tokens and the first `n_cols` output columns of each:
+    per-token NVFP4 quantization of those rows plus the exact block-scaled GEMM.
+    The weights' quantization is offline on both arms and is not timed.
+    Returns (TFLOPS, seconds, flops)."""
+    import oracle
+    oracle.build()
+    t_total, flops = 0.0, 0.0
+    for li, (name, K, N) in enumerate(LLAMA):
+        n = min(N, n_cols)
+        key = (li, n)
+        if key not in _ORACLE_W:
+            W = synth.weights("llama2_70b", N, K, seed=0, tensor_id=100 + li)[:n]
+            _ORACLE_W[key] = oracle.quant_nvfp4(W, mode=0)
+        cw, sw, s2w = _ORACLE_W[key]
+        X = synth.activations("llama2_70b", M_rows, K, seed=0, tensor_id=200 + li)
+        t0 = time.perf_counter()
+        ca, sa, s2a = oracle.quant_nvfp4(X, mode=1)
+        oracle.gemm_nvfp4(ca, sa, s2a, 1, cw, sw, s2w, want_ref=False)
+        t_total += time.perf_counter() - t0
+        flops += 2.0 * M_rows * n * K
+    return flops / t_total / 1e12, t_total, flops
+
+
+def run_reference(args, rank, world):
+    if rank != 0:
+        return
+    K, W = args.steps, args.warmup
+    rows, cols = args.ref_rows, args.ref_cols
+    for _ in range(W):
+        oracle_sample(1, cols)
+    vals, secs = [], []
+    for _ in range(K):
+        v, s, _ = oracle_sample(rows, cols)
+        vals.append(v)
+        secs.append(s)
+    value = statistics.median(vals)
+    line = {
+        "impl": "reference", "metric": "W4A4 linear TFLOPS (Llama-2-70B layer, NVFP4 per-token)",
+        "value": value, "unit": "TFLOPS", "n_gpus": world, "steps": K, "warmup": W,
+        "ms_per_step": statistics.median(secs) * 1e3, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "nvfp4", "data": "synthetic",
+        "config": {"workload": f"llama2_70b layer linears (qkv,o,w1,w3,w2), oracle on {rows} tokens x "
+                               f"{cols} output columns per linear per step", "tokens": rows},
+        "cpu_baseline": {"value": value, "unit": "TFLOPS", "cores": 1, "kind": "oracle",
+                         "sample": f"{rows} tokens x {cols} output columns of each of the 5 layer linears "
+                                   f"(full K), one host thread"},
+        "e2e": {"value": value, "unit": "TFLOPS", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+# ----------------------------------------------------------------------------------------------
+# our arm
+# ----------------------------------------------------------------------------------------------
+def to_dev(bits, device):
+    import torch
+    return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).to(device).view(torch.bfloat16)
+
+
+def time_loop(fn, iters, stream):
+    """Average device time (ms) of fn() over iters launches, CUDA events on `stream`."""
+    import torch
+    s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    s.record(stream)
+    for _ in range(iters):
+        fn()
+    e.record(stream)
+    e.synchronize()
+    return s.elapsed_time(e) / iters
+
+
+def run_ours(args, rank, world):
+    import torch
+    import torch.distributed as dist
+    import w4a4_quantized_gemm_token_b200 as w4
+
+    dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", 0)))
+    torch.cuda.set_device(dev)
+    stream = torch.cuda.current_stream()
+    P = peaks()
+    fp4_peak = P["bf16"] * FP4_PER_BF16
+    M = args.tokens
+
+    # ---- workload: Llama-2-70B layer linears, NVFP4 weights quantized once ----
+    layers = []
+    for li, (name, K, N) in enumerate(LLAMA):
+        Wd = to_dev(synth.weights("llama2_70b", N, K, seed=0, tensor_id=100 + li), dev)
+        Wq = w4.quantize_weight(Wd, w4.NVFP4)
+        del Wd
+        X = to_dev(synth.activations("llama2_70b", M, K, seed=rank, tensor_id=200 + li), dev)
+        Y = torch.empty(M, N, dtype=torch.bfloat16, device=dev)
+        ws = torch.empty(w4.linear_workspace(M, N, K, w4.NVFP4), dtype=torch.uint8, device=dev)
+        layers.append((name, K, N, Wq, X, Y, ws))
+    torch.cuda.synchronize()
+    flops_step = sum(2.0 * M * N * K for (_, K, N, *_r) in layers)
+
+    def step():
+        for (_, K, N, Wq, X, Y, ws) in layers:
+            w4.linear(X, Wq, w4.SCALE_TOKEN, Y=Y, ws=ws)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    assert w4.device_status() == w4.OK
+
+    sampler = ClockSampler(dev.index)
+    sampler.start()
+    time.sleep(0.3)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    ev0.record(stream)
+    for _ in range(args.steps):
+        step()
+    ev1.record(stream)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    clocks = sampler.stop()
+    ms = ev0.elapsed_time(ev1) / args.steps
+    if world > 1:
+        t = torch.tensor([ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+    value = flops_step * world / (ms * 1e-3) / 1e12
+    assert w4.device_status() == w4.OK
+    launches = 2 * len(layers) * args.steps
+
+    # ---- end to end through the public API with host buffers ----
+    hX = [torch.empty(X.shape, dtype=torch.bfloat16, pin_memory=True) for (_, _, _, _, X, _, _) in layers]
+    hY = [torch.empty(Y.shape, dtype=torch.bfloat16, pin_memory=True) for (_, _, _, _, _, Y, _) in layers]
+    for h, (_, _, _, _, X, _, _) in zip(hX, layers):
+        h.copy_(X)
+    h2d = sum(h.numel() * 2 for h in hX)
+    d2h = sum(h.numel() * 2 for h in hY)
+
+    def e2e_step():
+        for i, (_, K, N, Wq, X, Y, ws) in enumerate(layers):
+            X.copy_(hX[i], non_blocking=True)
+            w4.linear(X, Wq, w4.SCALE_TOKEN, Y=Y, ws=ws)
+            hY[i].copy_(Y, non_blocking=True)
+
+    e2e_iters = max(3, min(args.steps, 10))
+    e2e_step()
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    e2e_ms = time_loop(e2e_step, e2e_iters, stream)
+    if world > 1:
+        t = torch.tensor([e2e_ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+    e2e_value = flops_step * world / (e2e_ms * 1e-3) / 1e12
+
+    # ---- dominant kernel: the block-scaled GEMM alone, per shape ----
+    gemm_ms, gemm_flops = 0.0, 0.0
+    per_shape = {}
+    for (name, K, N, Wq, X, Y, ws) in layers:
+        Xq = w4.quantize_act(X, w4.NVFP4, w4.SCALE_TOKEN)
+        w4.gemm(Xq, Wq, Y)
+        t_ms = time_loop(lambda: w4.gemm(Xq, Wq, Y), max(5, args.steps), stream)
+        f = 2.0 * M * N * K
+        per_shape[name] = round(f / (t_ms * 1e-3) / 1e12, 1)
+        gemm_ms += t_ms
+        gemm_flops += f
+        del Xq
+    gemm_tflops = gemm_flops / (gemm_ms * 1e-3) / 1e12
+    roofline = {"bound": "tensor", "achieved": round(gemm_tflops, 1), "peak": round(fp4_peak, 1),
+                "unit": "TFLOP/s", "frac": round(gemm_tflops / fp4_peak, 4), "traffic": None,
+                "peak_src": f"{P['src']} bf16 burst x {FP4_PER_BF16:g} (nominal fp4/bf16)",
+                "kernel": "gemm_fp4_kernel (NVFP4, 128x256 tile)", "per_shape_tflops": per_shape}
+
+    rows = {} if args.no_rows else extra_rows(args, dev, stream, P)
+
+    if rank == 0:
+        line = {
+            "metric": "W4A4 linear TFLOPS (Llama-2-70B layer, NVFP4 per-token)",
+            "value": round(value, 2), "unit": "TFLOPS", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": round(ms, 4), "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "nvfp4", "data": "synthetic",
+            "config": {"workload": f"llama2_70b layer linears (qkv,o,w1,w3,w2), fused per-token NVFP4 "
+                                   f"W4A4 linear, M={M} tokens per GPU",
+                       "tokens_per_gpu": M, "l2": "inputs larger than L2 (0.47 GB of weights per step)",
+                       "parallelism": f"replicas x{world}"},
+            "frac_of_fp4_peak": round(value / world / fp4_peak, 4),
+            "roofline": roofline,
+            "e2e": {"value": round(e2e_value, 3), "unit": "TFLOPS", "h2d_bytes_per_step": h2d,
+                    "d2h_bytes_per_step": d2h},
+            "gpu_launches": launches,
+            "clocks": clocks,
+            "rows": rows,
+        }
+        if world == 1 and not args.no_cpu:
+            v, s, f = oracle_sample(args.cpu_rows, args.cpu_cols)
+            line["cpu_baseline"] = {"value": v, "unit": "TFLOPS", "cores": 1, "kind": "oracle",
+                                    "sample": f"{args.cpu_rows} tokens x {args.cpu_cols} output columns of each "
+                                              f"of the 5 layer linears (full K), one host thread, {s:.1f} s"}
+        print(json.dumps(line), flush=True)
+
+
+def extra_rows(args, dev, stream, P):
+    """The other hot-path rows, each timed with CUDA events on the launching stream."""
+    import torch
+    import w4a4_quantized_gemm_token_b200 as w4
+    out = {}
+    hbm = P["hbm"]
+    it = max(5, args.steps)
+
+    # activation quantizer, per-token NVFP4 (and MXFP4 / INT4), Llama qkv and w2 inputs
+    for (name, M, K) in [("qkv_in", args.tokens, 8192), ("w2_in", args.tokens, 28672)]:
+        X = to_dev(synth.activations("llama2_70b", M, K, seed=3), dev)
+        for fmt, g, sb in [(w4.NVFP4, 16, 1), (w4.MXFP4, 32, 1), (w4.INT4, 128, 4)]:
+            q = w4.QTensor(fmt, M, K, w4.SCALE_TOKEN if fmt == w4.NVFP4 else 0, dev)
+            f = lambda: w4.quantize_act(X, fmt, w4.SCALE_TOKEN, out=q)
+            f()
+            ms = time_loop(f, it, stream)
+            byts = 2 * M * K + M * K / 2 + M * K / g * sb + (4 * M if fmt == w4.NVFP4 else 0)
+            key = {w4.NVFP4: "nvfp4_token", w4.MXFP4: "mxfp4", w4.INT4: "int4"}[fmt]
+            out[f"quant_{key}_{name}"] = {"GB/s": round(byts / ms / 1e6, 1), "frac_hbm": round(byts / ms / 1e6 / hbm, 3),
+                                          "us": round(ms * 1e3, 2)}
+        q = w4.QTensor(w4.NVFP4, M, K, w4.SCALE_TENSOR, dev)
+        f = lambda: w4.quantize_act(X, w4.NVFP4, w4.SCALE_TENSOR, out=q)
+        f()
+        ms = time_loop(f, it, stream)
+        byts = 4 * M * K + M * K / 2 + M * K / 16
+        out[f"quant_nvfp4_tensor_2pass_{name}"] = {"GB/s": round(byts / ms / 1e6, 1), "us": round(ms * 1e3, 2)}
+        del X
+
+    # decode: M = 1 and 16 over the layer (weights streamed from HBM)
+    Ws = []
+    for li, (name, K, N) in enumerate(LLAMA):
+        Wd = to_dev(synth.weights("llama2_70b", N, K, seed=0, tensor_id=100 + li), dev)
+        Ws.append((K, N, w4.quantize_weight(Wd, w4.NVFP4)))
+        del Wd
+    for Md in (1, 16):
+        bufs = []
+        for (K, N, Wq) in Ws:
+            X = to_dev(synth.activations("llama2_70b", Md, K, seed=5), dev)
+            Y = torch.empty(Md, N, dtype=torch.bfloat16, device=dev)
+            ws = torch.empty(w4.linear_workspace(Md, N, K, w4.NVFP4), dtype=torch.uint8, device=dev)
+            bufs.append((X, Wq, Y, ws))
+
+        def dec():
+            for (X, Wq, Y, ws) in bufs:
+                w4.linear(X, Wq, w4.SCALE_TOKEN, Y=Y, ws=ws)
+        dec()
+        ms = time_loop(dec, it, stream)
+        byts = sum(N * K * 0.5625 + 2 * Md * K + 2 * Md * N for (K, N, _) in Ws)
+        out[f"decode_m{Md}_llama_layer"] = {"GB/s": round(byts / ms / 1e6, 1), "frac_hbm": round(byts / ms / 1e6 / hbm, 3),
+                                            "us": round(ms * 1e3, 2)}
+    del Ws
+
+    # INT4-g128, Qwen2.5-7B shapes at M = 2048
+    tot_ms, tot_ops = 0.0, 0.0
+    for li, (name, K, N) in enumerate(synth.SHAPES["qwen25_7b_int4"]):
+        M = 2048
+        Wq = w4.quantize_weight(to_dev(synth.weights("qwen25_7b_int4", N, K, tensor_id=300 + li), dev), w4.INT4)
+        X = to_dev(synth.activations("qwen25_7b_int4", M, K), dev)
+        Y = torch.empty(M, N, dtype=torch.bfloat16, device=dev)
+        ws = torch.empty(w4.linear_workspace(M, N, K, w4.INT4), dtype=torch.uint8, device=dev)
+        f = lambda: w4.linear(X, Wq, 0, Y=Y, ws=ws)
+        f()
+        ms = time_loop(f, it, stream)
+        tot_ms += ms
+        tot_ops += 2.0 * M * N * K
+    i8_peak = P["bf16"] * INT8_PER_BF16
+    v = tot_ops / (tot_ms * 1e-3) / 1e12
+    out["int4_g128_qwen25_7b_m2048"] = {"TOPS": round(v, 1), "frac_int8_peak": round(v / i8_peak, 3)}
+
+    # dual-stage residual augmentation, Qwen2.5-3B shapes at M = 8192
+    tot_ms, tot_f, tot_fk = 0.0, 0.0, 0.0
+    for li, (name, K, N) in enumerate(synth.SHAPES["qwen25_3b_aug"]):
+        M, nS = 8192, 256
+        Xc = to_dev(synth.calibration("qwen25_3b_aug", K), dev)
+        S = w4.select_channels(Xc, nS)
+        Wq = w4.quantize_weight(to_dev(synth.weights("qwen25_3b_aug", N, K, tensor_id=400 + li), dev), w4.NVFP4, S=S)
+        X = to_dev(synth.activations("qwen25_3b_aug", M, K), dev)
+        Y = torch.empty(M, N, dtype=torch.bfloat16, device=dev)
+        ws = torch.empty(w4.linear_workspace(M, N, K, w4.NVFP4, nS), dtype=torch.uint8, device=dev)
+        f = lambda: w4.linear(X, Wq, w4.SCALE_TOKEN, S=S, Y=Y, ws=ws)
+        f()
+        ms = time_loop(f, it, stream)
+        tot_ms += ms
+        tot_f += 2.0 * M * N * (K + nS)
+        tot_fk += 2.0 * M * N * K
+    out["aug_nvfp4_qwen25_3b_m8192"] = {"TFLOPS_exec": round(tot_f / (tot_ms * 1e-3) / 1e12, 1),
+                                        "TFLOPS_effective_K": round(tot_fk / (tot_ms * 1e-3) / 1e12, 1)}
+
+    # MXFP4 GEMM on the Llama qkv shape, M = 4096
+    K, N, M = 8192, 10240, args.tokens
+    Wq = w4.quantize_weight(to_dev(synth.weights("llama2_70b", N, K, tensor_id=100), dev), w4.MXFP4)
+    X = to_dev(synth.activations("llama2_70b", M, K), dev)
+    Y = torch.empty(M, N, dtype=torch.bfloat16, device=dev)
+    ws = torch.empty(w4.linear_workspace(M, N, K, w4.MXFP4), dtype=torch.uint8, device=dev)
+    f = lambda: w4.linear(X, Wq, 0, Y=Y, ws=ws)
+    f()
+    ms = time_loop(f, it, stream)
+    out["mxfp4_linear_llama_qkv"] = {"TFLOPS": round(2.0 * M * N * K / (ms * 1e-3) / 1e12, 1)}
+    torch.cuda.synchronize()
+    assert w4.device_status() == w4.OK
+    return out
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--tokens", type=int, default=4096)
+    ap.add_argument("--ref-rows", type=int, default=2, help="reference arm: tokens per step")
+    ap.add_argument("--ref-cols", type=int, default=2048, help="reference arm: output columns per linear")
+    ap.add_argument("--cpu-rows", type=int, default=8, help="cpu_baseline sample: tokens")
+    ap.add_argument("--cpu-cols", type=int, default=4096, help="cpu_baseline sample: output columns")
+    ap.add_argument("--no-rows", action="store_true", help="skip the secondary rows")
+    ap.add_argument("--no-cpu", action="store_true", help="skip the oracle CPU baseline")
+    args = ap.parse_args()
+    args.warmup = max(3, args.warmup)
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    if world > 1:
+        import datetime
+
+        import torch
+        import torch.distributed as dist
+        torch.cuda.set_device(int(os.environ.get("LOCAL_RANK", 0)))
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    try:
+        if args.impl == "reference":
+            run_reference(args, rank, world)
+        else:
+            run_ours(args, rank, world)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -43,21 +43,18 @@ struct Fp4Layout {
     static constexpr int STAGE = A_BYTES + B_BYTES + SFA_BYTES + SFB_BYTES;
     static constexpr int BAR_OFF = STAGES * STAGE;
     static constexpr int SMEM = BAR_OFF + 256 + 1024;              // barriers + alignment slack
-    // TMEM columns: accumulator, then the scale factors of one stage
+    // TMEM columns: accumulator, then one scale-factor region per pipeline stage
+    // (SFA 16 columns, SFB 16 per 128 rows), so that copying the next stage's
+    // scales never waits for the MMAs still reading the previous ones.
+    static constexpr int SF_COLS = 16 + 16 * SFB_HALVES;
     static constexpr int SFA_COL = BN;
     static constexpr int SFB_COL = BN + 16;
-    static constexpr int TMEM_USED = BN + 16 + 16 * SFB_HALVES;
+    static constexpr int TMEM_USED = BN + STAGES * SF_COLS;
     static constexpr int TMEM_COLS = TMEM_USED <= 32 ? 32 : TMEM_USED <= 64 ? 64 : TMEM_USED <= 128 ? 128
                                      : TMEM_USED <= 256 ? 256 : 512;
     static_assert(STAGE % 1024 == 0, "stage must keep 1024-byte alignment of the swizzled tiles");
+    static_assert(TMEM_USED <= 512, "tensor memory holds 512 columns");
 };
-
-__device__ __forceinline__ bool mbar_wait_drain(uint64_t* bar, uint32_t parity, uint64_t limit_ns) {
-    const uint64_t t0 = globaltimer();
-    while (!mbar_try_wait(bar, parity))
-        if (globaltimer() - t0 > limit_ns) return false;
-    return true;
-}
 
 __device__ __forceinline__ void tmem_ld_32x32b_x16(uint32_t taddr, uint32_t (&r)[16]) {
     asm volatile(
@@ -173,8 +170,6 @@ __global__ void __launch_bounds__(192, 1)
         if (lane == 0) {
             // ------------------------------ MMA issuer ------------------------------
             const uint32_t acc = tmem;
-            const uint32_t sfa_t = tmem + L::SFA_COL;
-            const uint32_t sfb_t = tmem + L::SFB_COL;
             constexpr int MMA_N = BN;
             int i = 0;
             bool ok = true;
@@ -186,6 +181,8 @@ __global__ void __launch_bounds__(192, 1)
                 }
                 tc_fence_after();
                 const uint8_t* st = smem + s * L::STAGE;
+                const uint32_t sfa_t = tmem + L::SFA_COL + s * L::SF_COLS;
+                const uint32_t sfb_t = tmem + L::SFB_COL + s * L::SF_COLS;
                 const uint32_t sA = smem_u32(st), sB = smem_u32(st + L::A_BYTES);
                 const uint32_t sSFA = smem_u32(st + L::A_BYTES + L::B_BYTES);
                 const uint32_t sSFB = sSFA + L::SFA_BYTES;
@@ -298,27 +295,6 @@ static cudaError_t launch_ex(Kern kern, dim3 grid, dim3 block, size_t smem, bool
     cfg.attrs = attr;
     cfg.numAttrs = pdl ? 1 : 0;
     return cudaLaunchKernelEx(&cfg, kern, a, b, g);
-}
-
-template <bool NV>
-static cudaError_t launch_fp4_t(const CUtensorMap& tmA, const CUtensorMap& tmB, const GemmArgs& g, bool pdl,
-                                cudaStream_t st) {
-    constexpr int STAGES = 4;
-    using L = Fp4Layout<kBN, STAGES>;
-    auto kern = gemm_fp4_kernel<NV, kBN, STAGES, false>;
-    static bool attr_set = false;
-    if (!attr_set) {
-        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::SMEM);
-        if (e != cudaSuccess) return e;
-        attr_set = true;
-    }
-    const int tiles = ((g.M + kBM - 1) / kBM) * ((g.N + kBN - 1) / kBN);
-    return launch_ex(kern, dim3(tiles), dim3(192), L::SMEM, pdl, st, tmA, tmB, g);
-}
-
-cudaError_t launch_gemm_fp4(bool nvfp4, const CUtensorMap& tmA, const CUtensorMap& tmB, const GemmArgs& g,
-                            int /*num_sms*/, bool pdl, cudaStream_t st) {
-    return nvfp4 ? launch_fp4_t<true>(tmA, tmB, g, pdl, st) : launch_fp4_t<false>(tmA, tmB, g, pdl, st);
 }
 
 template <bool NV>

@@ -26,6 +26,7 @@ struct QuantArgs {
     const float* static_s2;  // nullable
     float* s2_out;           // NVFP4 s2 ([1] or [M])
     const float* tensor_amax;  // NVFP4 tensor mode without static s2
+    int rows_pad;              // pad128(M): rows of the scale atoms (set by the launcher)
 };
 
 struct ResidualArgs {

@@ -22,9 +22,9 @@ __constant__ float kE2M1Mag[8] = {0.0f, 0.5f, 1.0f, 1.5f, 2.0f, 3.0f, 4.0f, 6.0f
 __device__ __forceinline__ float bf16lo(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float bf16hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
 
-// E2M1 codes of 8 floats packed into one word, element i in nibble i; the sign
-// bit of each nibble is the sign bit of its input (so a negative value that
-// rounds to zero encodes as 0x8), independent of how cvt treats -0.
+// E2M1 codes of 8 floats packed into one word, element i in nibble i (round
+// to nearest even, saturating at 6).  The conversion keeps the input's sign
+// bit, so a negative value that rounds to zero (and -0) encodes as 0x8.
 __device__ __forceinline__ uint32_t e2m1x8(const float (&v)[8]) {
     uint32_t out;
     asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\t"
@@ -35,10 +35,70 @@ __device__ __forceinline__ uint32_t e2m1x8(const float (&v)[8]) {
         "mov.b32 %0, {b0, b1, b2, b3};\n\t}"
         : "=r"(out)
         : "f"(v[0]), "f"(v[1]), "f"(v[2]), "f"(v[3]), "f"(v[4]), "f"(v[5]), "f"(v[6]), "f"(v[7]));
-    uint32_t sgn = 0;
+    return out;
+}
+
+// Bracketing multipliers for a divisor d: with r = RN(1/d),
+// rlo = RN(r * (1 - 2^-21)) and rhi = RN(r * (1 + 2^-21)) satisfy, for every x
+// whose quotient is a normal float, |x*rlo| < |RN(x/d)| < |x*rhi| (the three
+// roundings contribute at most 3 * 2^-24 relative error, less than 2^-21).
+// Any function of the quotient that is monotone in its magnitude (E2M1
+// conversion, rint) therefore gives RN(x/d)'s result whenever it gives the
+// same result at both brackets; otherwise the exact division decides.
+// Quotients below the normal range convert to zero at both brackets.
+struct Bracket {
+    float lo, hi;
+    bool ok;  // false: 1/d is not finite, always divide
+};
+__device__ __forceinline__ Bracket make_bracket(float d) {
+    const float r = __frcp_rn(d);
+    Bracket b;
+    b.lo = __fmul_rn(r, 1.0f - 0x1p-21f);
+    b.hi = __fmul_rn(r, 1.0f + 0x1p-21f);
+    b.ok = fabsf(r) <= 3.0e38f;
+    return b;
+}
+
+// E2M1 codes of x[i] / d for 8 values, bit-exact with the correctly rounded quotient.
+__device__ __forceinline__ uint32_t e2m1x8_div(const float* x, float d, const Bracket& br) {
+    if (br.ok) {
+        float lo[8], hi[8];
 #pragma unroll
-    for (int i = 0; i < 8; ++i) sgn |= (__float_as_uint(v[i]) >> 31) << (4 * i + 3);
-    return out | sgn;
+        for (int i = 0; i < 8; ++i) {
+            lo[i] = __fmul_rn(x[i], br.lo);
+            hi[i] = __fmul_rn(x[i], br.hi);
+        }
+        const uint32_t clo = e2m1x8(lo), chi = e2m1x8(hi);
+        if (clo == chi) return clo;
+    }
+    float q[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) q[i] = __fdiv_rn(x[i], d);
+    return e2m1x8(q);
+}
+
+// 4-bit two's-complement codes of clamp(rint(x[i] / s), -8, 7) for 8 values,
+// bit-exact with the correctly rounded quotient (same bracketing).
+__device__ __forceinline__ uint32_t int4x8_div(const float* x, float s, const Bracket& br) {
+    int q[8];
+    bool same = br.ok;
+    if (br.ok) {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            const int a = __float2int_rn(__fmul_rn(x[i], br.lo));
+            const int b = __float2int_rn(__fmul_rn(x[i], br.hi));
+            q[i] = a;
+            same &= (a == b);
+        }
+    }
+    if (!same) {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) q[i] = __float2int_rn(__fdiv_rn(x[i], s));
+    }
+    uint32_t w = 0;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) w |= (uint32_t)(min(max(q[i], -8), 7) & 15) << (4 * i);
+    return w;
 }
 
 __device__ __forceinline__ uint8_t e4m3_rn_sat(float t) {
@@ -69,125 +129,132 @@ __device__ __forceinline__ float warp_max(float v) {
 }
 
 // ---------------------------------------------------------------------------
-// Quantize rows.  Grid: one CTA per row r in [0, rows_pad); rows >= M only
-// write zero scales (padding of the 128-row scale atoms).
+// Quantize rows.  A CTA owns `rows_per_cta` consecutive rows: one bulk copy
+// per row brings the bf16 row into shared memory (several CTAs per SM keep
+// tens of KB in flight), a first pass takes per-token amaxes (NVFP4 TOKEN),
+// a second quantizes.  Work item = (row, chunk of 16 elements), flattened so
+// that every thread is busy whatever K is; since K/16 is a multiple of 8,
+// the groups of 2 (MXFP4) and 8 (INT4, scale packing) consecutive items that
+// the shuffles combine never straddle two rows.  Rows >= M only write zero
+// scales (padding of the 128-row scale atoms).
 // ---------------------------------------------------------------------------
-template <int FMT, int J, bool GATHER>
-__global__ void __launch_bounds__(256) quant_rows_kernel(QuantArgs a) {
+template <int FMT, bool GATHER>
+__global__ void __launch_bounds__(256) quant_rows_kernel(QuantArgs a, int rows_per_cta) {
     pdl_launch_dependents();
-    const int r = blockIdx.x;
-    const int T = blockDim.x;
-    const int t = threadIdx.x;
-    const int nchunk = a.K / 16;           // chunks of the quantized columns
-    const bool live = r < a.M;
-    const int lane = t & 31;
+    extern __shared__ __align__(16) uint8_t qsm[];
+    const int row_bytes = a.K_src * 2;                        // bf16 source row in shared memory
+    uint64_t* bar = reinterpret_cast<uint64_t*>(qsm + (size_t)rows_per_cta * row_bytes);
+    float* rmax = reinterpret_cast<float*>(bar + 1);          // [rows_per_cta] per-token amax
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(rmax + rows_per_cta);
+    const int t = threadIdx.x, T = blockDim.x;
+    const int r0 = blockIdx.x * rows_per_cta;
+    const int nrows = min(rows_per_cta, a.rows_pad - r0);
+    const int nlive = max(0, min(nrows, a.M - r0));
+    const int nchunk = a.K / 16;
 
-    uint32_t raw[J][8];
-    float amax_thread = 0.0f;
+    if (t == 0) {
+        mbar_init(bar, 1);
+        *abort_flag = 0;
+        fence_mbar_init();
+    }
+    if (t < rows_per_cta) rmax[t] = 0.0f;
+    __syncthreads();
+    if (t == 0 && nlive > 0) {
+        mbar_arrive_expect_tx(bar, (uint32_t)(nlive * row_bytes));
+        for (int i = 0; i < nlive; ++i)
+            bulk_load(qsm + (size_t)i * row_bytes, a.X + (size_t)(r0 + i) * a.ldx, row_bytes, bar);
+    }
+    bool ok = true;
+    if (nlive > 0) ok = mbar_wait(bar, 0, 2000000000ull, abort_flag);
+    if (!ok) {
+        if (t == 0) mbar_wait(bar, 0, 100000000ull, abort_flag);  // drain (abort already set: returns)
+        return;
+    }
+
+    const bool token = FMT == FMT_NVFP4 && a.mode == 1 && !a.static_s2;
+    const int items = nrows * nchunk;
+    if (token) {
+        for (int it = t; it < items; it += T) {
+            const int i = it / nchunk, c = it - i * nchunk;
+            if (i >= nlive) break;
+            const uint4* p = reinterpret_cast<const uint4*>(qsm + (size_t)i * row_bytes) + 2 * c;
+            // the augmented weight columns never take this path (weights use TENSOR)
+            const uint4 v0 = p[0], v1 = p[1];
+            const uint32_t w[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
+            float m = 0.0f;
 #pragma unroll
-    for (int j = 0; j < J; ++j) {
-        const int c = t + T * j;
-        if (live && c < nchunk) {
+            for (int e = 0; e < 8; ++e) m = fmaxf(m, fmaxf(fabsf(bf16lo(w[e])), fabsf(bf16hi(w[e]))));
+            atomicMax(reinterpret_cast<unsigned int*>(rmax + i), __float_as_uint(m));  // m >= 0
+        }
+        __syncthreads();
+    }
+    float tensor_s2 = 1.0f;
+    if constexpr (FMT == FMT_NVFP4) {
+        if (a.mode == 0) tensor_s2 = a.static_s2 ? a.static_s2[0] : nvfp4_s2(*a.tensor_amax);
+        if (a.mode == 0 && blockIdx.x == 0 && t == 0 && a.s2_out) a.s2_out[0] = tensor_s2;
+        if (a.mode == 1 && t < nlive) a.s2_out[r0 + t] = a.static_s2 ? a.static_s2[r0 + t] : nvfp4_s2(rmax[t]);
+    }
+
+    const int iters = (items + T - 1) / T;
+    for (int j = 0; j < iters; ++j) {
+        const int it = t + T * j;
+        const bool valid = it < items;           // uniform per group of 8 lanes
+        const int i = valid ? it / nchunk : 0;
+        const int c = valid ? it - i * nchunk : 0;
+        const int r = r0 + i;
+        const bool live = valid && i < nlive;
+        float x[16];
+        if (live) {
+            const uint8_t* row = qsm + (size_t)i * row_bytes;
             if (!GATHER || 16 * c + 16 <= a.K_src) {
-                const uint4* p = reinterpret_cast<const uint4*>(a.X + (size_t)r * a.ldx + 16 * c);
-                uint4 v0 = __ldg(p), v1 = __ldg(p + 1);
-                raw[j][0] = v0.x; raw[j][1] = v0.y; raw[j][2] = v0.z; raw[j][3] = v0.w;
-                raw[j][4] = v1.x; raw[j][5] = v1.y; raw[j][6] = v1.z; raw[j][7] = v1.w;
+                const uint4* p = reinterpret_cast<const uint4*>(row) + 2 * c;
+                const uint4 v0 = p[0], v1 = p[1];
+                const uint32_t w[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
+#pragma unroll
+                for (int e = 0; e < 8; ++e) {
+                    x[2 * e] = bf16lo(w[e]);
+                    x[2 * e + 1] = bf16hi(w[e]);
+                }
             } else {
                 // augmented weight columns: element k >= K_src is column S[k - K_src]
-                const uint16_t* row = a.X + (size_t)r * a.ldx;
+                const uint16_t* rw = reinterpret_cast<const uint16_t*>(row);
 #pragma unroll
-                for (int i = 0; i < 8; ++i) {
-                    int k0 = 16 * c + 2 * i - a.K_src;
-                    uint32_t lo = row[checked_channel(a.S, k0, a.K_src)];
-                    uint32_t hi = row[checked_channel(a.S, k0 + 1, a.K_src)];
-                    raw[j][i] = lo | (hi << 16);
-                }
+                for (int e = 0; e < 16; ++e)
+                    x[e] = __uint_as_float((uint32_t)rw[checked_channel(a.S, 16 * c + e - a.K_src, a.K_src)] << 16);
             }
         } else {
 #pragma unroll
-            for (int i = 0; i < 8; ++i) raw[j][i] = 0;
-        }
-#pragma unroll
-        for (int i = 0; i < 8; ++i)
-            amax_thread = fmaxf(amax_thread, fmaxf(fabsf(bf16lo(raw[j][i])), fabsf(bf16hi(raw[j][i]))));
-    }
-
-    // ---- NVFP4 second-level scale of this row ----
-    float s2 = 1.0f;
-    if constexpr (FMT == FMT_NVFP4) {
-        if (a.mode == 1) {  // per token
-            if (a.static_s2) {
-                s2 = live ? a.static_s2[r] : 1.0f;
-            } else {
-                __shared__ float red[32];
-                float w = warp_max(amax_thread);
-                if (lane == 0) red[t >> 5] = w;
-                __syncthreads();
-                if (t < 32) {
-                    float v = (t < (T >> 5)) ? red[t] : 0.0f;
-                    v = warp_max(v);
-                    if (t == 0) red[0] = v;
-                }
-                __syncthreads();
-                s2 = nvfp4_s2(red[0]);
-            }
-            if (live && t == 0) a.s2_out[r] = s2;
-        } else {  // one scale for the tensor
-            if (a.static_s2) {
-                s2 = a.static_s2[0];
-            } else {
-                s2 = nvfp4_s2(*a.tensor_amax);
-            }
-            if (r == 0 && t == 0 && a.s2_out) a.s2_out[0] = s2;
-        }
-    }
-
-#pragma unroll
-    for (int j = 0; j < J; ++j) {
-        const int c = t + T * j;
-        // every lane takes part in the shuffles below; `valid` is uniform per
-        // group of 8 lanes because nchunk % 8 == 0 and T % 32 == 0
-        const bool valid = c < nchunk;
-        float x[16];
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-            x[2 * i] = bf16lo(raw[j][i]);
-            x[2 * i + 1] = bf16hi(raw[j][i]);
+            for (int e = 0; e < 16; ++e) x[e] = 0.0f;
         }
         float bmax = 0.0f;
 #pragma unroll
-        for (int i = 0; i < 16; ++i) bmax = fmaxf(bmax, fabsf(x[i]));
+        for (int e = 0; e < 16; ++e) bmax = fmaxf(bmax, fabsf(x[e]));
 
         uint32_t w0 = 0, w1 = 0;  // 16 codes
         if constexpr (FMT == FMT_NVFP4) {
             uint8_t sb = 0;
-            if (live && valid) {
+            if (live) {
+                const float s2 = a.mode == 1 ? (a.static_s2 ? a.static_s2[r] : nvfp4_s2(rmax[i])) : tensor_s2;
                 sb = e4m3_rn_sat(__fdiv_rn(__fdiv_rn(bmax, 6.0f), s2));
                 if (sb != 0) {
                     const float d = __fmul_rn(e4m3_value(sb), s2);
-                    float q0[8], q1[8];
-#pragma unroll
-                    for (int i = 0; i < 8; ++i) {
-                        q0[i] = __fdiv_rn(x[i], d);
-                        q1[i] = __fdiv_rn(x[8 + i], d);
-                    }
-                    w0 = e2m1x8(q0);
-                    w1 = e2m1x8(q1);
+                    const Bracket br = make_bracket(d);
+                    w0 = e2m1x8_div(x, d, br);
+                    w1 = e2m1x8_div(x + 8, d, br);
                 }
             }
             // gather 4 consecutive block scales (lanes l..l+3) into one word
-            uint32_t b = sb;
-            uint32_t b1 = __shfl_down_sync(0xffffffffu, b, 1);
-            uint32_t b2 = __shfl_down_sync(0xffffffffu, b, 2);
-            uint32_t b3 = __shfl_down_sync(0xffffffffu, b, 3);
+            const uint32_t b = sb;
+            const uint32_t b1 = __shfl_down_sync(0xffffffffu, b, 1);
+            const uint32_t b2 = __shfl_down_sync(0xffffffffu, b, 2);
+            const uint32_t b3 = __shfl_down_sync(0xffffffffu, b, 3);
             if (valid && (c & 3) == 0)
                 *reinterpret_cast<uint32_t*>(a.sf + sf_offset(r, c, a.sf_col_atoms)) =
                     b | (b1 << 8) | (b2 << 16) | (b3 << 24);
         } else if constexpr (FMT == FMT_MXFP4) {
-            bmax = fmaxf(bmax, __shfl_xor_sync(0xffffffffu, bmax, 1));  // 32-element block = 2 lanes
+            bmax = fmaxf(bmax, __shfl_xor_sync(0xffffffffu, bmax, 1));  // 32-element block = 2 items
             uint32_t code = 0;
-            if (live && valid && bmax > 0.0f) {
+            if (live && bmax > 0.0f) {
                 const uint32_t u = __float_as_uint(bmax);
                 const int E = (int)(u >> 23);
                 const int e = (E != 0) ? E - 127 : (31 - __clz((int)(u & 0x7FFFFF))) - 149;
@@ -195,38 +262,32 @@ __global__ void __launch_bounds__(256) quant_rows_kernel(QuantArgs a) {
                 const float inv = __uint_as_float((254u - code) << 23);  // 2^(127 - code)
                 float q0[8], q1[8];
 #pragma unroll
-                for (int i = 0; i < 8; ++i) {
-                    q0[i] = __fmul_rn(x[i], inv);
-                    q1[i] = __fmul_rn(x[8 + i], inv);
+                for (int e2 = 0; e2 < 8; ++e2) {
+                    q0[e2] = __fmul_rn(x[e2], inv);
+                    q1[e2] = __fmul_rn(x[8 + e2], inv);
                 }
                 w0 = e2m1x8(q0);
                 w1 = e2m1x8(q1);
             }
-            uint32_t b1 = __shfl_down_sync(0xffffffffu, code, 2);
-            uint32_t b2 = __shfl_down_sync(0xffffffffu, code, 4);
-            uint32_t b3 = __shfl_down_sync(0xffffffffu, code, 6);
+            const uint32_t b1 = __shfl_down_sync(0xffffffffu, code, 2);
+            const uint32_t b2 = __shfl_down_sync(0xffffffffu, code, 4);
+            const uint32_t b3 = __shfl_down_sync(0xffffffffu, code, 6);
             if (valid && (c & 7) == 0)
                 *reinterpret_cast<uint32_t*>(a.sf + sf_offset(r, c >> 1, a.sf_col_atoms)) =
                     code | (b1 << 8) | (b2 << 16) | (b3 << 24);
-        } else {  // INT4, 128-element group = 8 lanes
+        } else {  // INT4, 128-element group = 8 items
             bmax = fmaxf(bmax, __shfl_xor_sync(0xffffffffu, bmax, 1));
             bmax = fmaxf(bmax, __shfl_xor_sync(0xffffffffu, bmax, 2));
             bmax = fmaxf(bmax, __shfl_xor_sync(0xffffffffu, bmax, 4));
-            const float s = (live && valid) ? __fdiv_rn(bmax, 7.0f) : 0.0f;
-            if (s != 0.0f) {
-#pragma unroll
-                for (int i = 0; i < 8; ++i) {
-                    int q = __float2int_rn(__fdiv_rn(x[i], s));
-                    q = min(max(q, -8), 7);
-                    w0 |= (uint32_t)(q & 15) << (4 * i);
-                    int p = __float2int_rn(__fdiv_rn(x[8 + i], s));
-                    p = min(max(p, -8), 7);
-                    w1 |= (uint32_t)(p & 15) << (4 * i);
-                }
+            const float sc = live ? __fdiv_rn(bmax, 7.0f) : 0.0f;
+            if (sc != 0.0f) {
+                const Bracket br = make_bracket(sc);
+                w0 = int4x8_div(x, sc, br);
+                w1 = int4x8_div(x + 8, sc, br);
             }
-            if (valid && (c & 7) == 0) a.sfi[(size_t)(c >> 3) * a.sfi_ld + r] = s;
+            if (valid && (c & 7) == 0) a.sfi[(size_t)(c >> 3) * a.sfi_ld + r] = sc;
         }
-        if (live && valid) *reinterpret_cast<uint2*>(a.codes + (size_t)r * a.ldc + 8 * c) = make_uint2(w0, w1);
+        if (live) *reinterpret_cast<uint2*>(a.codes + (size_t)r * a.ldc + 8 * c) = make_uint2(w0, w1);
     }
 }
 
@@ -291,13 +352,9 @@ __global__ void __launch_bounds__(128) residual_kernel(ResidualArgs a) {
         sb = e4m3_rn_sat(__fdiv_rn(__fdiv_rn(bmax, 6.0f), s2));
         if (sb != 0) {
             const float d = __fmul_rn(e4m3_value(sb), s2);
-            float q0[8], q1[8];
-            for (int i = 0; i < 8; ++i) {
-                q0[i] = __fdiv_rn(R[i], d);
-                q1[i] = __fdiv_rn(R[8 + i], d);
-            }
-            w0 = e2m1x8(q0);
-            w1 = e2m1x8(q1);
+            const Bracket br = make_bracket(d);
+            w0 = e2m1x8_div(R, d, br);
+            w1 = e2m1x8_div(R + 8, d, br);
         }
         *reinterpret_cast<uint2*>(a.codes + (size_t)r * a.ldc + (a.K >> 1) + 8 * b) = make_uint2(w0, w1);
     }
@@ -360,20 +417,23 @@ __global__ void __launch_bounds__(1024) compact_kernel(const int* selected, int 
 // ---------------------------------------------------------------------------
 template <int FMT, bool GATHER>
 static cudaError_t launch_quant_fmt(const QuantArgs& a, int rows_pad, cudaStream_t st) {
-    const int nchunk = a.K / 16;
-    int J = 1;
-    while (J < 16 && (nchunk + J - 1) / J > 256) J <<= 1;
-    int T = (nchunk + J - 1) / J;
-    T = (T + 31) / 32 * 32;
-    if (T > 256) return cudaErrorInvalidValue;
-    dim3 grid(rows_pad), block(T);
-    switch (J) {
-        case 1: quant_rows_kernel<FMT, 1, GATHER><<<grid, block, 0, st>>>(a); break;
-        case 2: quant_rows_kernel<FMT, 2, GATHER><<<grid, block, 0, st>>>(a); break;
-        case 4: quant_rows_kernel<FMT, 4, GATHER><<<grid, block, 0, st>>>(a); break;
-        case 8: quant_rows_kernel<FMT, 8, GATHER><<<grid, block, 0, st>>>(a); break;
-        default: quant_rows_kernel<FMT, 16, GATHER><<<grid, block, 0, st>>>(a); break;
+    const int row_bytes = a.K_src * 2;
+    int rpc = 32768 / row_bytes;                 // about 32 KB of rows per CTA
+    rpc = rpc < 1 ? 1 : (rpc > 64 ? 64 : rpc);
+    const size_t smem = (size_t)rpc * row_bytes + 16 + 4 * rpc + 16;
+    if (smem > 200 * 1024) return cudaErrorInvalidValue;
+    auto kern = quant_rows_kernel<FMT, GATHER>;
+    static size_t attr = 0;
+    if (smem > 48 * 1024 && smem > attr) {
+        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e != cudaSuccess) return e;
+        attr = smem;
     }
+    const int items = rpc * (a.K / 16);
+    int T = items < 256 ? (items + 31) / 32 * 32 : 256;
+    QuantArgs b = a;
+    b.rows_pad = rows_pad;
+    kern<<<(rows_pad + rpc - 1) / rpc, T, smem, st>>>(b, rpc);
     return cudaGetLastError();
 }
 

@@ -186,6 +186,9 @@ def run_ours(args, rank, world):
     P = peaks()
     fp4_peak = P["bf16"] * FP4_PER_BF16
     M = args.tokens
+    if args.only is not None:
+        print(json.dumps({"only": args.only, "rows": extra_rows(args, dev, stream, P)}), flush=True)
+        return
 
     # ---- workload: Llama-2-70B layer linears, NVFP4 weights quantized once ----
     layers = []
@@ -312,9 +315,10 @@ def extra_rows(args, dev, stream, P):
     out = {}
     hbm = P["hbm"]
     it = max(5, args.steps)
+    want = lambda name: args.only is None or args.only == name
 
     # activation quantizer, per-token NVFP4 (and MXFP4 / INT4), Llama qkv and w2 inputs
-    for (name, M, K) in [("qkv_in", args.tokens, 8192), ("w2_in", args.tokens, 28672)]:
+    for (name, M, K) in [] if not want("quant") else [("qkv_in", args.tokens, 8192), ("w2_in", args.tokens, 28672)]:
         X = to_dev(synth.activations("llama2_70b", M, K, seed=3), dev)
         for fmt, g, sb in [(w4.NVFP4, 16, 1), (w4.MXFP4, 32, 1), (w4.INT4, 128, 4)]:
             q = w4.QTensor(fmt, M, K, w4.SCALE_TOKEN if fmt == w4.NVFP4 else 0, dev)
@@ -335,11 +339,13 @@ def extra_rows(args, dev, stream, P):
 
     # decode: M = 1 and 16 over the layer (weights streamed from HBM)
     Ws = []
-    for li, (name, K, N) in enumerate(LLAMA):
+    if not want("decode"):
+        Ws = None
+    for li, (name, K, N) in enumerate(LLAMA if Ws is not None else []):
         Wd = to_dev(synth.weights("llama2_70b", N, K, seed=0, tensor_id=100 + li), dev)
         Ws.append((K, N, w4.quantize_weight(Wd, w4.NVFP4)))
         del Wd
-    for Md in (1, 16):
+    for Md in ((1, 16) if Ws is not None else ()):
         bufs = []
         for (K, N, Wq) in Ws:
             X = to_dev(synth.activations("llama2_70b", Md, K, seed=5), dev)
@@ -359,7 +365,7 @@ def extra_rows(args, dev, stream, P):
 
     # INT4-g128, Qwen2.5-7B shapes at M = 2048
     tot_ms, tot_ops = 0.0, 0.0
-    for li, (name, K, N) in enumerate(synth.SHAPES["qwen25_7b_int4"]):
+    for li, (name, K, N) in enumerate(synth.SHAPES["qwen25_7b_int4"] if want("int4") else []):
         M = 2048
         Wq = w4.quantize_weight(to_dev(synth.weights("qwen25_7b_int4", N, K, tensor_id=300 + li), dev), w4.INT4)
         X = to_dev(synth.activations("qwen25_7b_int4", M, K), dev)
@@ -371,12 +377,13 @@ def extra_rows(args, dev, stream, P):
         tot_ms += ms
         tot_ops += 2.0 * M * N * K
     i8_peak = P["bf16"] * INT8_PER_BF16
-    v = tot_ops / (tot_ms * 1e-3) / 1e12
-    out["int4_g128_qwen25_7b_m2048"] = {"TOPS": round(v, 1), "frac_int8_peak": round(v / i8_peak, 3)}
+    if tot_ms > 0:
+        v = tot_ops / (tot_ms * 1e-3) / 1e12
+        out["int4_g128_qwen25_7b_m2048"] = {"TOPS": round(v, 1), "frac_int8_peak": round(v / i8_peak, 3)}
 
     # dual-stage residual augmentation, Qwen2.5-3B shapes at M = 8192
     tot_ms, tot_f, tot_fk = 0.0, 0.0, 0.0
-    for li, (name, K, N) in enumerate(synth.SHAPES["qwen25_3b_aug"]):
+    for li, (name, K, N) in enumerate(synth.SHAPES["qwen25_3b_aug"] if want("aug") else []):
         M, nS = 8192, 256
         Xc = to_dev(synth.calibration("qwen25_3b_aug", K), dev)
         S = w4.select_channels(Xc, nS)
@@ -390,8 +397,13 @@ def extra_rows(args, dev, stream, P):
         tot_ms += ms
         tot_f += 2.0 * M * N * (K + nS)
         tot_fk += 2.0 * M * N * K
-    out["aug_nvfp4_qwen25_3b_m8192"] = {"TFLOPS_exec": round(tot_f / (tot_ms * 1e-3) / 1e12, 1),
-                                        "TFLOPS_effective_K": round(tot_fk / (tot_ms * 1e-3) / 1e12, 1)}
+    if tot_ms > 0:
+        out["aug_nvfp4_qwen25_3b_m8192"] = {"TFLOPS_exec": round(tot_f / (tot_ms * 1e-3) / 1e12, 1),
+                                            "TFLOPS_effective_K": round(tot_fk / (tot_ms * 1e-3) / 1e12, 1)}
+    if not want("mxfp4"):
+        torch.cuda.synchronize()
+        assert w4.device_status() == w4.OK
+        return out
 
     # MXFP4 GEMM on the Llama qkv shape, M = 4096
     K, N, M = 8192, 10240, args.tokens
@@ -420,6 +432,8 @@ def main():
     ap.add_argument("--cpu-rows", type=int, default=8, help="cpu_baseline sample: tokens")
     ap.add_argument("--cpu-cols", type=int, default=4096, help="cpu_baseline sample: output columns")
     ap.add_argument("--no-rows", action="store_true", help="skip the secondary rows")
+    ap.add_argument("--only", choices=["quant", "decode", "int4", "aug", "mxfp4"], default=None,
+                    help="run only one secondary row (for profiling) and print it")
     ap.add_argument("--no-cpu", action="store_true", help="skip the oracle CPU baseline")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)

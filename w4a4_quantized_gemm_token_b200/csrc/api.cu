@@ -125,7 +125,7 @@ int quantize_rows(const uint16_t* X, int M, int K, int ldx, const int32_t* S, in
         if (e != cudaSuccess) return W4A4_ERR_CUDA;
         a.tensor_amax = q->s2 + 1;
     }
-    return cuda_status(launch_quant(q->format, S != nullptr, a, pad128(M), st));
+    return cuda_status(launch_quant(q->format, S != nullptr, a, pad128(M), num_sms, st));
 }
 
 int check_S_args(const int32_t* S, int nS, int K) {

@@ -60,7 +60,7 @@ struct GemmArgs {
     unsigned long long wait_limit_ns;
 };
 
-cudaError_t launch_quant(int fmt, bool gather, const QuantArgs& a, int rows_pad, cudaStream_t st);
+cudaError_t launch_quant(int fmt, bool gather, const QuantArgs& a, int rows_pad, int num_sms, cudaStream_t st);
 cudaError_t launch_amax(const uint16_t* X, int M, int K, int ldx, float* out, int num_sms, cudaStream_t st);
 cudaError_t launch_residual(const ResidualArgs& a, cudaStream_t st);
 cudaError_t launch_select(const uint16_t* X, int Mc, int K, int ldx, int nS, int32_t* S, float* amax, int* sel,

@@ -22,6 +22,19 @@ __constant__ float kE2M1Mag[8] = {0.0f, 0.5f, 1.0f, 1.5f, 2.0f, 3.0f, 4.0f, 6.0f
 __device__ __forceinline__ float bf16lo(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float bf16hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
 
+// max |x| of the 16 bf16 elements held in w[8]: packed bf16x2 maxima of the
+// magnitudes (exact; the xorsign result sign is discarded), then the halves.
+__device__ __forceinline__ float bmax16(const uint32_t* w) {
+    uint32_t m[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) asm("max.xorsign.abs.bf16x2 %0, %1, %2;" : "=r"(m[e]) : "r"(w[e]), "r"(w[e + 4]));
+    asm("max.xorsign.abs.bf16x2 %0, %0, %1;" : "+r"(m[0]) : "r"(m[2]));
+    asm("max.xorsign.abs.bf16x2 %0, %0, %1;" : "+r"(m[1]) : "r"(m[3]));
+    asm("max.xorsign.abs.bf16x2 %0, %0, %1;" : "+r"(m[0]) : "r"(m[1]));
+    const uint32_t a = m[0] & 0x7FFF7FFFu;
+    return fmaxf(__uint_as_float(a << 16), __uint_as_float(a & 0xFFFF0000u));
+}
+
 // E2M1 codes of 8 floats packed into one word, element i in nibble i (round
 // to nearest even, saturating at 6).  The conversion keeps the input's sign
 // bit, so a negative value that rounds to zero (and -0) encodes as 0x8.
@@ -38,67 +51,92 @@ __device__ __forceinline__ uint32_t e2m1x8(const float (&v)[8]) {
     return out;
 }
 
-// Bracketing multipliers for a divisor d: with r = RN(1/d),
-// rlo = RN(r * (1 - 2^-21)) and rhi = RN(r * (1 + 2^-21)) satisfy, for every x
-// whose quotient is a normal float, |x*rlo| < |RN(x/d)| < |x*rhi| (the three
-// roundings contribute at most 3 * 2^-24 relative error, less than 2^-21).
-// Any function of the quotient that is monotone in its magnitude (E2M1
-// conversion, rint) therefore gives RN(x/d)'s result whenever it gives the
-// same result at both brackets; otherwise the exact division decides.
-// Quotients below the normal range convert to zero at both brackets.
-struct Bracket {
-    float lo, hi;
-    bool ok;  // false: 1/d is not finite, always divide
-};
-__device__ __forceinline__ Bracket make_bracket(float d) {
-    const float r = __frcp_rn(d);
-    Bracket b;
-    b.lo = __fmul_rn(r, 1.0f - 0x1p-21f);
-    b.hi = __fmul_rn(r, 1.0f + 0x1p-21f);
-    b.ok = fabsf(r) <= 3.0e38f;
-    return b;
+// Correctly rounded quotient x/d from a correctly rounded reciprocal
+// y = RN(1/d): q = RN(x*y) is within an ulp of x/d, the residual x - q*d is
+// exact in one FMA, and one more FMA rounds q + residual*y to RN(x/d).  This
+// holds whenever the quotient is a normal float; the callers keep operands in
+// that range (or their results do not depend on it: quotients below the
+// normal range encode to zero anyway) and fall back to IEEE division outside.
+// d > 0, so the quotient carries x's sign; restoring it keeps -0 for x = -0
+// (the residual step would otherwise return +0).
+__device__ __forceinline__ float div_refined(float x, float d, float y) {
+    const float q = __fmul_rn(x, y);
+    return copysignf(__fmaf_rn(__fmaf_rn(-q, d, x), y, q), x);
 }
 
-// E2M1 codes of x[i] / d for 8 values, bit-exact with the correctly rounded quotient.
-__device__ __forceinline__ uint32_t e2m1x8_div(const float* x, float d, const Bracket& br) {
-    if (br.ok) {
-        float lo[8], hi[8];
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-            lo[i] = __fmul_rn(x[i], br.lo);
-            hi[i] = __fmul_rn(x[i], br.hi);
-        }
-        const uint32_t clo = e2m1x8(lo), chi = e2m1x8(hi);
-        if (clo == chi) return clo;
-    }
+// Two correctly rounded quotients at once with sm_100's packed FP32 pipe.
+// Inputs are the NEGATED dividends nx = -x (the bf16 unpack yields them at no
+// cost) and ny = -y.  q = nx*ny = x*y, R = q*d + nx = q*d - x (exact), and
+// q' = R*ny + q = q - R*y, the same refinement as div_refined; written this
+// way a dividend of -0 keeps its sign (q = -0, R = +0, q' = -0 + -0 = -0).
+__device__ __forceinline__ void div2_refined(uint32_t nx0, uint32_t nx1, uint64_t ny2, uint64_t d2, float& q0,
+                                             float& q1) {
+    asm("{\n\t.reg .b64 x, q, r;\n\t"
+        "mov.b64 x, {%2, %3};\n\t"
+        "mul.rn.f32x2 q, x, %4;\n\t"
+        "fma.rn.f32x2 r, q, %5, x;\n\t"
+        "fma.rn.f32x2 q, r, %4, q;\n\t"
+        "mov.b64 {%0, %1}, q;\n\t}"
+        : "=f"(q0), "=f"(q1)
+        : "r"(nx0), "r"(nx1), "l"(ny2), "l"(d2));
+}
+__device__ __forceinline__ uint64_t pack2(float v) {
+    const uint32_t u = __float_as_uint(v);
+    return ((uint64_t)u << 32) | u;
+}
+
+// Negated dividends of the 16 bf16 elements held in w[8] (element 2e in the
+// low half of w[e]): -x = float bits of the bf16 with the sign flipped.
+__device__ __forceinline__ uint32_t neg_lo(uint32_t w) { return (w << 16) ^ 0x80000000u; }
+__device__ __forceinline__ uint32_t neg_hi(uint32_t w) { return (w & 0xFFFF0000u) ^ 0x80000000u; }
+
+// E2M1 codes of x/d for the 8 elements held in w[0..3], quotients correctly
+// rounded by the refined division (divisor and quotients in normal range).
+__device__ __forceinline__ uint32_t e2m1x8_fast(const uint32_t* w, uint64_t ny2, uint64_t d2) {
     float q[8];
 #pragma unroll
-    for (int i = 0; i < 8; ++i) q[i] = __fdiv_rn(x[i], d);
+    for (int e = 0; e < 4; ++e) div2_refined(neg_lo(w[e]), neg_hi(w[e]), ny2, d2, q[2 * e], q[2 * e + 1]);
+    return e2m1x8(q);
+}
+// The same with IEEE division (any operands).
+__device__ __forceinline__ uint32_t e2m1x8_exact(uint4 v, float d) {
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+    float q[8];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+        q[2 * e] = __fdiv_rn(bf16lo(w[e]), d);
+        q[2 * e + 1] = __fdiv_rn(bf16hi(w[e]), d);
+    }
     return e2m1x8(q);
 }
 
-// 4-bit two's-complement codes of clamp(rint(x[i] / s), -8, 7) for 8 values,
-// bit-exact with the correctly rounded quotient (same bracketing).
-__device__ __forceinline__ uint32_t int4x8_div(const float* x, float s, const Bracket& br) {
-    int q[8];
-    bool same = br.ok;
-    if (br.ok) {
+// 4-bit two's-complement codes of clamp(rint(x/s), -8, 7) for the 8 elements
+// held in w[0..3].  Rounding to the nearest integer, ties to even, is an
+// addition of 1.5 * 2^23: the low bits of the sum are rint(q) in two's
+// complement.  On the refined path |x/s| <= 7(1 + 2^-24), so no clamp.
+__device__ __forceinline__ uint32_t int4x8_fast(const uint32_t* w, uint64_t ny2, uint64_t d2) {
+    constexpr float kMagic = 12582912.0f;  // 1.5 * 2^23
+    uint32_t out = 0;
 #pragma unroll
-        for (int i = 0; i < 8; ++i) {
-            const int a = __float2int_rn(__fmul_rn(x[i], br.lo));
-            const int b = __float2int_rn(__fmul_rn(x[i], br.hi));
-            q[i] = a;
-            same &= (a == b);
-        }
+    for (int e = 0; e < 4; ++e) {
+        float q0, q1;
+        div2_refined(neg_lo(w[e]), neg_hi(w[e]), ny2, d2, q0, q1);
+        const uint32_t n0 = __float_as_uint(__fadd_rn(q0, kMagic)) & 15u;
+        const uint32_t n1 = __float_as_uint(__fadd_rn(q1, kMagic)) & 15u;
+        out |= (n0 | (n1 << 4)) << (8 * e);
     }
-    if (!same) {
+    return out;
+}
+__device__ __forceinline__ uint32_t int4x8_exact(uint4 v, float s) {
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+    uint32_t out = 0;
 #pragma unroll
-        for (int i = 0; i < 8; ++i) q[i] = __float2int_rn(__fdiv_rn(x[i], s));
+    for (int e = 0; e < 4; ++e) {
+        const int n0 = min(max(__float2int_rn(__fdiv_rn(bf16lo(w[e]), s)), -8), 7);
+        const int n1 = min(max(__float2int_rn(__fdiv_rn(bf16hi(w[e]), s)), -8), 7);
+        out |= (uint32_t)((n0 & 15) | ((n1 & 15) << 4)) << (8 * e);
     }
-    uint32_t w = 0;
-#pragma unroll
-    for (int i = 0; i < 8; ++i) w |= (uint32_t)(min(max(q[i], -8), 7) & 15) << (4 * i);
-    return w;
+    return out;
 }
 
 __device__ __forceinline__ uint8_t e4m3_rn_sat(float t) {
@@ -138,38 +176,62 @@ __device__ __forceinline__ float warp_max(float v) {
 // the shuffles combine never straddle two rows.  Rows >= M only write zero
 // scales (padding of the 128-row scale atoms).
 // ---------------------------------------------------------------------------
+// Per-row constants of the NVFP4 block rule, kept in shared memory.
+struct RowConsts {
+    float s2;    // second-level scale
+    float rinv;  // RN(1/s2)
+    int fast;    // s2 in the range where refined division is exact
+    int pad;
+};
+
 template <int FMT, bool GATHER>
-__global__ void __launch_bounds__(256) quant_rows_kernel(QuantArgs a, int rows_per_cta) {
+__global__ void __launch_bounds__(256, 4) quant_rows_kernel(QuantArgs a, int rows_per_cta, int nbuf) {
     pdl_launch_dependents();
     extern __shared__ __align__(16) uint8_t qsm[];
     const int row_bytes = a.K_src * 2;                        // bf16 source row in shared memory
-    uint64_t* bar = reinterpret_cast<uint64_t*>(qsm + (size_t)rows_per_cta * row_bytes);
-    float* rmax = reinterpret_cast<float*>(bar + 1);          // [rows_per_cta] per-token amax
-    volatile int* abort_flag = reinterpret_cast<volatile int*>(rmax + rows_per_cta);
+    const size_t buf_bytes = (size_t)rows_per_cta * row_bytes;
+    uint64_t* bars = reinterpret_cast<uint64_t*>(qsm + nbuf * buf_bytes);
+    float* rmax = reinterpret_cast<float*>(bars + nbuf);      // [rows_per_cta] per-token amax
+    RowConsts* rc = reinterpret_cast<RowConsts*>(rmax + rows_per_cta);
+    float* bm = reinterpret_cast<float*>(rc + rows_per_cta);  // per-item block max (NVFP4 token mode)
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(bm + (FMT == FMT_NVFP4 ? rows_per_cta * (a.K / 16) : 0));
     const int t = threadIdx.x, T = blockDim.x;
-    const int r0 = blockIdx.x * rows_per_cta;
-    const int nrows = min(rows_per_cta, a.rows_pad - r0);
-    const int nlive = max(0, min(nrows, a.M - r0));
     const int nchunk = a.K / 16;
+    const int nblocks = (a.rows_pad + rows_per_cta - 1) / rows_per_cta;
+
+    // live rows of row block bi (rows >= M are scale padding, never loaded)
+    auto live_rows = [&](int bi) { return max(0, min(rows_per_cta, a.M - bi * rows_per_cta)); };
+    auto issue_load = [&](int bi, int buf) {
+        const int nl = live_rows(bi);
+        if (nl == 0) return;
+        mbar_arrive_expect_tx(&bars[buf], (uint32_t)(nl * row_bytes));
+        for (int i = 0; i < nl; ++i)
+            bulk_load(qsm + buf * buf_bytes + (size_t)i * row_bytes,
+                      a.X + (size_t)(bi * rows_per_cta + i) * a.ldx, row_bytes, &bars[buf]);
+    };
 
     if (t == 0) {
-        mbar_init(bar, 1);
+        for (int b = 0; b < nbuf; ++b) mbar_init(&bars[b], 1);
         *abort_flag = 0;
         fence_mbar_init();
     }
-    if (t < rows_per_cta) rmax[t] = 0.0f;
     __syncthreads();
-    if (t == 0 && nlive > 0) {
-        mbar_arrive_expect_tx(bar, (uint32_t)(nlive * row_bytes));
-        for (int i = 0; i < nlive; ++i)
-            bulk_load(qsm + (size_t)i * row_bytes, a.X + (size_t)(r0 + i) * a.ldx, row_bytes, bar);
-    }
-    bool ok = true;
-    if (nlive > 0) ok = mbar_wait(bar, 0, 2000000000ull, abort_flag);
-    if (!ok) {
-        if (t == 0) mbar_wait(bar, 0, 100000000ull, abort_flag);  // drain (abort already set: returns)
-        return;
-    }
+    if (t == 0)
+        for (int k = 0; k < nbuf; ++k) {
+            const int bi = blockIdx.x + k * gridDim.x;
+            if (bi < nblocks) issue_load(bi, k);
+        }
+
+    int li = 0;
+    for (int bi = blockIdx.x; bi < nblocks; bi += gridDim.x, ++li) {
+    const int buf = li % nbuf;
+    const uint8_t* rows = qsm + buf * buf_bytes;
+    const int r0 = bi * rows_per_cta;
+    const int nrows = min(rows_per_cta, a.rows_pad - r0);
+    const int nlive = live_rows(bi);
+    if (t < rows_per_cta) rmax[t] = 0.0f;
+    if (nlive > 0 && !mbar_wait(&bars[buf], (li / nbuf) & 1, 2000000000ull, abort_flag, 20000)) break;
+    __syncthreads();
 
     const bool token = FMT == FMT_NVFP4 && a.mode == 1 && !a.static_s2;
     const int items = nrows * nchunk;
@@ -177,74 +239,95 @@ __global__ void __launch_bounds__(256) quant_rows_kernel(QuantArgs a, int rows_p
         for (int it = t; it < items; it += T) {
             const int i = it / nchunk, c = it - i * nchunk;
             if (i >= nlive) break;
-            const uint4* p = reinterpret_cast<const uint4*>(qsm + (size_t)i * row_bytes) + 2 * c;
-            // the augmented weight columns never take this path (weights use TENSOR)
+            const uint4* p = reinterpret_cast<const uint4*>(rows + (size_t)i * row_bytes) + 2 * c;
             const uint4 v0 = p[0], v1 = p[1];
             const uint32_t w[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
-            float m = 0.0f;
-#pragma unroll
-            for (int e = 0; e < 8; ++e) m = fmaxf(m, fmaxf(fabsf(bf16lo(w[e])), fabsf(bf16hi(w[e]))));
-            atomicMax(reinterpret_cast<unsigned int*>(rmax + i), __float_as_uint(m));  // m >= 0
+            float m = bmax16(w);
+            bm[it] = m;  // reused by the quantization pass
+            // items of one row are consecutive: reduce over the 8-lane group first
+            m = fmaxf(m, __shfl_xor_sync(__activemask(), m, 1));
+            m = fmaxf(m, __shfl_xor_sync(__activemask(), m, 2));
+            m = fmaxf(m, __shfl_xor_sync(__activemask(), m, 4));
+            if ((c & 7) == 0) atomicMax(reinterpret_cast<unsigned int*>(rmax + i), __float_as_uint(m));  // m >= 0
         }
         __syncthreads();
     }
-    float tensor_s2 = 1.0f;
     if constexpr (FMT == FMT_NVFP4) {
-        if (a.mode == 0) tensor_s2 = a.static_s2 ? a.static_s2[0] : nvfp4_s2(*a.tensor_amax);
-        if (a.mode == 0 && blockIdx.x == 0 && t == 0 && a.s2_out) a.s2_out[0] = tensor_s2;
-        if (a.mode == 1 && t < nlive) a.s2_out[r0 + t] = a.static_s2 ? a.static_s2[r0 + t] : nvfp4_s2(rmax[t]);
+        const float tensor_s2 = a.mode == 0 ? (a.static_s2 ? a.static_s2[0] : nvfp4_s2(*a.tensor_amax)) : 1.0f;
+        if (a.mode == 0 && bi == 0 && t == 0 && a.s2_out) a.s2_out[0] = tensor_s2;
+        if (t < nrows) {
+            float s2 = tensor_s2;
+            if (a.mode == 1) s2 = t < nlive ? (a.static_s2 ? a.static_s2[r0 + t] : nvfp4_s2(rmax[t])) : 1.0f;
+            if (a.mode == 1 && t < nlive) a.s2_out[r0 + t] = s2;
+            RowConsts k;
+            k.s2 = s2;
+            k.rinv = __frcp_rn(s2);
+            k.fast = (s2 >= 0x1p-100f && s2 <= 0x1p100f) ? 1 : 0;
+            k.pad = 0;
+            rc[t] = k;
+        }
+        __syncthreads();
     }
 
     const int iters = (items + T - 1) / T;
+    // (row, chunk) of item t + T*j, advanced without a division per item
+    const int di = T / nchunk, dc = T - di * nchunk;
+    int i = t / nchunk, c = t - i * nchunk;
     for (int j = 0; j < iters; ++j) {
         const int it = t + T * j;
         const bool valid = it < items;           // uniform per group of 8 lanes
-        const int i = valid ? it / nchunk : 0;
-        const int c = valid ? it - i * nchunk : 0;
         const int r = r0 + i;
         const bool live = valid && i < nlive;
-        float x[16];
+        uint32_t w[8];  // 16 bf16 elements, element 2e in the low half of w[e]
         if (live) {
-            const uint8_t* row = qsm + (size_t)i * row_bytes;
+            const uint8_t* row = rows + (size_t)i * row_bytes;
             if (!GATHER || 16 * c + 16 <= a.K_src) {
                 const uint4* p = reinterpret_cast<const uint4*>(row) + 2 * c;
                 const uint4 v0 = p[0], v1 = p[1];
-                const uint32_t w[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
-#pragma unroll
-                for (int e = 0; e < 8; ++e) {
-                    x[2 * e] = bf16lo(w[e]);
-                    x[2 * e + 1] = bf16hi(w[e]);
-                }
+                w[0] = v0.x; w[1] = v0.y; w[2] = v0.z; w[3] = v0.w;
+                w[4] = v1.x; w[5] = v1.y; w[6] = v1.z; w[7] = v1.w;
             } else {
                 // augmented weight columns: element k >= K_src is column S[k - K_src]
                 const uint16_t* rw = reinterpret_cast<const uint16_t*>(row);
 #pragma unroll
-                for (int e = 0; e < 16; ++e)
-                    x[e] = __uint_as_float((uint32_t)rw[checked_channel(a.S, 16 * c + e - a.K_src, a.K_src)] << 16);
+                for (int e = 0; e < 8; ++e)
+                    w[e] = (uint32_t)rw[checked_channel(a.S, 16 * c + 2 * e - a.K_src, a.K_src)] |
+                           ((uint32_t)rw[checked_channel(a.S, 16 * c + 2 * e + 1 - a.K_src, a.K_src)] << 16);
             }
         } else {
 #pragma unroll
-            for (int e = 0; e < 16; ++e) x[e] = 0.0f;
+            for (int e = 0; e < 8; ++e) w[e] = 0;
         }
-        float bmax = 0.0f;
-#pragma unroll
-        for (int e = 0; e < 16; ++e) bmax = fmaxf(bmax, fabsf(x[e]));
+        float bmax = (token && live) ? bm[it] : bmax16(w);
 
         uint32_t w0 = 0, w1 = 0;  // 16 codes
         if constexpr (FMT == FMT_NVFP4) {
-            uint8_t sb = 0;
-            if (live) {
-                const float s2 = a.mode == 1 ? (a.static_s2 ? a.static_s2[r] : nvfp4_s2(rmax[i])) : tensor_s2;
-                sb = e4m3_rn_sat(__fdiv_rn(__fdiv_rn(bmax, 6.0f), s2));
-                if (sb != 0) {
-                    const float d = __fmul_rn(e4m3_value(sb), s2);
-                    const Bracket br = make_bracket(d);
-                    w0 = e2m1x8_div(x, d, br);
-                    w1 = e2m1x8_div(x + 8, d, br);
+            const RowConsts k = rc[i < nrows ? i : 0];
+            // block scale E4M3(RN(RN(bmax/6)/s2)) and quotients x/(scale*s2), by refined
+            // division on the hot path; operands outside its range go to IEEE division
+            const float u = div_refined(bmax, 6.0f, 0x1.555556p-3f);  // RN(1/6)
+            const uint8_t sb = live ? e4m3_rn_sat(div_refined(u, k.s2, k.rinv)) : 0;
+            const float d = sb ? __fmul_rn(e4m3_value(sb), k.s2) : 1.0f;
+            const float y = __frcp_rn(d);
+            w0 = e2m1x8_fast(w, pack2(-y), pack2(d));
+            w1 = e2m1x8_fast(w + 4, pack2(-y), pack2(d));
+            const bool slow = live && !(k.fast && bmax >= 0x1p-100f && d >= 0x1p-100f && d <= 0x1p100f &&
+                                        __fmul_rn(bmax, y) <= 0x1p60f);
+            uint8_t sbf = sb;
+            if (__any_sync(0xffffffffu, slow)) {
+                if (slow) {
+                    sbf = e4m3_rn_sat(__fdiv_rn(__fdiv_rn(bmax, 6.0f), k.s2));
+                    const float de = __fmul_rn(e4m3_value(sbf), k.s2);
+                    w0 = sbf ? e2m1x8_exact(make_uint4(w[0], w[1], w[2], w[3]), de) : 0u;
+                    w1 = sbf ? e2m1x8_exact(make_uint4(w[4], w[5], w[6], w[7]), de) : 0u;
                 }
             }
+            if (sbf == 0) {
+                w0 = 0;
+                w1 = 0;
+            }
             // gather 4 consecutive block scales (lanes l..l+3) into one word
-            const uint32_t b = sb;
+            const uint32_t b = sbf;
             const uint32_t b1 = __shfl_down_sync(0xffffffffu, b, 1);
             const uint32_t b2 = __shfl_down_sync(0xffffffffu, b, 2);
             const uint32_t b3 = __shfl_down_sync(0xffffffffu, b, 3);
@@ -262,9 +345,11 @@ __global__ void __launch_bounds__(256) quant_rows_kernel(QuantArgs a, int rows_p
                 const float inv = __uint_as_float((254u - code) << 23);  // 2^(127 - code)
                 float q0[8], q1[8];
 #pragma unroll
-                for (int e2 = 0; e2 < 8; ++e2) {
-                    q0[e2] = __fmul_rn(x[e2], inv);
-                    q1[e2] = __fmul_rn(x[8 + e2], inv);
+                for (int e2 = 0; e2 < 4; ++e2) {
+                    q0[2 * e2] = __fmul_rn(bf16lo(w[e2]), inv);
+                    q0[2 * e2 + 1] = __fmul_rn(bf16hi(w[e2]), inv);
+                    q1[2 * e2] = __fmul_rn(bf16lo(w[4 + e2]), inv);
+                    q1[2 * e2 + 1] = __fmul_rn(bf16hi(w[4 + e2]), inv);
                 }
                 w0 = e2m1x8(q0);
                 w1 = e2m1x8(q1);
@@ -279,16 +364,41 @@ __global__ void __launch_bounds__(256) quant_rows_kernel(QuantArgs a, int rows_p
             bmax = fmaxf(bmax, __shfl_xor_sync(0xffffffffu, bmax, 1));
             bmax = fmaxf(bmax, __shfl_xor_sync(0xffffffffu, bmax, 2));
             bmax = fmaxf(bmax, __shfl_xor_sync(0xffffffffu, bmax, 4));
-            const float sc = live ? __fdiv_rn(bmax, 7.0f) : 0.0f;
-            if (sc != 0.0f) {
-                const Bracket br = make_bracket(sc);
-                w0 = int4x8_div(x, sc, br);
-                w1 = int4x8_div(x + 8, sc, br);
+            const bool fast = bmax >= 0x1p-100f && bmax <= 0x1p100f;
+            float sc = live ? div_refined(bmax, 7.0f, 0x1.24924ap-3f) : 0.0f;  // RN(1/7)
+            const float y = __frcp_rn(sc > 0.0f ? sc : 1.0f);
+            w0 = int4x8_fast(w, pack2(-y), pack2(sc));
+            w1 = int4x8_fast(w + 4, pack2(-y), pack2(sc));
+            const bool slow = live && !fast;
+            if (__any_sync(0xffffffffu, slow)) {
+                if (slow) {
+                    sc = __fdiv_rn(bmax, 7.0f);
+                    w0 = sc != 0.0f ? int4x8_exact(make_uint4(w[0], w[1], w[2], w[3]), sc) : 0u;
+                    w1 = sc != 0.0f ? int4x8_exact(make_uint4(w[4], w[5], w[6], w[7]), sc) : 0u;
+                }
+            }
+            if (sc == 0.0f) {
+                w0 = 0;
+                w1 = 0;
             }
             if (valid && (c & 7) == 0) a.sfi[(size_t)(c >> 3) * a.sfi_ld + r] = sc;
         }
         if (live) *reinterpret_cast<uint2*>(a.codes + (size_t)r * a.ldc + 8 * c) = make_uint2(w0, w1);
+        i += di;
+        c += dc;
+        if (c >= nchunk) {
+            c -= nchunk;
+            ++i;
+        }
     }
+    __syncthreads();  // every thread is done with this buffer and with rmax/rc
+    if (t == 0) {
+        const int nb = bi + nbuf * gridDim.x;
+        if (nb < nblocks) issue_load(nb, buf);
+    }
+    }
+    if (*abort_flag && t == 0)  // wait for the loads still in flight
+        for (int b = 0; b < nbuf; ++b) mbar_wait_drain(&bars[b], 0, 100000000ull);
 }
 
 // ---------------------------------------------------------------------------
@@ -352,9 +462,16 @@ __global__ void __launch_bounds__(128) residual_kernel(ResidualArgs a) {
         sb = e4m3_rn_sat(__fdiv_rn(__fdiv_rn(bmax, 6.0f), s2));
         if (sb != 0) {
             const float d = __fmul_rn(e4m3_value(sb), s2);
-            const Bracket br = make_bracket(d);
-            w0 = e2m1x8_div(R, d, br);
-            w1 = e2m1x8_div(R + 8, d, br);
+            const float y = __frcp_rn(d);
+            const bool exact = !(d >= 0x1p-100f && d <= 0x1p100f && __fmul_rn(bmax, y) <= 0x1p60f);
+            float q0[8], q1[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+                q0[e] = exact ? __fdiv_rn(R[e], d) : div_refined(R[e], d, y);
+                q1[e] = exact ? __fdiv_rn(R[8 + e], d) : div_refined(R[8 + e], d, y);
+            }
+            w0 = e2m1x8(q0);
+            w1 = e2m1x8(q1);
         }
         *reinterpret_cast<uint2*>(a.codes + (size_t)r * a.ldc + (a.K >> 1) + 8 * b) = make_uint2(w0, w1);
     }
@@ -416,11 +533,16 @@ __global__ void __launch_bounds__(1024) compact_kernel(const int* selected, int 
 // Host launchers
 // ---------------------------------------------------------------------------
 template <int FMT, bool GATHER>
-static cudaError_t launch_quant_fmt(const QuantArgs& a, int rows_pad, cudaStream_t st) {
+static cudaError_t launch_quant_fmt(const QuantArgs& a, int rows_pad, int num_sms, cudaStream_t st) {
     const int row_bytes = a.K_src * 2;
-    int rpc = 32768 / row_bytes;                 // about 32 KB of rows per CTA
+    // One row block per CTA (about 32 KB of rows, several CTAs resident per
+    // SM): many warps in flight hide the latency of the per-item arithmetic.
+    int rpc = 32768 / row_bytes;
     rpc = rpc < 1 ? 1 : (rpc > 64 ? 64 : rpc);
-    const size_t smem = (size_t)rpc * row_bytes + 16 + 4 * rpc + 16;
+    const size_t buf = (size_t)rpc * row_bytes;
+    const int nbuf = 1;
+    const size_t smem = nbuf * buf + 8 * nbuf + 4 * rpc + sizeof(RowConsts) * rpc +
+                        (FMT == FMT_NVFP4 ? 4 * (size_t)rpc * (a.K / 16) : 0) + 16;
     if (smem > 200 * 1024) return cudaErrorInvalidValue;
     auto kern = quant_rows_kernel<FMT, GATHER>;
     static size_t attr = 0;
@@ -430,19 +552,23 @@ static cudaError_t launch_quant_fmt(const QuantArgs& a, int rows_pad, cudaStream
         attr = smem;
     }
     const int items = rpc * (a.K / 16);
-    int T = items < 256 ? (items + 31) / 32 * 32 : 256;
+    const int T = items < 256 ? (items + 31) / 32 * 32 : 256;
+    const int nblocks = (rows_pad + rpc - 1) / rpc;
+    const int grid = nblocks;
+    (void)num_sms;
     QuantArgs b = a;
     b.rows_pad = rows_pad;
-    kern<<<(rows_pad + rpc - 1) / rpc, T, smem, st>>>(b, rpc);
+    kern<<<grid, T, smem, st>>>(b, rpc, nbuf);
     return cudaGetLastError();
 }
 
-cudaError_t launch_quant(int fmt, bool gather, const QuantArgs& a, int rows_pad, cudaStream_t st) {
-    if (fmt == FMT_NVFP4) return gather ? launch_quant_fmt<FMT_NVFP4, true>(a, rows_pad, st)
-                                        : launch_quant_fmt<FMT_NVFP4, false>(a, rows_pad, st);
-    if (fmt == FMT_MXFP4) return gather ? launch_quant_fmt<FMT_MXFP4, true>(a, rows_pad, st)
-                                        : launch_quant_fmt<FMT_MXFP4, false>(a, rows_pad, st);
-    return gather ? launch_quant_fmt<FMT_INT4, true>(a, rows_pad, st) : launch_quant_fmt<FMT_INT4, false>(a, rows_pad, st);
+cudaError_t launch_quant(int fmt, bool gather, const QuantArgs& a, int rows_pad, int num_sms, cudaStream_t st) {
+    if (fmt == FMT_NVFP4) return gather ? launch_quant_fmt<FMT_NVFP4, true>(a, rows_pad, num_sms, st)
+                                        : launch_quant_fmt<FMT_NVFP4, false>(a, rows_pad, num_sms, st);
+    if (fmt == FMT_MXFP4) return gather ? launch_quant_fmt<FMT_MXFP4, true>(a, rows_pad, num_sms, st)
+                                        : launch_quant_fmt<FMT_MXFP4, false>(a, rows_pad, num_sms, st);
+    return gather ? launch_quant_fmt<FMT_INT4, true>(a, rows_pad, num_sms, st)
+                  : launch_quant_fmt<FMT_INT4, false>(a, rows_pad, num_sms, st);
 }
 
 cudaError_t launch_amax(const uint16_t* X, int M, int K, int ldx, float* out, int num_sms, cudaStream_t st) {

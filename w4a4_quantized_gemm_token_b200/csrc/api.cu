@@ -174,18 +174,6 @@ int setup_gemm(const w4a4_qtensor* A, const w4a4_qtensor* B, uint16_t* Y, int ld
     return rc;
 }
 
-// Split-K factor of the small-M variant: enough CTAs to cover every SM.
-void decode_split(int N, int K, int num_sms, int* splits, int* kps) {
-    const int KT = (K + kBK_FP4 - 1) / kBK_FP4;
-    const int ntiles = (N + kBM - 1) / kBM;
-    int want = (num_sms + ntiles - 1) / ntiles;
-    if (want < 1) want = 1;
-    if (want > KT) want = KT;
-    int per = (KT + want - 1) / want;
-    *kps = per;
-    *splits = (KT + per - 1) / per;
-}
-
 int run_gemm(const w4a4_qtensor* A, const w4a4_qtensor* B, uint16_t* Y, int ldy, float* partial, int num_sms,
              bool pdl, cudaStream_t st) {
     const bool decode = A->format != W4A4_INT4 && partial != nullptr;
@@ -196,9 +184,8 @@ int run_gemm(const w4a4_qtensor* A, const w4a4_qtensor* B, uint16_t* Y, int ldy,
     if (A->format == W4A4_INT4) {
         e = launch_gemm_int4(s.ta, s.tb, s.g, num_sms, pdl, st);
     } else if (decode) {
-        decode_split(s.g.N, s.g.K, num_sms, &s.g.splits, &s.g.k_tiles_per_split);
         s.g.partial = partial;
-        e = launch_gemm_fp4_decode(A->format == W4A4_NVFP4, s.ta, s.tb, s.g, pdl, st);
+        e = launch_gemm_fp4_decode(A->format == W4A4_NVFP4, s.ta, s.tb, s.g, num_sms, st);
     } else {
         e = launch_gemm_fp4(A->format == W4A4_NVFP4, s.ta, s.tb, s.g, num_sms, pdl, st);
     }
@@ -223,8 +210,10 @@ WsLayout ws_layout(int M, int N, int K, int fmt, int nS) {
     w.partial = w.s2 + align256(s2b);
     size_t pb = 0;
     if (fmt != W4A4_INT4 && M <= 16) {
-        const int KT = (cols + kBK_FP4 - 1) / kBK_FP4;
-        pb = (size_t)KT * M * N * sizeof(float);  // upper bound on splits x M x N
+        // FP32 segment partials of the small-M variant: [tiles][owners][16][128];
+        // the owner count grows with the SM count, bounded here for up to 1024 SMs
+        const int ntiles = (N + kBM - 1) / kBM;
+        pb = (size_t)ntiles * decode_max_owners(N, cols, 1024) * kBN_DEC * kBM * sizeof(float);
     }
     w.total = w.partial + align256(pb);
     return w;

@@ -1,27 +1,20 @@
-// Block-scaled FP4 GEMM on sm_100a tensor cores (tcgen05.mma kind::mxf4nvf4).
+// Small-M ("decode") block-scaled FP4 GEMM: Y[M,N] = X[M,K] W[N,K]^T for
+// M <= 16, bound by streaming the 4-bit weights from HBM.
 //
-// Y[m,n] = alpha_mn * sum_b sa[m,b] sb[n,b] sum_{k in b} ea[m,k] eb[n,k]: the
-// MMA applies the E4M3 (NVFP4, 16-element blocks) or E8M0 (MXFP4, 32-element
-// blocks) scales itself and accumulates in FP32 in tensor memory, so no
-// dequantization runs on the CUDA cores ("APEX4..." page, para 1 (MSD) and
-// "Depth Registers..." thelatestinai page, para 2 (APEX4) both locate the
-// cost of W4A4 in that dequantization).
-//
-// One CTA computes one 128 x BN output tile.  Warp roles:
-//   warp 0, lane 0  TMA producer: codes of A and B (128-byte swizzled K-major
-//                   tiles of 256 elements), scale atoms by bulk copy, into a
-//                   STAGES-deep shared-memory ring (full/empty mbarriers).
-//   warp 1          owns the tensor memory; lane 0 issues tcgen05.cp (scales
-//                   -> TMEM) and 4 MMAs (K=64 each) per stage, then commits
-//                   the stage back to the producer.
-//   warps 2..5      epilogue: TMEM -> registers (each warp its 32-lane
-//                   quarter), x alpha, bf16, 16-byte stores.
-// Every wait is bounded; on expiry the kernel records a timeout, drains its
-// own in-flight copies and MMAs, frees TMEM and returns.
-//
-// The decode variant (DECODE = true) swaps the operands: 128 weight rows take
-// the MMA's M side, the (<= 16) tokens its N side, and K is split across
-// CTAs; FP32 partial sums are reduced by a second kernel.
+// The weights take the MMA's M side (128 rows per tile) and the tokens its N
+// side (16), so one tcgen05.mma kind::mxf4nvf4 covers 128 x 16 x 64.  The
+// (weight tile, K-stage of 256) work units are split into equal contiguous
+// ranges, one per SM (stream-K), so every SM streams the same number of
+// weight bytes whatever N and K are.  A CTA accumulates in TMEM while its
+// range stays in one weight tile and writes an FP32 partial sum per tile
+// segment (double-buffered accumulators); a second kernel adds the segments
+// of each tile in a fixed order (deterministic), applies alpha and rounds to
+// bf16.  Launched as a programmatic dependent, the kernel starts streaming
+// weights while the activation quantizer still runs and waits only before
+// its first activation load.
+// Warp roles (256 threads): warp 0 lane 0 TMA producer (8-stage ring),
+// warp 1 TMEM owner + MMA issuer, warp 2 lane 0 scale-factor copies,
+// warps 4..7 epilogue (TMEM lane quarter = warp % 4).
 #include <cstdint>
 #include <cuda_bf16.h>
 
@@ -32,29 +25,24 @@ namespace w4a4 {
 
 __device__ int g_error_word = 0;
 
-template <int BN, int STAGES>
-struct Fp4Layout {
-    static constexpr int A_BYTES = kBM * 128;
-    static constexpr int B_BYTES = BN * 128;
-    static constexpr int SF_ATOM = 512;
-    static constexpr int SFA_BYTES = 4 * SF_ATOM;                  // <= 4 atoms per stage
-    static constexpr int SFB_HALVES = BN >= 128 ? BN / 128 : 1;    // 128-row scale atoms per B tile
-    static constexpr int SFB_BYTES = SFB_HALVES * 4 * SF_ATOM;
-    static constexpr int STAGE = A_BYTES + B_BYTES + SFA_BYTES + SFB_BYTES;
-    static constexpr int BAR_OFF = STAGES * STAGE;
-    static constexpr int SMEM = BAR_OFF + 256 + 1024;              // barriers + alignment slack
-    // TMEM columns: accumulator, then one scale-factor region per pipeline stage
-    // (SFA 16 columns, SFB 16 per 128 rows), so that copying the next stage's
-    // scales never waits for the MMAs still reading the previous ones.
-    static constexpr int SF_COLS = 16 + 16 * SFB_HALVES;
-    static constexpr int SFA_COL = BN;
-    static constexpr int SFB_COL = BN + 16;
-    static constexpr int TMEM_USED = BN + STAGES * SF_COLS;
-    static constexpr int TMEM_COLS = TMEM_USED <= 32 ? 32 : TMEM_USED <= 64 ? 64 : TMEM_USED <= 128 ? 128
-                                     : TMEM_USED <= 256 ? 256 : 512;
-    static_assert(STAGE % 1024 == 0, "stage must keep 1024-byte alignment of the swizzled tiles");
-    static_assert(TMEM_USED <= 512, "tensor memory holds 512 columns");
-};
+namespace dec {
+constexpr int BN = kBN_DEC;                 // tokens per MMA (16)
+constexpr int STAGES = 8;
+constexpr int A_BYTES = kBM * 128;          // weight tile, 16 KB
+constexpr int B_BYTES = BN * 128;           // token tile, 2 KB
+constexpr int ATOM = 512;
+constexpr int SFA_C = 4 * ATOM;
+constexpr int SFB_C = 4 * ATOM;
+constexpr int STAGE = A_BYTES + B_BYTES + SFA_C + SFB_C;
+constexpr int BAR_OFF = STAGES * STAGE;
+constexpr int SMEM = BAR_OFF + 512 + 1024;
+constexpr int SF_COLS = 32;                 // per stage: A 16 + B 16 columns
+constexpr int SF_COL0 = 2 * BN;             // after two accumulators of 16 columns
+constexpr int TMEM_COLS = 512;
+constexpr int THREADS = 256;
+static_assert(STAGE % 1024 == 0, "stages keep the 1024-byte alignment of swizzled tiles");
+static_assert(SF_COL0 + STAGES * SF_COLS <= TMEM_COLS, "tensor memory holds 512 columns");
+}  // namespace dec
 
 __device__ __forceinline__ void tmem_ld_32x32b_x16(uint32_t taddr, uint32_t (&r)[16]) {
     asm volatile(
@@ -65,225 +53,250 @@ __device__ __forceinline__ void tmem_ld_32x32b_x16(uint32_t taddr, uint32_t (&r)
         : "r"(taddr));
 }
 
-template <bool NV, int BN, int STAGES, bool DECODE>
-__global__ void __launch_bounds__(192, 1)
-    gemm_fp4_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB, GemmArgs g) {
-    using L = Fp4Layout<BN, STAGES>;
+// First unit of CTA c when U units are split into G equal contiguous ranges.
+__host__ __device__ __forceinline__ long long unit_begin(int c, long long U, int G) { return (long long)c * U / G; }
+
+// The CTA whose range holds unit u.
+__device__ __forceinline__ int unit_owner(long long u, long long U, int G) {
+    int c = (int)(u * G / U);
+    while (c + 1 < G && unit_begin(c + 1, U, G) <= u) ++c;
+    while (c > 0 && unit_begin(c, U, G) > u) --c;
+    return c;
+}
+
+template <bool NV>
+__global__ void __launch_bounds__(dec::THREADS, 1)
+    gemm_fp4_decode_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmX,
+                           GemmArgs g) {
+    using namespace dec;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    uint64_t* full = reinterpret_cast<uint64_t*>(smem + L::BAR_OFF);
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem + BAR_OFF);
     uint64_t* empty = full + STAGES;
-    uint64_t* accf = empty + STAGES;
-    uint64_t* drain = accf + 1;
-    uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(drain + 1);
+    uint64_t* sfull = empty + STAGES;
+    uint64_t* accf = sfull + STAGES;  // [2]
+    uint64_t* acce = accf + 2;        // [2]
+    uint64_t* drain = acce + 2;
+    uint64_t* drain2 = drain + 1;
+    uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(drain2 + 1);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int KT = (g.K + kBK_FP4 - 1) / kBK_FP4;
-    // A side = rows of the MMA's M (activations, or weights when DECODE)
-    const int a_rows = DECODE ? g.N : g.M;
-    const int b_rows = DECODE ? g.M : g.N;
-    int a_tile, b_tile, kt_begin, kt_end, split = 0;
-    if constexpr (!DECODE) {
-        // grouped raster: 8 consecutive A tiles share each B tile within a wave
-        const int num_a = (a_rows + kBM - 1) / kBM, num_b = (b_rows + BN - 1) / BN;
-        const int G = 8;
-        const int per_group = G * num_b;
-        const int grp = blockIdx.x / per_group, first = grp * G;
-        const int gsz = min(G, num_a - first);
-        const int in = blockIdx.x - grp * per_group;
-        a_tile = first + in % gsz;
-        b_tile = in / gsz;
-        kt_begin = 0;
-        kt_end = KT;
-    } else {
-        a_tile = blockIdx.x;
-        b_tile = 0;
-        split = blockIdx.y;
-        kt_begin = split * g.k_tiles_per_split;
-        kt_end = min(KT, kt_begin + g.k_tiles_per_split);
-    }
-    const uint8_t* sfa_g = DECODE ? g.sfb : g.sfa;
-    const uint8_t* sfb_g = DECODE ? g.sfa : g.sfb;
+    const int ntiles = (g.N + kBM - 1) / kBM;
+    const long long U = (long long)ntiles * KT;
+    const int G = gridDim.x;
+    const long long u0 = unit_begin(blockIdx.x, U, G), u1 = unit_begin(blockIdx.x + 1, U, G);
+    const int nunits = (int)(u1 - u0);
     const uint64_t limit = g.wait_limit_ns;
+    // weights are the MMA's A side, tokens its B side
+    const uint8_t* sfw = g.sfb;
+    const uint8_t* sfx = g.sfa;
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < STAGES; ++s) {
             mbar_init(&full[s], 1);
             mbar_init(&empty[s], 1);
+            mbar_init(&sfull[s], 1);
         }
-        mbar_init(accf, 1);
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&accf[b], 1);
+            mbar_init(&acce[b], 4);
+        }
         mbar_init(drain, 1);
+        mbar_init(drain2, 1);
         *abort_flag = 0;
         fence_mbar_init();
     }
     if (warp == 0 && lane == 0) {
-        tma_prefetch_desc(&tmA);
-        tma_prefetch_desc(&tmB);
+        tma_prefetch_desc(&tmW);
+        tma_prefetch_desc(&tmX);
     }
     if (warp == 1) {
-        tmem_alloc(tmem_holder, L::TMEM_COLS);
+        tmem_alloc(tmem_holder, TMEM_COLS);
         tmem_relinquish();
     }
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_holder;
-    pdl_wait();  // operands written by the preceding kernel are visible from here on
+    pdl_launch_dependents();  // the reduction kernel may be scheduled; it waits for this grid
 
     if (warp == 0) {
         if (lane == 0) {
             // ------------------------------ producer ------------------------------
-            int i = 0;
-            for (int kt = kt_begin; kt < kt_end; ++kt, ++i) {
-                const int s = i % STAGES, n = i / STAGES;
-                if (i >= STAGES && !mbar_wait(&empty[s], (n - 1) & 1, limit, abort_flag)) break;
-                if (kt == g.skip_k_tile) continue;  // test hook: this stage never fills
-                uint8_t* st = smem + s * L::STAGE;
-                const int nk = min(4, (g.K - kt * kBK_FP4) / 64);              // MMAs in this stage
-                const int atoms = NV ? nk : (nk + 1) / 2;                      // scale atoms per 128 rows
-                const int atom_k0 = NV ? kt * 4 : kt * 2;
-                const uint32_t sf_bytes = atoms * L::SF_ATOM;
-                int halves = 0;
-#pragma unroll
-                for (int h = 0; h < L::SFB_HALVES; ++h)
-                    if ((b_tile * L::SFB_HALVES + h) * 128 < max(b_rows, 1)) ++halves;
-                mbar_arrive_expect_tx(&full[s], L::A_BYTES + L::B_BYTES + sf_bytes * (1 + halves));
-                tma_load_2d(st, &tmA, kt * 128, a_tile * kBM, &full[s]);
-                tma_load_2d(st + L::A_BYTES, &tmB, kt * 128, b_tile * BN, &full[s]);
-                bulk_load(st + L::A_BYTES + L::B_BYTES,
-                          sfa_g + ((size_t)a_tile * g.sf_col_atoms + atom_k0) * L::SF_ATOM, sf_bytes, &full[s]);
-                for (int h = 0; h < halves; ++h)
-                    bulk_load(st + L::A_BYTES + L::B_BYTES + L::SFA_BYTES + h * 4 * L::SF_ATOM,
-                              sfb_g + ((size_t)(b_tile * L::SFB_HALVES + h) * g.sf_col_atoms + atom_k0) * L::SF_ATOM,
-                              sf_bytes, &full[s]);
+            auto atoms_of = [&](int kt, int& atoms, int& atom_k0) {
+                const int nk = min(4, (g.K - kt * kBK_FP4) / 64);
+                atoms = NV ? nk : (nk + 1) / 2;
+                atom_k0 = NV ? kt * 4 : kt * 2;
+            };
+            auto load_w = [&](long long u, int s) {
+                const int nt = (int)(u / KT), kt = (int)(u % KT);
+                int atoms, k0;
+                atoms_of(kt, atoms, k0);
+                uint8_t* st = smem + s * STAGE;
+                mbar_arrive_expect_tx(&full[s], (uint32_t)(A_BYTES + B_BYTES + 2 * atoms * ATOM));
+                tma_load_2d(st, &tmW, kt * 128, nt * kBM, &full[s]);
+                bulk_load(st + A_BYTES + B_BYTES, sfw + ((size_t)nt * g.sf_col_atoms + k0) * ATOM, atoms * ATOM,
+                          &full[s]);
+            };
+            auto load_x = [&](long long u, int s) {
+                const int kt = (int)(u % KT);
+                int atoms, k0;
+                atoms_of(kt, atoms, k0);
+                uint8_t* st = smem + s * STAGE;
+                tma_load_2d(st + A_BYTES, &tmX, kt * 128, 0, &full[s]);
+                bulk_load(st + A_BYTES + B_BYTES + SFA_C, sfx + (size_t)k0 * ATOM, atoms * ATOM, &full[s]);
+            };
+            // stream the first weight tiles before the activations are known to be ready
+            const int pre = min(STAGES, nunits);
+            int it = 0;
+            for (; it < pre; ++it)
+                if (it != g.skip_k_tile) load_w(u0 + it, it);
+            pdl_wait();
+            for (int j = 0; j < pre; ++j)
+                if (j != g.skip_k_tile) load_x(u0 + j, j);
+            for (; it < nunits; ++it) {
+                const int s = it % STAGES, n = it / STAGES;
+                if (!mbar_wait(&empty[s], (n - 1) & 1, limit, abort_flag)) break;
+                if (it == g.skip_k_tile) continue;  // test hook: this stage never fills
+                load_w(u0 + it, s);
+                load_x(u0 + it, s);
             }
-            if (*abort_flag) {
-                // wait for the copies this thread still has in flight
-                const int issued = i;
-                for (int j = max(0, issued - STAGES); j < issued; ++j)
-                    if (kt_begin + j != g.skip_k_tile)
-                        mbar_wait_drain(&full[j % STAGES], (j / STAGES) & 1, 100000000ull);
-            }
+            if (*abort_flag)
+                for (int j = max(0, it - STAGES); j < it; ++j)
+                    mbar_wait_drain(&full[j % STAGES], (j / STAGES) & 1, 100000000ull);
         }
     } else if (warp == 1) {
         if (lane == 0) {
             // ------------------------------ MMA issuer ------------------------------
-            const uint32_t acc = tmem;
-            constexpr int MMA_N = BN;
-            int i = 0;
             bool ok = true;
-            for (int kt = kt_begin; kt < kt_end; ++kt, ++i) {
-                const int s = i % STAGES, n = i / STAGES;
+            int it = 0, seg = 0;
+            long long u = u0;
+            while (u < u1 && ok) {
+                const int nt = (int)(u / KT);
+                const long long sbeg = u, send = min(u1, (long long)(nt + 1) * KT);
+                const int buf = seg & 1;
+                if (seg >= 2 && !mbar_wait(&acce[buf], ((seg >> 1) - 1) & 1, limit, abort_flag)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                for (; u < send; ++u, ++it) {
+                    const int s = it % STAGES, n = it / STAGES;
+                    if (!mbar_wait(&sfull[s], n & 1, limit, abort_flag)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const int kt = (int)(u % KT);
+                    const uint32_t sA = smem_u32(smem + s * STAGE), sB = sA + A_BYTES;
+                    const uint32_t sfa_t = tmem + SF_COL0 + s * SF_COLS, sfb_t = sfa_t + 16;
+                    const int nk = min(4, (g.K - kt * kBK_FP4) / 64);
+                    for (int j = 0; j < nk; ++j) {
+                        const int sfid = NV ? 0 : (j & 1) * 2;
+                        const int aj = NV ? j : (j >> 1);
+                        mma_fp4<NV>(tmem + buf * BN, desc_kmajor_sw128(sA + 32 * j), desc_kmajor_sw128(sB + 32 * j),
+                                    idesc_fp4(kBM, BN, !NV, sfid, sfid), (sfa_t + 4 * aj) | ((uint32_t)sfid << 30),
+                                    (sfb_t + 4 * aj) | ((uint32_t)sfid << 30), (u > sbeg || j > 0) ? 1u : 0u);
+                    }
+                    tc_commit(&empty[s]);
+                }
+                if (!ok) break;
+                tc_commit(&accf[buf]);
+                ++seg;
+            }
+            if (!ok) {
+                tc_commit(drain);
+                mbar_wait_drain(drain, 0, 100000000ull);
+            }
+        }
+    } else if (warp == 2) {
+        if (lane == 0) {
+            // ------------------------- scale-factor copies -------------------------
+            bool ok = true;
+            for (int it = 0; it < nunits; ++it) {
+                const int s = it % STAGES, n = it / STAGES;
                 if (!mbar_wait(&full[s], n & 1, limit, abort_flag)) {
                     ok = false;
                     break;
                 }
                 tc_fence_after();
-                const uint8_t* st = smem + s * L::STAGE;
-                const uint32_t sfa_t = tmem + L::SFA_COL + s * L::SF_COLS;
-                const uint32_t sfb_t = tmem + L::SFB_COL + s * L::SF_COLS;
-                const uint32_t sA = smem_u32(st), sB = smem_u32(st + L::A_BYTES);
-                const uint32_t sSFA = smem_u32(st + L::A_BYTES + L::B_BYTES);
-                const uint32_t sSFB = sSFA + L::SFA_BYTES;
+                const int kt = (int)((u0 + it) % KT);
                 const int nk = min(4, (g.K - kt * kBK_FP4) / 64);
                 const int atoms = NV ? nk : (nk + 1) / 2;
+                const uint32_t ca = smem_u32(smem + s * STAGE + A_BYTES + B_BYTES), cb = ca + SFA_C;
+                const uint32_t sfa_t = tmem + SF_COL0 + s * SF_COLS, sfb_t = sfa_t + 16;
                 for (int j = 0; j < atoms; ++j) {
-                    tc_cp_32x128b_x4(sfa_t + 4 * j, desc_sf_32x16(sSFA + j * L::SF_ATOM));
-#pragma unroll
-                    for (int h = 0; h < L::SFB_HALVES; ++h)
-                        tc_cp_32x128b_x4(sfb_t + 4 * L::SFB_HALVES * j + 4 * h,
-                                         desc_sf_32x16(sSFB + h * 4 * L::SF_ATOM + j * L::SF_ATOM));
+                    tc_cp_32x128b_x4(sfa_t + 4 * j, desc_sf_32x16(ca + j * ATOM));
+                    tc_cp_32x128b_x4(sfb_t + 4 * j, desc_sf_32x16(cb + j * ATOM));
                 }
-                for (int j = 0; j < nk; ++j) {
-                    const uint64_t ad = desc_kmajor_sw128(sA + 32 * j);
-                    const uint64_t bd = desc_kmajor_sw128(sB + 32 * j);
-                    const int atom = NV ? j : j >> 1;
-                    const int sfid = NV ? 0 : (j & 1) * 2;
-                    const uint32_t ta = (sfa_t + 4 * atom) | ((uint32_t)sfid << 30);
-                    const uint32_t tb = (sfb_t + 4 * L::SFB_HALVES * atom) | ((uint32_t)sfid << 30);
-                    mma_fp4<NV>(acc, ad, bd, idesc_fp4(kBM, MMA_N, !NV, sfid, sfid), ta, tb,
-                                (kt > kt_begin || j > 0) ? 1u : 0u);
-                }
-                tc_commit(&empty[s]);
+                tc_commit(sfull + s);
             }
-            if (ok) {
-                tc_commit(accf);
-            } else {
-                tc_commit(drain);  // let every MMA already issued finish before TMEM is freed
-                mbar_wait_drain(drain, 0, 100000000ull);
+            if (!ok) {
+                tc_commit(drain2);
+                mbar_wait_drain(drain2, 0, 100000000ull);
             }
         }
-    } else {
+    } else if (warp >= 4) {
         // ------------------------------ epilogue ------------------------------
-        const int q = warp & 3;  // TMEM lane quarter this warp may access
-        const bool ok = mbar_wait(accf, 0, limit, abort_flag);
-        tc_fence_after();
-        const int row = q * 32 + lane;
-        const uint32_t taddr = tmem + ((uint32_t)(q * 32) << 16);
-        if (ok) {
-            if constexpr (!DECODE) {
-                const int m = a_tile * kBM + row;
-                float alpha = 1.0f;
-                if (NV && m < g.M) alpha = __fmul_rn(g.s2a[g.s2a_per_row ? m : 0], g.s2b[0]);
-#pragma unroll 1
-                for (int ch = 0; ch < BN / 32; ++ch) {
-                    uint32_t r[32];
-                    tmem_ld_32x32b_x32(taddr + 32 * ch, r);
-                    tmem_ld_wait();
-                    const int n0 = b_tile * BN + 32 * ch;
-                    if (m < g.M && n0 < g.N) {
-                        uint32_t pk[16];
+        // segment partial sums -> workspace slot (tile, owner offset): [16 tokens][128 rows] FP32
+        const int q = warp & 3;
+        int seg = 0;
+        long long u = u0;
+        while (u < u1) {
+            const int nt = (int)(u / KT);
+            const long long send = min(u1, (long long)(nt + 1) * KT);
+            const int buf = seg & 1;
+            if (!mbar_wait(&accf[buf], (seg >> 1) & 1, limit, abort_flag, 20000)) break;
+            tc_fence_after();
+            uint32_t r[16];
+            tmem_ld_32x32b_x16(tmem + ((uint32_t)(q * 32) << 16) + buf * BN, r);
+            tmem_ld_wait();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&acce[buf]);
+            const int first = unit_owner((long long)nt * KT, U, G);
+            float* slot = g.partial + ((size_t)nt * g.splits + (blockIdx.x - first)) * (BN * kBM);
+            const int row = q * 32 + lane;
 #pragma unroll
-                        for (int e = 0; e < 16; ++e) {
-                            __nv_bfloat162 h = __floats2bfloat162_rn(__fmul_rn(__uint_as_float(r[2 * e]), alpha),
-                                                                     __fmul_rn(__uint_as_float(r[2 * e + 1]), alpha));
-                            pk[e] = *reinterpret_cast<uint32_t*>(&h);
-                        }
-                        uint4* dst = reinterpret_cast<uint4*>(g.Y + (size_t)m * g.ldy + n0);
-#pragma unroll
-                        for (int v = 0; v < 4; ++v) dst[v] = make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
-                    }
-                }
-            } else {
-                const int n = a_tile * kBM + row;  // weight row = output column
-                uint32_t r[16];
-                tmem_ld_32x32b_x16(taddr, r);
-                tmem_ld_wait();
-                if (n < g.N) {
-                    float* out = g.partial + (size_t)split * g.M * g.N + n;
-#pragma unroll
-                    for (int j = 0; j < 16; ++j)
-                        if (j < g.M) out[(size_t)j * g.N] = __uint_as_float(r[j]);
-                }
-            }
+            for (int t = 0; t < BN; ++t) slot[t * kBM + row] = __uint_as_float(r[t]);
+            u = send;
+            ++seg;
         }
     }
     tc_fence_before();
     __syncthreads();
     if (warp == 1) {
         tc_fence_after();
-        tmem_dealloc(tmem, L::TMEM_COLS);
+        tmem_dealloc(tmem, TMEM_COLS);
     }
 }
 
-// Sum the split-K partials, apply alpha, round to bf16.
+// Y[m, n] = bf16(alpha_m * sum of the tile's segment partials, in owner order).
 template <bool NV>
-__global__ void __launch_bounds__(256) splitk_reduce_kernel(GemmArgs g) {
-    const long long idx = blockIdx.x * 256LL + threadIdx.x;
-    const long long total = (long long)g.M * g.N;
-    if (idx >= total) return;
-    const int m = (int)(idx / g.N), n = (int)(idx % g.N);
-    float acc = 0.0f;
-    for (int s = 0; s < g.splits; ++s) acc += g.partial[(size_t)s * total + idx];
-    float alpha = NV ? __fmul_rn(g.s2a[g.s2a_per_row ? m : 0], g.s2b[0]) : 1.0f;
-    __nv_bfloat16 h = __float2bfloat16_rn(__fmul_rn(acc, alpha));
-    g.Y[(size_t)m * g.ldy + n] = *reinterpret_cast<uint16_t*>(&h);
+__global__ void __launch_bounds__(256) decode_reduce_kernel(GemmArgs g, int grid_g) {
+    pdl_wait();
+    const int KT = (g.K + kBK_FP4 - 1) / kBK_FP4;
+    const int ntiles = (g.N + kBM - 1) / kBM;
+    const long long U = (long long)ntiles * KT;
+    const int nt = blockIdx.x;
+    const int first = unit_owner((long long)nt * KT, U, grid_g);
+    const int last = unit_owner((long long)(nt + 1) * KT - 1, U, grid_g);
+    for (int idx = threadIdx.x; idx < dec::BN * kBM; idx += blockDim.x) {
+        const int t = idx / kBM, row = idx % kBM;
+        const int n = nt * kBM + row;
+        if (t >= g.M || n >= g.N) continue;
+        float acc = 0.0f;
+        for (int c = first; c <= last; ++c)
+            acc += g.partial[((size_t)nt * g.splits + (c - first)) * (dec::BN * kBM) + idx];
+        const float alpha = NV ? __fmul_rn(g.s2a[g.s2a_per_row ? t : 0], g.s2b[0]) : 1.0f;
+        __nv_bfloat16 h = __float2bfloat16_rn(__fmul_rn(acc, alpha));
+        g.Y[(size_t)t * g.ldy + n] = *reinterpret_cast<uint16_t*>(&h);
+    }
 }
 
-template <typename Kern>
-static cudaError_t launch_ex(Kern kern, dim3 grid, dim3 block, size_t smem, bool pdl, cudaStream_t st,
-                             const CUtensorMap& a, const CUtensorMap& b, const GemmArgs& g) {
+static cudaError_t launch_pdl(const void* kern, dim3 grid, dim3 block, size_t smem, cudaStream_t st, void** args) {
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = grid;
     cfg.blockDim = block;
@@ -293,33 +306,49 @@ static cudaError_t launch_ex(Kern kern, dim3 grid, dim3 block, size_t smem, bool
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
-    cfg.numAttrs = pdl ? 1 : 0;
-    return cudaLaunchKernelEx(&cfg, kern, a, b, g);
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelExC(&cfg, kern, args);
+}
+
+int decode_grid(int N, int K, int num_sms) {
+    const long long U = (long long)((N + kBM - 1) / kBM) * ((K + kBK_FP4 - 1) / kBK_FP4);
+    return (int)(U < num_sms ? U : num_sms);
+}
+
+int decode_max_owners(int N, int K, int num_sms) {
+    const int KT = (K + kBK_FP4 - 1) / kBK_FP4;
+    const long long U = (long long)((N + kBM - 1) / kBM) * KT;
+    const int G = decode_grid(N, K, num_sms);
+    const long long per = U / G;  // every range holds per or per + 1 units
+    return (int)((KT + per - 1) / per) + 1;
 }
 
 template <bool NV>
-static cudaError_t launch_dec_t(const CUtensorMap& tmW, const CUtensorMap& tmX, const GemmArgs& g, bool pdl,
+static cudaError_t launch_dec_t(const CUtensorMap& tmW, const CUtensorMap& tmX, const GemmArgs& g0, int num_sms,
                                 cudaStream_t st) {
-    constexpr int STAGES = 8;
-    using L = Fp4Layout<kBN_DEC, STAGES>;
-    auto kern = gemm_fp4_kernel<NV, kBN_DEC, STAGES, true>;
+    auto kern = gemm_fp4_decode_kernel<NV>;
     static bool attr_set = false;
     if (!attr_set) {
-        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::SMEM);
+        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, dec::SMEM);
         if (e != cudaSuccess) return e;
         attr_set = true;
     }
-    dim3 grid((g.N + kBM - 1) / kBM, g.splits);
-    cudaError_t e = launch_ex(kern, grid, dim3(192), L::SMEM, pdl, st, tmW, tmX, g);
+    GemmArgs g = g0;
+    const int G = decode_grid(g.N, g.K, num_sms);
+    g.splits = decode_max_owners(g.N, g.K, num_sms);  // slots per weight tile in the workspace
+    CUtensorMap a = tmW, b = tmX;
+    void* args[] = {&a, &b, &g};
+    cudaError_t e = launch_pdl(reinterpret_cast<const void*>(kern), dim3(G), dim3(dec::THREADS), dec::SMEM, st, args);
     if (e != cudaSuccess) return e;
-    const long long total = (long long)g.M * g.N;
-    splitk_reduce_kernel<NV><<<(unsigned)((total + 255) / 256), 256, 0, st>>>(g);
-    return cudaGetLastError();
+    int gg = G;
+    void* rargs[] = {&g, &gg};
+    return launch_pdl(reinterpret_cast<const void*>(decode_reduce_kernel<NV>), dim3((g.N + kBM - 1) / kBM),
+                      dim3(256), 0, st, rargs);
 }
 
 cudaError_t launch_gemm_fp4_decode(bool nvfp4, const CUtensorMap& tmW, const CUtensorMap& tmX, const GemmArgs& g,
-                                   bool pdl, cudaStream_t st) {
-    return nvfp4 ? launch_dec_t<true>(tmW, tmX, g, pdl, st) : launch_dec_t<false>(tmW, tmX, g, pdl, st);
+                                   int num_sms, cudaStream_t st) {
+    return nvfp4 ? launch_dec_t<true>(tmW, tmX, g, num_sms, st) : launch_dec_t<false>(tmW, tmX, g, num_sms, st);
 }
 
 }  // namespace w4a4

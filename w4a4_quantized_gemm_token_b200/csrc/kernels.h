@@ -71,11 +71,14 @@ cudaError_t launch_select(const uint16_t* X, int Mc, int K, int ldx, int nS, int
 // 128 x bn (B) bytes.  pdl: launched as a programmatic dependent.
 cudaError_t launch_gemm_fp4(bool nvfp4, const CUtensorMap& tmA, const CUtensorMap& tmB, const GemmArgs& g,
                             int num_sms, bool pdl, cudaStream_t st);
-// Small-M variant: weights take the MMA's M side (128 rows per tile), the
-// tokens its N side (16), K is split across CTAs; FP32 partial sums go to
-// g.partial [splits][M][N] and a second kernel reduces them into Y.
+// Small-M variant (M <= 16): weights take the MMA's M side (128 rows per tile),
+// the tokens its N side; the (tile, K-stage) units are split evenly over the
+// SMs, FP32 segment partials go to g.partial and a second kernel reduces them
+// into Y.  Both kernels are programmatic dependents of the preceding launch.
 cudaError_t launch_gemm_fp4_decode(bool nvfp4, const CUtensorMap& tmW, const CUtensorMap& tmX, const GemmArgs& g,
-                                   bool pdl, cudaStream_t st);
+                                   int num_sms, cudaStream_t st);
+// Partial-sum slots per weight tile of the small-M variant on `num_sms` SMs.
+int decode_max_owners(int N, int K, int num_sms);
 // INT4-g128 GEMM on the 8-bit integer MMA with per-group FP32 rescaling.
 cudaError_t launch_gemm_int4(const CUtensorMap& tmA, const CUtensorMap& tmB, const GemmArgs& g, int num_sms,
                              bool pdl, cudaStream_t st);

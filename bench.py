@@ -162,17 +162,37 @@ def to_dev(bits, device):
     return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).to(device).view(torch.bfloat16)
 
 
-def time_loop(fn, iters, stream):
-    """Average device time (ms) of fn() over iters launches, CUDA events on `stream`."""
+def time_loop(fn, iters, stream, flush=None):
+    """Average device time (ms) of fn() over iters launches, CUDA events on `stream`.
+
+    With `flush` (a device buffer larger than L2) each launch is timed on its
+    own between events, after the buffer has been overwritten, so inputs that
+    would fit in L2 are read from HBM every time."""
     import torch
-    s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     torch.cuda.synchronize()
-    s.record(stream)
-    for _ in range(iters):
+    if flush is None:
+        s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        s.record(stream)
+        for _ in range(iters):
+            fn()
+        e.record(stream)
+        e.synchronize()
+        return s.elapsed_time(e) / iters
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(iters)]
+    for (s, e) in evs:
+        flush.fill_(1)
+        s.record(stream)
         fn()
-    e.record(stream)
-    e.synchronize()
-    return s.elapsed_time(e) / iters
+        e.record(stream)
+    torch.cuda.synchronize()
+    return sum(s.elapsed_time(e) for (s, e) in evs) / iters
+
+
+def l2_flush_buffer(dev):
+    """A buffer twice the size of L2 (written between timed launches)."""
+    import torch
+    l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+    return torch.empty(2 * l2 // 4, dtype=torch.int32, device=dev)
 
 
 def run_ours(args, rank, world):
@@ -317,14 +337,32 @@ def extra_rows(args, dev, stream, P):
     it = max(5, args.steps)
     want = lambda name: args.only is None or args.only == name
 
+    # the block-scaled GEMM alone on the Llama shapes (the profiling case)
+    for li, (name, K, N) in enumerate(LLAMA if args.only == "gemm" else []):
+        if args.shape and name != args.shape:
+            continue
+        M = args.tokens
+        Wq = w4.quantize_weight(to_dev(synth.weights("llama2_70b", N, K, seed=0, tensor_id=100 + li), dev), w4.NVFP4)
+        X = to_dev(synth.activations("llama2_70b", M, K, seed=0, tensor_id=200 + li), dev)
+        Xq = w4.quantize_act(X, w4.NVFP4, w4.SCALE_TOKEN)
+        Y = torch.empty(M, N, dtype=torch.bfloat16, device=dev)
+        for _ in range(args.warmup):
+            w4.gemm(Xq, Wq, Y)
+        ms = time_loop(lambda: w4.gemm(Xq, Wq, Y), args.steps, stream)
+        out[f"gemm_nvfp4_{name}_m{M}"] = {"TFLOPS": round(2.0 * M * N * K / (ms * 1e-3) / 1e12, 1),
+                                          "us": round(ms * 1e3, 2)}
+        del Wq, X, Xq, Y
+
     # activation quantizer, per-token NVFP4 (and MXFP4 / INT4), Llama qkv and w2 inputs
+    # (each launch timed after an L2 flush: the qkv input alone would fit in L2)
+    flush = l2_flush_buffer(dev) if want("quant") else None
     for (name, M, K) in [] if not want("quant") else [("qkv_in", args.tokens, 8192), ("w2_in", args.tokens, 28672)]:
         X = to_dev(synth.activations("llama2_70b", M, K, seed=3), dev)
         for fmt, g, sb in [(w4.NVFP4, 16, 1), (w4.MXFP4, 32, 1), (w4.INT4, 128, 4)]:
             q = w4.QTensor(fmt, M, K, w4.SCALE_TOKEN if fmt == w4.NVFP4 else 0, dev)
             f = lambda: w4.quantize_act(X, fmt, w4.SCALE_TOKEN, out=q)
             f()
-            ms = time_loop(f, it, stream)
+            ms = time_loop(f, it, stream, flush)
             byts = 2 * M * K + M * K / 2 + M * K / g * sb + (4 * M if fmt == w4.NVFP4 else 0)
             key = {w4.NVFP4: "nvfp4_token", w4.MXFP4: "mxfp4", w4.INT4: "int4"}[fmt]
             out[f"quant_{key}_{name}"] = {"GB/s": round(byts / ms / 1e6, 1), "frac_hbm": round(byts / ms / 1e6 / hbm, 3),
@@ -332,10 +370,11 @@ def extra_rows(args, dev, stream, P):
         q = w4.QTensor(w4.NVFP4, M, K, w4.SCALE_TENSOR, dev)
         f = lambda: w4.quantize_act(X, w4.NVFP4, w4.SCALE_TENSOR, out=q)
         f()
-        ms = time_loop(f, it, stream)
+        ms = time_loop(f, it, stream, flush)
         byts = 4 * M * K + M * K / 2 + M * K / 16
         out[f"quant_nvfp4_tensor_2pass_{name}"] = {"GB/s": round(byts / ms / 1e6, 1), "us": round(ms * 1e3, 2)}
         del X
+    del flush
 
     # decode: M = 1 and 16 over the layer (weights streamed from HBM)
     Ws = []
@@ -432,9 +471,10 @@ def main():
     ap.add_argument("--cpu-rows", type=int, default=8, help="cpu_baseline sample: tokens")
     ap.add_argument("--cpu-cols", type=int, default=4096, help="cpu_baseline sample: output columns")
     ap.add_argument("--no-rows", action="store_true", help="skip the secondary rows")
-    ap.add_argument("--only", choices=["quant", "decode", "int4", "aug", "mxfp4"], default=None,
+    ap.add_argument("--only", choices=["gemm", "quant", "decode", "int4", "aug", "mxfp4"], default=None,
                     help="run only one secondary row (for profiling) and print it")
     ap.add_argument("--no-cpu", action="store_true", help="skip the oracle CPU baseline")
+    ap.add_argument("--shape", default=None, help="--only gemm: one Llama linear (qkv, o, w1, w3, w2)")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)
 

@@ -188,7 +188,8 @@ int w4a4_augment_residual(const uint16_t* X, int M, int K, int ldx,
  * Offline channel selection for the augmentation: the nS channels with the
  * largest max|x| over the Mc calibration rows Xcal[Mc,K] (device bf16, row
  * stride ldx), ties to the lower index, written ascending to S_out (device
- * int32[nS]).  ws: device workspace of at least 4*K bytes.
+ * int32[nS]).  ws: device workspace of at least 8*K bytes (per-channel
+ * maxima and ranks).
  */
 int w4a4_select_channels(const uint16_t* Xcal, int Mc, int K, int ldx, int nS,
                          int32_t* S_out, void* ws, size_t ws_bytes, void* stream);

@@ -173,6 +173,29 @@ int w4a4_linear(const uint16_t* X, int M, int K, int ldx,
                 uint16_t* Y, int ldy, void* ws, size_t ws_bytes, void* stream);
 
 /*
+ * w4a4_linear without a caller workspace (the pages have no counterpart: it
+ * only changes where the scratch lives).  Same operation, arguments, layout
+ * and results as w4a4_linear; the scratch is a static device array inside
+ * this library, W4A4_NOALLOC_SCRATCH_BYTES per device, and the call
+ * allocates nothing.  It serves callers that hold no device allocator and so
+ * cannot provide a workspace.
+ *  - Sizes whose w4a4_linear_workspace() exceeds W4A4_NOALLOC_SCRATCH_BYTES
+ *    return W4A4_ERR_WORKSPACE and launch nothing (16 MiB covers, e.g., every
+ *    Llama-2-70B-sized linear at M <= 16, the small-M decode case).
+ *  - The first call on a device (with that device current) looks up the
+ *    array's address; make it before any stream capture.
+ *  - No scratch byte needs to start at zero: the call writes all it reads.
+ *  - One scratch per device: calls on one device whose kernels could overlap
+ *    (unordered streams, several host threads) race on it and must be
+ *    ordered by the caller.
+ */
+#define W4A4_NOALLOC_SCRATCH_BYTES (16u << 20)
+int w4a4_linear_noalloc(const uint16_t* X, int M, int K, int ldx,
+                        const w4a4_qtensor* Wq, int scale_mode,
+                        const int32_t* S, int nS,
+                        uint16_t* Y, int ldy, void* stream);
+
+/*
  * Second stage of the dual-stage NVFP4 quantization ("APEX4..." page,
  * para 2, ARCQuant): for every row, R_j = x[S_j] - x^[S_j] in FP32, where
  * x^ is the first-stage dequantized value (code * block scale * s2, rounded

@@ -98,6 +98,12 @@ def test_argument_errors_before_any_device_work(L):
     Wm = _qt(w4.MXFP4, 256, 384)
     assert L.w4a4_linear(C.c_void_p(16), 4, 256, 256, C.byref(Wm), 1, C.c_void_p(16), 128, C.c_void_p(16), 256,
                          C.c_void_p(256), 1 << 20, None) == w4.ERR_INVALID_ARG
+    # the static-scratch linear: sizes beyond its scratch, null weights
+    Wbig = _qt(w4.NVFP4, 1024, 8192, w4.SCALE_TENSOR)
+    assert L.w4a4_linear_noalloc(C.c_void_p(16), 4096, 8192, 8192, C.byref(Wbig), 1, None, 0, C.c_void_p(16),
+                                 1024, None) == w4.ERR_WORKSPACE
+    assert L.w4a4_linear_noalloc(C.c_void_p(16), 4, 256, 256, None, 1, None, 0, C.c_void_p(16), 256,
+                                 None) == w4.ERR_INVALID_ARG
     # S with nS not a multiple of 128
     assert L.w4a4_augment_residual(C.c_void_p(16), 4, 256, 256, C.c_void_p(16), 64, ref, None) == w4.ERR_INVALID_ARG
     # channel selection: workspace too small

@@ -25,7 +25,7 @@ OK, ERR_INVALID_ARG, ERR_MISALIGNED, ERR_WORKSPACE, ERR_ARCH, ERR_CUDA, ERR_DEVI
 # every entry point declared in include/w4a4.h
 EXPORTS = ("w4a4_qtensor_bytes", "w4a4_quantize_act", "w4a4_quantize_weight", "w4a4_gemm",
            "w4a4_linear_workspace", "w4a4_linear", "w4a4_augment_residual", "w4a4_select_channels",
-           "w4a4_device_status", "w4a4_debug_set", "w4a4_status_string")
+           "w4a4_device_status", "w4a4_debug_set", "w4a4_status_string", "w4a4_linear_noalloc")
 
 
 class W4A4Error(RuntimeError):
@@ -60,6 +60,7 @@ def lib():
         L.w4a4_linear_workspace.argtypes = [i, i, i, i, i]
         L.w4a4_linear_workspace.restype = sz
         L.w4a4_linear.argtypes = [vp, i, i, i, qp, i, vp, i, vp, i, vp, sz, vp]
+        L.w4a4_linear_noalloc.argtypes = [vp, i, i, i, qp, i, vp, i, vp, i, vp]
         L.w4a4_augment_residual.argtypes = [vp, i, i, i, vp, i, qp, vp]
         L.w4a4_select_channels.argtypes = [vp, i, i, i, i, vp, vp, sz, vp]
         L.w4a4_device_status.argtypes = [vp]
@@ -68,7 +69,8 @@ def lib():
         L.w4a4_status_string.argtypes = [i]
         L.w4a4_status_string.restype = C.c_char_p
         for name in ("w4a4_qtensor_bytes", "w4a4_quantize_act", "w4a4_quantize_weight", "w4a4_gemm",
-                     "w4a4_linear", "w4a4_augment_residual", "w4a4_select_channels", "w4a4_device_status"):
+                     "w4a4_linear", "w4a4_augment_residual", "w4a4_select_channels", "w4a4_device_status",
+                     "w4a4_linear_noalloc"):
             getattr(L, name).restype = i
         _lib = L
     return _lib
@@ -166,6 +168,23 @@ def linear(X, Wq: QTensor, scale_mode: int = SCALE_TOKEN, S=None, Y=None, ws=Non
     _check(lib().w4a4_linear(_ptr(X), M, K, X.stride(0), Wq.ref, scale_mode, _ptr(S), nS, _ptr(Y), Y.stride(0),
                              _ptr(ws), ws.numel(), _stream()), "w4a4_linear")
     return Y
+
+
+def linear_noalloc(X, Wq: QTensor, scale_mode: int = SCALE_TOKEN, S=None, Y=None):
+    """linear() with the library's static per-device scratch instead of a
+    workspace (sizes up to NOALLOC_SCRATCH_BYTES of workspace; calls on one
+    device must not overlap)."""
+    import torch
+    M, K = X.shape
+    nS = 0 if S is None else S.numel()
+    if Y is None:
+        Y = torch.empty(M, Wq.rows, dtype=torch.bfloat16, device=X.device)
+    _check(lib().w4a4_linear_noalloc(_ptr(X), M, K, X.stride(0), Wq.ref, scale_mode, _ptr(S), nS, _ptr(Y),
+                                     Y.stride(0), _stream()), "w4a4_linear_noalloc")
+    return Y
+
+
+NOALLOC_SCRATCH_BYTES = 16 << 20
 
 
 def augment_residual(X, S, Xaug: QTensor) -> QTensor:

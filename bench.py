@@ -303,7 +303,7 @@ def run_ours(args, rank, world):
     roofline = {"bound": "tensor", "achieved": round(gemm_tflops, 1), "peak": round(fp4_peak, 1),
                 "unit": "TFLOP/s", "frac": round(gemm_tflops / fp4_peak, 4), "traffic": None,
                 "peak_src": f"{P['src']} bf16 burst x {FP4_PER_BF16:g} (nominal fp4/bf16)",
-                "kernel": "gemm_fp4_kernel (NVFP4, 128x256 tile)", "per_shape_tflops": per_shape}
+                "kernel": "gemm_fp4_pair_kernel (NVFP4, 256x256 tile on a CTA pair)", "per_shape_tflops": per_shape}
 
     rows = {} if args.no_rows else extra_rows(args, dev, stream, P)
 

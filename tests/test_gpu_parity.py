@@ -124,7 +124,7 @@ def _gemm_case(orc, fmt, M, N, K, model="llama2_70b", a_mode=w4.SCALE_TOKEN, see
     return Y, yref
 
 
-GEMM_SHAPES = [(16, 256, 256), (1, 128, 256), (128, 256, 128), (200, 384, 640), (257, 512, 2048),
+GEMM_SHAPES = [(16, 256, 256), (1, 128, 256), (128, 256, 128), (200, 384, 640), (257, 512, 2048), (2304, 2304, 256),
                (130, 1024, 1024)]
 
 
@@ -254,6 +254,7 @@ def test_bounded_wait_reports_timeout(orc):
     Xw = synth.weights("llama2_70b", N, K, seed=2)
     A = w4.quantize_act(dev(Xa), w4.NVFP4, w4.SCALE_TOKEN)
     B = w4.quantize_weight(dev(Xw), w4.NVFP4)
+    A2 = w4.quantize_act(dev(synth.activations("llama2_70b", 2 * M, K, seed=3)), w4.NVFP4, w4.SCALE_TOKEN)
     Ai = w4.quantize_act(dev(Xa), w4.INT4, 0)
     Bi = w4.quantize_weight(dev(Xw), w4.INT4)
     torch.cuda.synchronize()
@@ -263,9 +264,13 @@ def test_bounded_wait_reports_timeout(orc):
         assert w4.device_status() == w4.ERR_DEVICE_TIMEOUT
         w4.gemm(Ai, Bi)
         assert w4.device_status() == w4.ERR_DEVICE_TIMEOUT
+        w4.gemm(A2, B)  # M > 128: the CTA-pair kernel
+        assert w4.device_status() == w4.ERR_DEVICE_TIMEOUT
     finally:
         w4.debug_set(-1, 0)
     Y = w4.gemm(A, B)
+    assert w4.device_status() == w4.OK
+    w4.gemm(A2, B)
     assert w4.device_status() == w4.OK
     ca, sa, s2a = orc.quant_nvfp4(Xa, mode=1)
     cw, sw, s2w = orc.quant_nvfp4(Xw, mode=0)

@@ -13,7 +13,8 @@ CSRC = os.path.join(HERE, "csrc")
 LIBDIR = os.path.join(HERE, "lib")
 LIB = os.path.join(LIBDIR, "libw4a4.so")
 INCLUDE = os.path.join(os.path.dirname(HERE), "include")
-SOURCES = ["api.cu", "quant.cu", "gemm_fp4.cu", "gemm_fp4_persistent.cu", "gemm_int4.cu", "noalloc.cu"]
+SOURCES = ["api.cu", "quant.cu", "gemm_fp4.cu", "gemm_fp4_persistent.cu", "gemm_fp4_pair.cu", "gemm_int4.cu",
+           "noalloc.cu"]
 
 NVCC_FLAGS = [
     "-gencode", "arch=compute_100a,code=sm_100a",

@@ -80,6 +80,19 @@ int make_map(CUtensorMap* map, const void* base, int rows, int row_bytes, int bo
     return r == CUDA_SUCCESS ? W4A4_OK : W4A4_ERR_CUDA;
 }
 
+// 3-D byte tensor map over scale atoms [row_tiles][col_atoms][512 bytes], seen
+// as [row_tiles][2*col_atoms][256]: a box of box_atoms atoms of box_tiles row tiles.
+int make_map_sf(CUtensorMap* map, const void* base, int row_tiles, int col_atoms, int box_atoms, int box_tiles) {
+    cuuint64_t dims[3] = {256, (cuuint64_t)(2 * col_atoms), (cuuint64_t)row_tiles};
+    cuuint64_t strides[2] = {256, (cuuint64_t)col_atoms * 512};
+    cuuint32_t box[3] = {256, (cuuint32_t)(2 * box_atoms), (cuuint32_t)box_tiles};
+    cuuint32_t estr[3] = {1, 1, 1};
+    CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(base), dims, strides, box, estr,
+                          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? W4A4_OK : W4A4_ERR_CUDA;
+}
+
 int check_qtensor(const w4a4_qtensor* q) {
     if (!q || !q->codes || !q->scales) return W4A4_ERR_INVALID_ARG;
     if (q->format < 0 || q->format > 2 || q->group != group_of(q->format) || q->reserved != 0)
@@ -135,9 +148,13 @@ int check_S_args(const int32_t* S, int nS, int K) {
 }
 
 struct GemmSetup {
-    CUtensorMap ta, tb;
+    CUtensorMap ta, tb, tsa, tsb;  // codes of A and B; scale atoms (pair kernel)
     GemmArgs g;
 };
+
+// Large-M FP4 products run on CTA pairs (256 x 256 tiles); up to 128 rows of A
+// the one-CTA kernel (128 x 256 tiles) wastes no MMA rows.
+inline bool use_pair(const w4a4_qtensor* A) { return A->format != W4A4_INT4 && A->rows > kBM; }
 
 // Fill tensor maps and arguments for A (activations) x B (weights).
 int setup_gemm(const w4a4_qtensor* A, const w4a4_qtensor* B, uint16_t* Y, int ldy, bool decode, GemmSetup* s) {
@@ -163,6 +180,15 @@ int setup_gemm(const w4a4_qtensor* A, const w4a4_qtensor* B, uint16_t* Y, int ld
     if (A->format == W4A4_INT4) {
         rc = make_map(&s->ta, A->codes, A->rows, row_bytes, 64, 128, false);
         if (rc == W4A4_OK) rc = make_map(&s->tb, B->codes, B->rows, row_bytes, 64, kBN_I4, false);
+    } else if (!decode && use_pair(A)) {
+        // each CTA of a pair stages 128 rows of A and 128 rows of B
+        const int atoms_ps = A->format == W4A4_NVFP4 ? 4 : 2;
+        rc = make_map(&s->ta, A->codes, A->rows, row_bytes, 128, kBM, true);
+        if (rc == W4A4_OK) rc = make_map(&s->tb, B->codes, B->rows, row_bytes, 128, kBM, true);
+        if (rc == W4A4_OK)
+            rc = make_map_sf(&s->tsa, A->scales, pad128(A->rows) / 128, g.sf_col_atoms, atoms_ps, 1);
+        if (rc == W4A4_OK)
+            rc = make_map_sf(&s->tsb, B->scales, pad128(B->rows) / 128, g.sf_col_atoms, atoms_ps, 2);
     } else if (!decode) {
         rc = make_map(&s->ta, A->codes, A->rows, row_bytes, 128, kBM, true);
         if (rc == W4A4_OK) rc = make_map(&s->tb, B->codes, B->rows, row_bytes, 128, kBN, true);
@@ -186,6 +212,8 @@ int run_gemm(const w4a4_qtensor* A, const w4a4_qtensor* B, uint16_t* Y, int ldy,
     } else if (decode) {
         s.g.partial = partial;
         e = launch_gemm_fp4_decode(A->format == W4A4_NVFP4, s.ta, s.tb, s.g, num_sms, st);
+    } else if (use_pair(A)) {
+        e = launch_gemm_fp4_pair(A->format == W4A4_NVFP4, s.ta, s.tb, s.tsa, s.tsb, s.g, num_sms, pdl, st);
     } else {
         e = launch_gemm_fp4(A->format == W4A4_NVFP4, s.ta, s.tb, s.g, num_sms, pdl, st);
     }

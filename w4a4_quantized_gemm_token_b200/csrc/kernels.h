@@ -71,6 +71,12 @@ cudaError_t launch_select(const uint16_t* X, int Mc, int K, int ldx, int nS, int
 // 128 x bn (B) bytes.  pdl: launched as a programmatic dependent.
 cudaError_t launch_gemm_fp4(bool nvfp4, const CUtensorMap& tmA, const CUtensorMap& tmB, const GemmArgs& g,
                             int num_sms, bool pdl, cudaStream_t st);
+// The same product on clusters of two CTAs (tcgen05 cta_group::2), 256 x 256
+// output tiles: tmA/tmB boxes of 128 x 128 bytes (each CTA stages its half of
+// A and of B), tmSA/tmSB 3-D maps over the scale atoms (boxes of one stage's
+// atoms for 1 (A) and 2 (B) row tiles).
+cudaError_t launch_gemm_fp4_pair(bool nvfp4, const CUtensorMap& tmA, const CUtensorMap& tmB, const CUtensorMap& tmSA,
+                                 const CUtensorMap& tmSB, const GemmArgs& g, int num_sms, bool pdl, cudaStream_t st);
 // Small-M variant (M <= 16): weights take the MMA's M side (128 rows per tile),
 // the tokens its N side; the (tile, K-stage) units are split evenly over the
 // SMs, FP32 segment partials go to g.partial and a second kernel reduces them

@@ -124,7 +124,7 @@ def _gemm_case(orc, fmt, M, N, K, model="llama2_70b", a_mode=w4.SCALE_TOKEN, see
     return Y, yref
 
 
-GEMM_SHAPES = [(16, 256, 256), (1, 128, 256), (128, 256, 128), (200, 384, 640), (257, 512, 2048), (2304, 2304, 256),
+GEMM_SHAPES = [(16, 256, 256), (1, 128, 256), (9, 256, 640), (128, 256, 128), (200, 384, 640), (257, 512, 2048), (2304, 2304, 256),
                (130, 1024, 1024)]
 
 

@@ -93,6 +93,20 @@ int make_map_sf(CUtensorMap* map, const void* base, int row_tiles, int col_atoms
     return r == CUDA_SUCCESS ? W4A4_OK : W4A4_ERR_CUDA;
 }
 
+// 3-D byte tensor map over codes[rows][row_bytes] (row_bytes a multiple of 128)
+// seen as (128-byte K-block, row, K-block): a box of box_rows rows x box_kb
+// consecutive K-blocks lands as box_kb 128-byte-swizzled [box_rows][128] tiles.
+int make_map_kblocks(CUtensorMap* map, const void* base, int rows, int row_bytes, int box_rows, int box_kb) {
+    cuuint64_t dims[3] = {128, (cuuint64_t)rows, (cuuint64_t)(row_bytes / 128)};
+    cuuint64_t strides[2] = {(cuuint64_t)row_bytes, 128};
+    cuuint32_t box[3] = {128, (cuuint32_t)box_rows, (cuuint32_t)box_kb};
+    cuuint32_t estr[3] = {1, 1, 1};
+    CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(base), dims, strides, box, estr,
+                          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? W4A4_OK : W4A4_ERR_CUDA;
+}
+
 int check_qtensor(const w4a4_qtensor* q) {
     if (!q || !q->codes || !q->scales) return W4A4_ERR_INVALID_ARG;
     if (q->format < 0 || q->format > 2 || q->group != group_of(q->format) || q->reserved != 0)
@@ -192,6 +206,11 @@ int setup_gemm(const w4a4_qtensor* A, const w4a4_qtensor* B, uint16_t* Y, int ld
     } else if (!decode) {
         rc = make_map(&s->ta, A->codes, A->rows, row_bytes, 128, kBM, true);
         if (rc == W4A4_OK) rc = make_map(&s->tb, B->codes, B->rows, row_bytes, 128, kBN, true);
+    } else if (decode_k_blocks(A->cols) == 2) {
+        // weights take the MMA's M side (128 rows), tokens its N side (16 rows);
+        // both read as boxes of two consecutive 128-byte K-blocks per row
+        rc = make_map_kblocks(&s->ta, B->codes, B->rows, row_bytes, kBM, 2);
+        if (rc == W4A4_OK) rc = make_map_kblocks(&s->tb, A->codes, A->rows, row_bytes, kBN_DEC, 2);
     } else {
         // weights take the MMA's M side (box of 128 rows), tokens its N side (16 rows)
         rc = make_map(&s->ta, B->codes, B->rows, row_bytes, 128, kBM, true);

@@ -2,19 +2,23 @@
 // M <= 16, bound by streaming the 4-bit weights from HBM.
 //
 // The weights take the MMA's M side (128 rows per tile) and the tokens its N
-// side (16), so one tcgen05.mma kind::mxf4nvf4 covers 128 x 16 x 64.  The
-// (weight tile, K-stage of 256) work units are split into equal contiguous
-// ranges, one per SM (stream-K), so every SM streams the same number of
-// weight bytes whatever N and K are.  A CTA accumulates in TMEM while its
-// range stays in one weight tile and writes an FP32 partial sum per tile
-// segment (double-buffered accumulators); a second kernel adds the segments
-// of each tile in a fixed order (deterministic), applies alpha and rounds to
-// bf16.  Launched as a programmatic dependent, the kernel starts streaming
-// weights while the activation quantizer still runs and waits only before
-// its first activation load.
-// Warp roles (256 threads): warp 0 lane 0 TMA producer (8-stage ring),
-// warp 1 TMEM owner + MMA issuer, warp 2 lane 0 scale-factor copies,
-// warps 4..7 epilogue (TMEM lane quarter = warp % 4).
+// side (16), so one tcgen05.mma kind::mxf4nvf4 covers 128 x 16 x 64.  A work
+// unit is a weight tile and KB consecutive K-stages of 256; the units are
+// split into equal contiguous ranges, one per SM (stream-K), so every SM
+// streams the same number of weight bytes whatever N and K are.  With KB = 2
+// the weights arrive as 3-D boxes (128-byte K-block, row, K-block): each row
+// contributes 256 contiguous bytes per copy instead of 128, which HBM serves
+// much faster, and the box still lands as standard 128-byte-swizzled tiles.
+// A CTA accumulates in TMEM while its range stays in one weight tile and
+// writes an FP32 partial sum per tile segment (double-buffered
+// accumulators); a second kernel adds the segments of each tile in a fixed
+// order (deterministic), applies alpha and rounds to bf16.  Launched as a
+// programmatic dependent, the kernel starts streaming weights while the
+// activation quantizer still runs and waits only before its first activation
+// load.
+// Warp roles (256 threads): warp 0 lane 0 TMA producer, warp 1 TMEM owner +
+// MMA issuer, warp 2 lane 0 scale-factor copies, warps 4..7 epilogue (TMEM
+// lane quarter = warp % 4).
 #include <cstdint>
 #include <cuda_bf16.h>
 
@@ -25,24 +29,30 @@ namespace w4a4 {
 
 __device__ int g_error_word = 0;
 
-namespace dec {
-constexpr int BN = kBN_DEC;                 // tokens per MMA (16)
-constexpr int STAGES = 8;
-constexpr int A_BYTES = kBM * 128;          // weight tile, 16 KB
-constexpr int B_BYTES = BN * 128;           // token tile, 2 KB
-constexpr int ATOM = 512;
-constexpr int SFA_C = 4 * ATOM;
-constexpr int SFB_C = 4 * ATOM;
-constexpr int STAGE = A_BYTES + B_BYTES + SFA_C + SFB_C;
-constexpr int BAR_OFF = STAGES * STAGE;
-constexpr int SMEM = BAR_OFF + 512 + 1024;
-constexpr int SF_COLS = 32;                 // per stage: A 16 + B 16 columns
-constexpr int SF_COL0 = 2 * BN;             // after two accumulators of 16 columns
-constexpr int TMEM_COLS = 512;
-constexpr int THREADS = 256;
-static_assert(STAGE % 1024 == 0, "stages keep the 1024-byte alignment of swizzled tiles");
-static_assert(SF_COL0 + STAGES * SF_COLS <= TMEM_COLS, "tensor memory holds 512 columns");
-}  // namespace dec
+// K-stages per work unit: two when the weights' K-block count is exact (the
+// 3-D box view needs K % 256 == 0), else one (2-D boxes).
+__host__ __device__ __forceinline__ int decode_kb(int K) { return K % kBK_FP4 == 0 ? 2 : 1; }
+
+template <int KB>
+struct Dec {
+    static constexpr int BN = kBN_DEC;                 // tokens per MMA (16)
+    static constexpr int STAGES = 8 / KB;
+    static constexpr int A_BYTES = KB * kBM * 128;     // weight tiles [kb][128 rows][128 B]
+    static constexpr int B_BYTES = KB * BN * 128;      // token tiles [kb][16 rows][128 B]
+    static constexpr int ATOM = 512;
+    static constexpr int SFA_C = KB * 4 * ATOM;        // weight scale atoms of a unit
+    static constexpr int SFB_C = KB * 4 * ATOM;        // token scale atoms of a unit
+    static constexpr int STAGE = A_BYTES + B_BYTES + SFA_C + SFB_C;
+    static constexpr int BAR_OFF = STAGES * STAGE;
+    static constexpr int SMEM = BAR_OFF + 512 + 1024;
+    static constexpr int SF_COLS = KB * 32;            // per stage: weights KB*16 + tokens KB*16 columns
+    static constexpr int SF_COL0 = 2 * BN;             // after two accumulators of 16 columns
+    static constexpr int TMEM_COLS = 512;
+    static constexpr int THREADS = 256;
+    static_assert(STAGE % 1024 == 0, "stages keep the 1024-byte alignment of swizzled tiles");
+    static_assert(SF_COL0 + STAGES * SF_COLS <= TMEM_COLS, "tensor memory holds 512 columns");
+    static_assert(SMEM <= 232448, "shared memory per block");
+};
 
 __device__ __forceinline__ void tmem_ld_32x32b_x16(uint32_t taddr, uint32_t (&r)[16]) {
     asm volatile(
@@ -64,14 +74,16 @@ __device__ __forceinline__ int unit_owner(long long u, long long U, int G) {
     return c;
 }
 
-template <bool NV>
-__global__ void __launch_bounds__(dec::THREADS, 1)
+template <bool NV, int KB>
+__global__ void __launch_bounds__(Dec<KB>::THREADS, 1)
     gemm_fp4_decode_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmX,
                            GemmArgs g) {
-    using namespace dec;
+    using D = Dec<KB>;
+    constexpr int STAGES = D::STAGES, A_BYTES = D::A_BYTES, B_BYTES = D::B_BYTES, ATOM = D::ATOM;
+    constexpr int BN = D::BN;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    uint64_t* full = reinterpret_cast<uint64_t*>(smem + BAR_OFF);
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem + D::BAR_OFF);
     uint64_t* empty = full + STAGES;
     uint64_t* sfull = empty + STAGES;
     uint64_t* accf = sfull + STAGES;  // [2]
@@ -83,8 +95,9 @@ __global__ void __launch_bounds__(dec::THREADS, 1)
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int KT = (g.K + kBK_FP4 - 1) / kBK_FP4;
+    const int KG = (KT + KB - 1) / KB;  // units per weight tile
     const int ntiles = (g.N + kBM - 1) / kBM;
-    const long long U = (long long)ntiles * KT;
+    const long long U = (long long)ntiles * KG;
     const int G = gridDim.x;
     const long long u0 = unit_begin(blockIdx.x, U, G), u1 = unit_begin(blockIdx.x + 1, U, G);
     const int nunits = (int)(u1 - u0);
@@ -92,6 +105,13 @@ __global__ void __launch_bounds__(dec::THREADS, 1)
     // weights are the MMA's A side, tokens its B side
     const uint8_t* sfw = g.sfb;
     const uint8_t* sfx = g.sfa;
+    // K-chunks of 64 and scale atoms of unit u (K tails have fewer)
+    auto unit_chunks = [&](long long u, int& nk, int& atoms, int& atom_k0) {
+        const int kt0 = (int)(u % KG) * KB;
+        nk = min(4 * KB, (g.K - kt0 * kBK_FP4) / 64);
+        atoms = NV ? nk : (nk + 1) / 2;
+        atom_k0 = NV ? kt0 * 4 : kt0 * 2;
+    };
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < STAGES; ++s) {
@@ -113,7 +133,7 @@ __global__ void __launch_bounds__(dec::THREADS, 1)
         tma_prefetch_desc(&tmX);
     }
     if (warp == 1) {
-        tmem_alloc(tmem_holder, TMEM_COLS);
+        tmem_alloc(tmem_holder, D::TMEM_COLS);
         tmem_relinquish();
     }
     tc_fence_before();
@@ -125,30 +145,32 @@ __global__ void __launch_bounds__(dec::THREADS, 1)
     if (warp == 0) {
         if (lane == 0) {
             // ------------------------------ producer ------------------------------
-            auto atoms_of = [&](int kt, int& atoms, int& atom_k0) {
-                const int nk = min(4, (g.K - kt * kBK_FP4) / 64);
-                atoms = NV ? nk : (nk + 1) / 2;
-                atom_k0 = NV ? kt * 4 : kt * 2;
-            };
             auto load_w = [&](long long u, int s) {
-                const int nt = (int)(u / KT), kt = (int)(u % KT);
-                int atoms, k0;
-                atoms_of(kt, atoms, k0);
-                uint8_t* st = smem + s * STAGE;
+                const int nt = (int)(u / KG), kt0 = (int)(u % KG) * KB;
+                int nk, atoms, k0;
+                unit_chunks(u, nk, atoms, k0);
+                uint8_t* st = smem + s * D::STAGE;
+                // full boxes (K-blocks past K are zero-filled) + the scale atoms in range
                 mbar_arrive_expect_tx(&full[s], (uint32_t)(A_BYTES + B_BYTES + 2 * atoms * ATOM));
-                tma_load_2d(st, &tmW, kt * 128, nt * kBM, &full[s]);
+                if (KB == 1)
+                    tma_load_2d(st, &tmW, kt0 * 128, nt * kBM, &full[s]);
+                else
+                    tma_load_3d(st, &tmW, 0, nt * kBM, kt0, &full[s]);
                 bulk_load(st + A_BYTES + B_BYTES, sfw + ((size_t)nt * g.sf_col_atoms + k0) * ATOM, atoms * ATOM,
                           &full[s]);
             };
             auto load_x = [&](long long u, int s) {
-                const int kt = (int)(u % KT);
-                int atoms, k0;
-                atoms_of(kt, atoms, k0);
-                uint8_t* st = smem + s * STAGE;
-                tma_load_2d(st + A_BYTES, &tmX, kt * 128, 0, &full[s]);
-                bulk_load(st + A_BYTES + B_BYTES + SFA_C, sfx + (size_t)k0 * ATOM, atoms * ATOM, &full[s]);
+                const int kt0 = (int)(u % KG) * KB;
+                int nk, atoms, k0;
+                unit_chunks(u, nk, atoms, k0);
+                uint8_t* st = smem + s * D::STAGE;
+                if (KB == 1)
+                    tma_load_2d(st + A_BYTES, &tmX, kt0 * 128, 0, &full[s]);
+                else
+                    tma_load_3d(st + A_BYTES, &tmX, 0, 0, kt0, &full[s]);
+                bulk_load(st + A_BYTES + B_BYTES + D::SFA_C, sfx + (size_t)k0 * ATOM, atoms * ATOM, &full[s]);
             };
-            // stream the first weight tiles before the activations are known to be ready
+            // stream the first weight units before the activations are known to be ready
             const int pre = min(STAGES, nunits);
             int it = 0;
             for (; it < pre; ++it)
@@ -174,8 +196,8 @@ __global__ void __launch_bounds__(dec::THREADS, 1)
             int it = 0, seg = 0;
             long long u = u0;
             while (u < u1 && ok) {
-                const int nt = (int)(u / KT);
-                const long long sbeg = u, send = min(u1, (long long)(nt + 1) * KT);
+                const int nt = (int)(u / KG);
+                const long long sbeg = u, send = min(u1, (long long)(nt + 1) * KG);
                 const int buf = seg & 1;
                 if (seg >= 2 && !mbar_wait(&acce[buf], ((seg >> 1) - 1) & 1, limit, abort_flag)) {
                     ok = false;
@@ -189,14 +211,16 @@ __global__ void __launch_bounds__(dec::THREADS, 1)
                         break;
                     }
                     tc_fence_after();
-                    const int kt = (int)(u % KT);
-                    const uint32_t sA = smem_u32(smem + s * STAGE), sB = sA + A_BYTES;
-                    const uint32_t sfa_t = tmem + SF_COL0 + s * SF_COLS, sfb_t = sfa_t + 16;
-                    const int nk = min(4, (g.K - kt * kBK_FP4) / 64);
+                    int nk, atoms, k0;
+                    unit_chunks(u, nk, atoms, k0);
+                    const uint32_t sA = smem_u32(smem + s * D::STAGE), sB = sA + A_BYTES;
+                    const uint32_t sfa_t = tmem + D::SF_COL0 + s * D::SF_COLS, sfb_t = sfa_t + 16 * KB;
                     for (int j = 0; j < nk; ++j) {
+                        const int kb = j >> 2, jj = j & 3;  // K-block of the unit, chunk within it
                         const int sfid = NV ? 0 : (j & 1) * 2;
                         const int aj = NV ? j : (j >> 1);
-                        mma_fp4<NV>(tmem + buf * BN, desc_kmajor_sw128(sA + 32 * j), desc_kmajor_sw128(sB + 32 * j),
+                        mma_fp4<NV>(tmem + buf * BN, desc_kmajor_sw128(sA + kb * (kBM * 128) + 32 * jj),
+                                    desc_kmajor_sw128(sB + kb * (BN * 128) + 32 * jj),
                                     idesc_fp4(kBM, BN, !NV, sfid, sfid), (sfa_t + 4 * aj) | ((uint32_t)sfid << 30),
                                     (sfb_t + 4 * aj) | ((uint32_t)sfid << 30), (u > sbeg || j > 0) ? 1u : 0u);
                     }
@@ -222,11 +246,10 @@ __global__ void __launch_bounds__(dec::THREADS, 1)
                     break;
                 }
                 tc_fence_after();
-                const int kt = (int)((u0 + it) % KT);
-                const int nk = min(4, (g.K - kt * kBK_FP4) / 64);
-                const int atoms = NV ? nk : (nk + 1) / 2;
-                const uint32_t ca = smem_u32(smem + s * STAGE + A_BYTES + B_BYTES), cb = ca + SFA_C;
-                const uint32_t sfa_t = tmem + SF_COL0 + s * SF_COLS, sfb_t = sfa_t + 16;
+                int nk, atoms, k0;
+                unit_chunks(u0 + it, nk, atoms, k0);
+                const uint32_t ca = smem_u32(smem + s * D::STAGE + A_BYTES + B_BYTES), cb = ca + D::SFA_C;
+                const uint32_t sfa_t = tmem + D::SF_COL0 + s * D::SF_COLS, sfb_t = sfa_t + 16 * KB;
                 for (int j = 0; j < atoms; ++j) {
                     tc_cp_32x128b_x4(sfa_t + 4 * j, desc_sf_32x16(ca + j * ATOM));
                     tc_cp_32x128b_x4(sfb_t + 4 * j, desc_sf_32x16(cb + j * ATOM));
@@ -245,8 +268,8 @@ __global__ void __launch_bounds__(dec::THREADS, 1)
         int seg = 0;
         long long u = u0;
         while (u < u1) {
-            const int nt = (int)(u / KT);
-            const long long send = min(u1, (long long)(nt + 1) * KT);
+            const int nt = (int)(u / KG);
+            const long long send = min(u1, (long long)(nt + 1) * KG);
             const int buf = seg & 1;
             if (!mbar_wait(&accf[buf], (seg >> 1) & 1, limit, abort_flag, 20000)) break;
             tc_fence_after();
@@ -256,7 +279,7 @@ __global__ void __launch_bounds__(dec::THREADS, 1)
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&acce[buf]);
-            const int first = unit_owner((long long)nt * KT, U, G);
+            const int first = unit_owner((long long)nt * KG, U, G);
             float* slot = g.partial + ((size_t)nt * g.splits + (blockIdx.x - first)) * (BN * kBM);
             const int row = q * 32 + lane;
 #pragma unroll
@@ -269,7 +292,7 @@ __global__ void __launch_bounds__(dec::THREADS, 1)
     __syncthreads();
     if (warp == 1) {
         tc_fence_after();
-        tmem_dealloc(tmem, TMEM_COLS);
+        tmem_dealloc(tmem, D::TMEM_COLS);
     }
 }
 
@@ -278,18 +301,19 @@ template <bool NV>
 __global__ void __launch_bounds__(256) decode_reduce_kernel(GemmArgs g, int grid_g) {
     pdl_wait();
     const int KT = (g.K + kBK_FP4 - 1) / kBK_FP4;
+    const int KG = (KT + decode_kb(g.K) - 1) / decode_kb(g.K);
     const int ntiles = (g.N + kBM - 1) / kBM;
-    const long long U = (long long)ntiles * KT;
+    const long long U = (long long)ntiles * KG;
     const int nt = blockIdx.x;
-    const int first = unit_owner((long long)nt * KT, U, grid_g);
-    const int last = unit_owner((long long)(nt + 1) * KT - 1, U, grid_g);
-    for (int idx = threadIdx.x; idx < dec::BN * kBM; idx += blockDim.x) {
+    const int first = unit_owner((long long)nt * KG, U, grid_g);
+    const int last = unit_owner((long long)(nt + 1) * KG - 1, U, grid_g);
+    for (int idx = threadIdx.x; idx < kBN_DEC * kBM; idx += blockDim.x) {
         const int t = idx / kBM, row = idx % kBM;
         const int n = nt * kBM + row;
         if (t >= g.M || n >= g.N) continue;
         float acc = 0.0f;
         for (int c = first; c <= last; ++c)
-            acc += g.partial[((size_t)nt * g.splits + (c - first)) * (dec::BN * kBM) + idx];
+            acc += g.partial[((size_t)nt * g.splits + (c - first)) * (kBN_DEC * kBM) + idx];
         const float alpha = NV ? __fmul_rn(g.s2a[g.s2a_per_row ? t : 0], g.s2b[0]) : 1.0f;
         __nv_bfloat16 h = __float2bfloat16_rn(__fmul_rn(acc, alpha));
         g.Y[(size_t)t * g.ldy + n] = *reinterpret_cast<uint16_t*>(&h);
@@ -310,26 +334,32 @@ static cudaError_t launch_pdl(const void* kern, dim3 grid, dim3 block, size_t sm
     return cudaLaunchKernelExC(&cfg, kern, args);
 }
 
+static long long decode_units(int N, int K) {
+    const int KT = (K + kBK_FP4 - 1) / kBK_FP4, kb = decode_kb(K);
+    return (long long)((N + kBM - 1) / kBM) * ((KT + kb - 1) / kb);
+}
+
 int decode_grid(int N, int K, int num_sms) {
-    const long long U = (long long)((N + kBM - 1) / kBM) * ((K + kBK_FP4 - 1) / kBK_FP4);
+    const long long U = decode_units(N, K);
     return (int)(U < num_sms ? U : num_sms);
 }
 
 int decode_max_owners(int N, int K, int num_sms) {
-    const int KT = (K + kBK_FP4 - 1) / kBK_FP4;
-    const long long U = (long long)((N + kBM - 1) / kBM) * KT;
+    const int KT = (K + kBK_FP4 - 1) / kBK_FP4, kb = decode_kb(K);
+    const int KG = (KT + kb - 1) / kb;
+    const long long U = decode_units(N, K);
     const int G = decode_grid(N, K, num_sms);
     const long long per = U / G;  // every range holds per or per + 1 units
-    return (int)((KT + per - 1) / per) + 1;
+    return (int)((KG + per - 1) / per) + 1;
 }
 
-template <bool NV>
+template <bool NV, int KB>
 static cudaError_t launch_dec_t(const CUtensorMap& tmW, const CUtensorMap& tmX, const GemmArgs& g0, int num_sms,
                                 cudaStream_t st) {
-    auto kern = gemm_fp4_decode_kernel<NV>;
+    auto kern = gemm_fp4_decode_kernel<NV, KB>;
     static bool attr_set = false;
     if (!attr_set) {
-        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, dec::SMEM);
+        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Dec<KB>::SMEM);
         if (e != cudaSuccess) return e;
         attr_set = true;
     }
@@ -338,7 +368,8 @@ static cudaError_t launch_dec_t(const CUtensorMap& tmW, const CUtensorMap& tmX, 
     g.splits = decode_max_owners(g.N, g.K, num_sms);  // slots per weight tile in the workspace
     CUtensorMap a = tmW, b = tmX;
     void* args[] = {&a, &b, &g};
-    cudaError_t e = launch_pdl(reinterpret_cast<const void*>(kern), dim3(G), dim3(dec::THREADS), dec::SMEM, st, args);
+    cudaError_t e =
+        launch_pdl(reinterpret_cast<const void*>(kern), dim3(G), dim3(Dec<KB>::THREADS), Dec<KB>::SMEM, st, args);
     if (e != cudaSuccess) return e;
     int gg = G;
     void* rargs[] = {&g, &gg};
@@ -346,9 +377,13 @@ static cudaError_t launch_dec_t(const CUtensorMap& tmW, const CUtensorMap& tmX, 
                       dim3(256), 0, st, rargs);
 }
 
+int decode_k_blocks(int K) { return decode_kb(K); }
+
 cudaError_t launch_gemm_fp4_decode(bool nvfp4, const CUtensorMap& tmW, const CUtensorMap& tmX, const GemmArgs& g,
                                    int num_sms, cudaStream_t st) {
-    return nvfp4 ? launch_dec_t<true>(tmW, tmX, g, num_sms, st) : launch_dec_t<false>(tmW, tmX, g, num_sms, st);
+    if (decode_kb(g.K) == 2)
+        return nvfp4 ? launch_dec_t<true, 2>(tmW, tmX, g, num_sms, st) : launch_dec_t<false, 2>(tmW, tmX, g, num_sms, st);
+    return nvfp4 ? launch_dec_t<true, 1>(tmW, tmX, g, num_sms, st) : launch_dec_t<false, 1>(tmW, tmX, g, num_sms, st);
 }
 
 }  // namespace w4a4

@@ -85,6 +85,9 @@ cudaError_t launch_gemm_fp4_decode(bool nvfp4, const CUtensorMap& tmW, const CUt
                                    int num_sms, cudaStream_t st);
 // Partial-sum slots per weight tile of the small-M variant on `num_sms` SMs.
 int decode_max_owners(int N, int K, int num_sms);
+// K-stages of 256 per work unit of the small-M variant: 2 (weights and tokens
+// read as 3-D boxes of two K-blocks) when K % 256 == 0, else 1 (2-D boxes).
+int decode_k_blocks(int K);
 // INT4-g128 GEMM on the 8-bit integer MMA with per-group FP32 rescaling.
 cudaError_t launch_gemm_int4(const CUtensorMap& tmA, const CUtensorMap& tmB, const GemmArgs& g, int num_sms,
                              bool pdl, cudaStream_t st);

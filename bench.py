@@ -166,8 +166,9 @@ def time_loop(fn, iters, stream, flush=None):
     """Average device time (ms) of fn() over iters launches, CUDA events on `stream`.
 
     With `flush` (a device buffer larger than L2) each launch is timed on its
-    own between events, after the buffer has been overwritten, so inputs that
-    would fit in L2 are read from HBM every time."""
+    own between events, after the buffer has been read through, so inputs
+    that would fit in L2 are read from HBM every time (reading leaves clean
+    lines in L2: the timed kernel pays no write-back of the flush)."""
     import torch
     torch.cuda.synchronize()
     if flush is None:
@@ -180,7 +181,7 @@ def time_loop(fn, iters, stream, flush=None):
         return s.elapsed_time(e) / iters
     evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(iters)]
     for (s, e) in evs:
-        flush.fill_(1)
+        flush.max()
         s.record(stream)
         fn()
         e.record(stream)
@@ -189,10 +190,10 @@ def time_loop(fn, iters, stream, flush=None):
 
 
 def l2_flush_buffer(dev):
-    """A buffer twice the size of L2 (written between timed launches)."""
+    """A buffer twice the size of L2 (read between timed launches)."""
     import torch
     l2 = torch.cuda.get_device_properties(dev).L2_cache_size
-    return torch.empty(2 * l2 // 4, dtype=torch.int32, device=dev)
+    return torch.ones(2 * l2 // 4, dtype=torch.int32, device=dev)
 
 
 def max_over_ranks(x: float, device, world: int) -> float:

@@ -532,6 +532,166 @@ __global__ void __launch_bounds__(1024) compact_kernel(const int* selected, int 
 // ---------------------------------------------------------------------------
 // Host launchers
 // ---------------------------------------------------------------------------
+// ---------------------------------------------------------------------------
+// NVFP4 with a dynamic per-token scale (the activation hot path).  Persistent
+// CTAs walk rows r = blockIdx.x, +gridDim.x, ...; thread 0 keeps the next
+// NB-1 rows in flight as bulk copies into a ring of shared-memory row
+// buffers, so each SM has its loads outstanding while it computes.  For the
+// current row every thread takes J chunks of 16 elements (items t, t+T, ...)
+// into registers, the CTA reduces the row amax, and the threads tabulate for
+// the row d_c = E4M3(c) * s2 and RN(1/d_c) for all 128 scale codes, so a
+// block needs no reciprocal of its own.  Each item is then quantized from
+// registers: block scale by two refined divisions, codes by refined division
+// with the tabulated reciprocal.  The refined division is exact here whenever
+// s2 >= 2^-100 (the block quotients are then either below 2^-10, which
+// encodes to zero either way, or normal and at most about 12); a row below
+// that takes IEEE division throughout (a CTA-uniform branch).  Rows
+// M .. rows_pad-1 write the zero scales of the 128-row atoms' padding.
+// ---------------------------------------------------------------------------
+template <int J>
+__global__ void __launch_bounds__(512) quant_nvfp4_token_kernel(QuantArgs a, int nb) {
+    pdl_launch_dependents();
+    extern __shared__ __align__(128) uint8_t qsm[];
+    __shared__ float wmax[16];
+    __shared__ float2 tab[128];  // (d_c, RN(1/d_c)) for E4M3 codes c (sign 0)
+    const int t = threadIdx.x, T = blockDim.x;
+    const int lane = t & 31, warp = t >> 5, nwarps = T >> 5;
+    const int items = a.K / 16;
+    const int row_bytes = a.K * 2;
+    uint64_t* bars = reinterpret_cast<uint64_t*>(qsm + (size_t)nb * row_bytes);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + nb);
+    const int G = gridDim.x;
+    // rows of this CTA that are loaded: blockIdx.x + i*G < M
+    const int nlive = a.M > (int)blockIdx.x ? (a.M - 1 - (int)blockIdx.x) / G + 1 : 0;
+    auto issue = [&](int i) {
+        const int b = i % nb, r = blockIdx.x + i * G;
+        mbar_arrive_expect_tx(&bars[b], (uint32_t)row_bytes);
+        bulk_load(qsm + (size_t)b * row_bytes, a.X + (size_t)r * a.ldx, row_bytes, &bars[b]);
+    };
+    if (t == 0) {
+        for (int b = 0; b < nb; ++b) mbar_init(&bars[b], 1);
+        *abort_flag = 0;
+        fence_mbar_init();
+        for (int i = 0; i < nb && i < nlive; ++i) issue(i);
+    }
+    __syncthreads();
+    for (int i = 0; i < nlive; ++i) {
+        const int b = i % nb, r = blockIdx.x + i * G;
+        if (!mbar_wait(&bars[b], (i / nb) & 1, 2000000000ull, abort_flag)) break;
+        const uint4* xr = reinterpret_cast<const uint4*>(qsm + (size_t)b * row_bytes);
+        uint32_t w[J][8];
+#pragma unroll
+        for (int j = 0; j < J; ++j) {
+            const int it = t + T * j;
+            uint4 v0 = make_uint4(0, 0, 0, 0), v1 = v0;
+            if (it < items) {
+                v0 = xr[2 * it];
+                v1 = xr[2 * it + 1];
+            }
+            w[j][0] = v0.x; w[j][1] = v0.y; w[j][2] = v0.z; w[j][3] = v0.w;
+            w[j][4] = v1.x; w[j][5] = v1.y; w[j][6] = v1.z; w[j][7] = v1.w;
+        }
+        float bm[J], m = 0.0f;
+#pragma unroll
+        for (int j = 0; j < J; ++j) {
+            bm[j] = bmax16(w[j]);
+            m = fmaxf(m, bm[j]);
+        }
+        m = warp_max(m);
+        if (lane == 0) wmax[warp] = m;
+        __syncthreads();  // (also: every thread has its row data in registers)
+        if (t == 0 && i + nb < nlive) issue(i + nb);  // the buffer is free again
+        const float amax = warp_max(lane < nwarps ? wmax[lane] : 0.0f);
+        const float s2 = nvfp4_s2(amax);
+        const bool fast = s2 >= 0x1p-100f;  // the same for the whole CTA
+        for (int c = t; c < 128; c += T) {
+            const float d = c ? __fmul_rn(e4m3_value((uint8_t)c), s2) : 1.0f;
+            tab[c] = make_float2(d, __frcp_rn(d));
+        }
+        if (t == 0) a.s2_out[r] = s2;
+        __syncthreads();
+        const float rinv = __frcp_rn(s2);
+#pragma unroll
+        for (int j = 0; j < J; ++j) {
+            const int it = t + T * j;
+            uint32_t sb, w0, w1;
+            if (fast) {
+                const float u = div_refined(bm[j], 6.0f, 0x1.555556p-3f);  // RN(1/6)
+                sb = e4m3_rn_sat(div_refined(u, s2, rinv));
+                const float2 dy = tab[sb];
+                w0 = e2m1x8_fast(w[j], pack2(-dy.y), pack2(dy.x));
+                w1 = e2m1x8_fast(w[j] + 4, pack2(-dy.y), pack2(dy.x));
+            } else {
+                sb = e4m3_rn_sat(__fdiv_rn(__fdiv_rn(bm[j], 6.0f), s2));
+                const float d = tab[sb].x;
+                w0 = e2m1x8_exact(make_uint4(w[j][0], w[j][1], w[j][2], w[j][3]), d);
+                w1 = e2m1x8_exact(make_uint4(w[j][4], w[j][5], w[j][6], w[j][7]), d);
+            }
+            if (sb == 0) {
+                w0 = 0;
+                w1 = 0;
+            }
+            // four consecutive items sit on lanes l .. l+3 (T is a multiple of 32)
+            const uint32_t b1 = __shfl_down_sync(0xffffffffu, sb, 1);
+            const uint32_t b2 = __shfl_down_sync(0xffffffffu, sb, 2);
+            const uint32_t b3 = __shfl_down_sync(0xffffffffu, sb, 3);
+            if (it < items) {
+                if ((it & 3) == 0)
+                    *reinterpret_cast<uint32_t*>(a.sf + sf_offset(r, it, a.sf_col_atoms)) =
+                        sb | (b1 << 8) | (b2 << 16) | (b3 << 24);
+                *reinterpret_cast<uint2*>(a.codes + (size_t)r * a.ldc + 8 * it) = make_uint2(w0, w1);
+            }
+        }
+        __syncthreads();  // wmax and tab are rewritten for the next row
+    }
+    if (*abort_flag && t == 0)  // wait for the copies still in flight
+        for (int b = 0; b < nb; ++b) mbar_wait_drain(&bars[b], 0, 100000000ull);
+    // padding rows of the 128-row scale atoms: zero scales
+    for (int r = a.M + (int)blockIdx.x; r < a.rows_pad; r += G)
+        for (int c4 = t; c4 < items / 4; c4 += T)
+            *reinterpret_cast<uint32_t*>(a.sf + sf_offset(r, 4 * c4, a.sf_col_atoms)) = 0u;
+}
+
+static cudaError_t launch_nvfp4_token(const QuantArgs& a, int rows_pad, int num_sms, cudaStream_t st) {
+    // J items (32 J bytes of the row) per thread, at most 512 threads
+    const int items = a.K / 16;
+    const int J = items < 128 ? 1 : items <= 2048 ? 4 : 8;
+    int T = (items + J - 1) / J;
+    T = (T + 31) / 32 * 32;
+    // resident CTAs per SM from registers (about 44 + 8 J per thread) and from a
+    // ring of at least three row buffers each (two rows in flight while one is
+    // computed), within about 200 KB of shared memory per SM
+    const int row_bytes = a.K * 2;
+    const int regs = 44 + 8 * J;
+    int per_sm = 65536 / (T * regs);
+    const int by_smem = (200 * 1024) / (3 * row_bytes);
+    per_sm = per_sm < by_smem ? per_sm : by_smem;
+    per_sm = per_sm < 1 ? 1 : (per_sm > 16 ? 16 : per_sm);
+    int nb = (200 * 1024) / (per_sm * row_bytes);
+    nb = nb < 2 ? 2 : (nb > 8 ? 8 : nb);
+    const size_t smem = (size_t)nb * row_bytes + 8 * nb + 16;
+    if (smem > 220 * 1024) return cudaErrorInvalidValue;
+    int grid = num_sms * per_sm;
+    if (grid > rows_pad) grid = rows_pad;
+    QuantArgs b = a;
+    b.rows_pad = rows_pad;
+    cudaError_t e = cudaSuccess;
+    if (J == 1) {
+        static size_t attr = 0;
+        if (smem > 48 * 1024 && smem > attr) e = cudaFuncSetAttribute(quant_nvfp4_token_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem), attr = smem;
+        if (e == cudaSuccess) quant_nvfp4_token_kernel<1><<<grid, T, smem, st>>>(b, nb);
+    } else if (J == 4) {
+        static size_t attr = 0;
+        if (smem > 48 * 1024 && smem > attr) e = cudaFuncSetAttribute(quant_nvfp4_token_kernel<4>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem), attr = smem;
+        if (e == cudaSuccess) quant_nvfp4_token_kernel<4><<<grid, T, smem, st>>>(b, nb);
+    } else {
+        static size_t attr = 0;
+        if (smem > 48 * 1024 && smem > attr) e = cudaFuncSetAttribute(quant_nvfp4_token_kernel<8>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem), attr = smem;
+        if (e == cudaSuccess) quant_nvfp4_token_kernel<8><<<grid, T, smem, st>>>(b, nb);
+    }
+    return e != cudaSuccess ? e : cudaGetLastError();
+}
+
 template <int FMT, bool GATHER>
 static cudaError_t launch_quant_fmt(const QuantArgs& a, int rows_pad, int num_sms, cudaStream_t st) {
     const int row_bytes = a.K_src * 2;
@@ -563,6 +723,8 @@ static cudaError_t launch_quant_fmt(const QuantArgs& a, int rows_pad, int num_sm
 }
 
 cudaError_t launch_quant(int fmt, bool gather, const QuantArgs& a, int rows_pad, int num_sms, cudaStream_t st) {
+    if (fmt == FMT_NVFP4 && !gather && a.mode == 1 && !a.static_s2 && a.K == a.K_src && a.K <= 49152)
+        return launch_nvfp4_token(a, rows_pad, num_sms, st);
     if (fmt == FMT_NVFP4) return gather ? launch_quant_fmt<FMT_NVFP4, true>(a, rows_pad, num_sms, st)
                                         : launch_quant_fmt<FMT_NVFP4, false>(a, rows_pad, num_sms, st);
     if (fmt == FMT_MXFP4) return gather ? launch_quant_fmt<FMT_MXFP4, true>(a, rows_pad, num_sms, st)

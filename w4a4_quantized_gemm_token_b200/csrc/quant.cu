@@ -549,10 +549,10 @@ __global__ void __launch_bounds__(1024) compact_kernel(const int* selected, int 
 // M .. rows_pad-1 write the zero scales of the 128-row atoms' padding.
 // ---------------------------------------------------------------------------
 template <int J>
-__global__ void __launch_bounds__(512) quant_nvfp4_token_kernel(QuantArgs a, int nb) {
+__global__ void __launch_bounds__(J <= 2 ? 1024 : 768) quant_nvfp4_token_kernel(QuantArgs a, int nb) {
     pdl_launch_dependents();
     extern __shared__ __align__(128) uint8_t qsm[];
-    __shared__ float wmax[16];
+    __shared__ float wmax[32];
     __shared__ float2 tab[128];  // (d_c, RN(1/d_c)) for E4M3 codes c (sign 0)
     const int t = threadIdx.x, T = blockDim.x;
     const int lane = t & 31, warp = t >> 5, nwarps = T >> 5;
@@ -653,16 +653,18 @@ __global__ void __launch_bounds__(512) quant_nvfp4_token_kernel(QuantArgs a, int
 }
 
 static cudaError_t launch_nvfp4_token(const QuantArgs& a, int rows_pad, int num_sms, cudaStream_t st) {
-    // J items (32 J bytes of the row) per thread, at most 512 threads
+    // J items (32 J bytes of the row) per thread: two, so that the resident
+    // CTAs bring enough warps to hide the per-item latency (at most 1024
+    // threads; four for the longest rows)
     const int items = a.K / 16;
-    const int J = items < 128 ? 1 : items <= 2048 ? 4 : 8;
+    const int J = items < 64 ? 1 : items <= 2048 ? 2 : 4;
     int T = (items + J - 1) / J;
     T = (T + 31) / 32 * 32;
     // resident CTAs per SM from registers (about 44 + 8 J per thread) and from a
     // ring of at least three row buffers each (two rows in flight while one is
     // computed), within about 200 KB of shared memory per SM
     const int row_bytes = a.K * 2;
-    const int regs = 44 + 8 * J;
+    const int regs = J == 1 ? 48 : J == 2 ? 56 : 72;
     int per_sm = 65536 / (T * regs);
     const int by_smem = (200 * 1024) / (3 * row_bytes);
     per_sm = per_sm < by_smem ? per_sm : by_smem;
@@ -680,14 +682,14 @@ static cudaError_t launch_nvfp4_token(const QuantArgs& a, int rows_pad, int num_
         static size_t attr = 0;
         if (smem > 48 * 1024 && smem > attr) e = cudaFuncSetAttribute(quant_nvfp4_token_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem), attr = smem;
         if (e == cudaSuccess) quant_nvfp4_token_kernel<1><<<grid, T, smem, st>>>(b, nb);
-    } else if (J == 4) {
+    } else if (J == 2) {
+        static size_t attr = 0;
+        if (smem > 48 * 1024 && smem > attr) e = cudaFuncSetAttribute(quant_nvfp4_token_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem), attr = smem;
+        if (e == cudaSuccess) quant_nvfp4_token_kernel<2><<<grid, T, smem, st>>>(b, nb);
+    } else {
         static size_t attr = 0;
         if (smem > 48 * 1024 && smem > attr) e = cudaFuncSetAttribute(quant_nvfp4_token_kernel<4>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem), attr = smem;
         if (e == cudaSuccess) quant_nvfp4_token_kernel<4><<<grid, T, smem, st>>>(b, nb);
-    } else {
-        static size_t attr = 0;
-        if (smem > 48 * 1024 && smem > attr) e = cudaFuncSetAttribute(quant_nvfp4_token_kernel<8>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem), attr = smem;
-        if (e == cudaSuccess) quant_nvfp4_token_kernel<8><<<grid, T, smem, st>>>(b, nb);
     }
     return e != cudaSuccess ? e : cudaGetLastError();
 }

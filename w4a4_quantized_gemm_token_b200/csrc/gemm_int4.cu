@@ -48,6 +48,28 @@ __device__ __forceinline__ void widen8(uint32_t w, uint32_t& o0, uint32_t& o1) {
     o1 = __byte_perm(lo, hi, 0x7362);  // e4 e5 e6 e7
 }
 
+__device__ __forceinline__ uint64_t pack2(float v) {
+    const uint32_t u = __float_as_uint(v);
+    return ((uint64_t)u << 32) | u;
+}
+
+// (a0, a1) += (float(p0), float(p1)) * (sa * b0, sa * b1) with sm_100's packed
+// FP32 operations; every lane is the IEEE result of the scalar sequence
+// (product of the scales, rounded; then one fused multiply-add).
+__device__ __forceinline__ void rescale2(float& a0, float& a1, uint32_t p0, uint32_t p1, uint64_t sa2, float b0,
+                                         float b1) {
+    const float f0 = __int2float_rn((int)p0), f1 = __int2float_rn((int)p1);
+    asm("{\n\t.reg .b64 b, s, f, a;\n\t"
+        "mov.b64 b, {%2, %3};\n\t"
+        "mul.rn.f32x2 s, %4, b;\n\t"
+        "mov.b64 f, {%5, %6};\n\t"
+        "mov.b64 a, {%0, %1};\n\t"
+        "fma.rn.f32x2 a, f, s, a;\n\t"
+        "mov.b64 {%0, %1}, a;\n\t}"
+        : "+f"(a0), "+f"(a1)
+        : "f"(b0), "f"(b1), "l"(sa2), "f"(f0), "f"(f1));
+}
+
 __device__ __forceinline__ void named_bar(int id, int n) { asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory"); }
 
 __global__ void __launch_bounds__(i4::THREADS, 1)
@@ -190,27 +212,41 @@ __global__ void __launch_bounds__(i4::THREADS, 1)
         float acc[64];
 #pragma unroll
         for (int i = 0; i < 64; ++i) acc[i] = 0.0f;
+        // the scales of group gi+1 are fetched while group gi is rescaled, so no
+        // global-memory latency sits between two groups
+        const int mrow = min(m, g.sfa_ld - 1);
+        float sa_next = sfa[mrow];
+        float sb_next = rt < 128 ? sfb[n_tile * kBN_I4 + rt] : 0.0f;
         // After a failed wait the loop keeps running (without waiting or reading
         // TMEM) so that every rescale thread passes the same named barriers.
         bool ok = true;
         for (int gi = 0; gi < G; ++gi) {
             const int buf = gi & 1;
             float* sbb = sb_smem + buf * 128;
-            if (rt < 128) sbb[rt] = sfb[(size_t)gi * g.sfb_ld + n_tile * kBN_I4 + rt];
-            const float sa = sfa[(size_t)gi * g.sfa_ld + min(m, g.sfa_ld - 1)];
+            if (rt < 128) sbb[rt] = sb_next;
+            const float sa = sa_next;
+            if (gi + 1 < G) {
+                sa_next = sfa[(size_t)(gi + 1) * g.sfa_ld + mrow];
+                if (rt < 128) sb_next = sfb[(size_t)(gi + 1) * g.sfb_ld + n_tile * kBN_I4 + rt];
+            }
             named_bar(1, 256);
             if (ok) ok = mbar_wait(&accf[buf], (gi >> 1) & 1, limit, abort_flag);
             if (!ok) continue;
             tc_fence_after();
+            const uint64_t sa2 = pack2(sa);
 #pragma unroll
             for (int ch = 0; ch < 2; ++ch) {
                 uint32_t r[32];
                 tmem_ld_32x32b_x32(tmem + ((uint32_t)(q * 32) << 16) + buf * 128 + 64 * half + 32 * ch, r);
                 tmem_ld_wait();
+                const float4* sb4 = reinterpret_cast<const float4*>(sbb + 64 * half + 32 * ch);
 #pragma unroll
-                for (int i = 0; i < 32; ++i) {
-                    const float sc = __fmul_rn(sa, sbb[64 * half + 32 * ch + i]);
-                    acc[32 * ch + i] = __fmaf_rn(__int2float_rn((int)r[i]), sc, acc[32 * ch + i]);
+                for (int i = 0; i < 8; ++i) {
+                    const float4 b = sb4[i];
+                    // acc += float(P) * (sa * sb), two columns per packed FP32 operation
+                    rescale2(acc[32 * ch + 4 * i], acc[32 * ch + 4 * i + 1], r[4 * i], r[4 * i + 1], sa2, b.x, b.y);
+                    rescale2(acc[32 * ch + 4 * i + 2], acc[32 * ch + 4 * i + 3], r[4 * i + 2], r[4 * i + 3], sa2, b.z,
+                             b.w);
                 }
             }
             tc_fence_before();

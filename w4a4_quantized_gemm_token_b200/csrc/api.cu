@@ -80,19 +80,6 @@ int make_map(CUtensorMap* map, const void* base, int rows, int row_bytes, int bo
     return r == CUDA_SUCCESS ? W4A4_OK : W4A4_ERR_CUDA;
 }
 
-// 3-D byte tensor map over scale atoms [row_tiles][col_atoms][512 bytes], seen
-// as [row_tiles][2*col_atoms][256]: a box of box_atoms atoms of box_tiles row tiles.
-int make_map_sf(CUtensorMap* map, const void* base, int row_tiles, int col_atoms, int box_atoms, int box_tiles) {
-    cuuint64_t dims[3] = {256, (cuuint64_t)(2 * col_atoms), (cuuint64_t)row_tiles};
-    cuuint64_t strides[2] = {256, (cuuint64_t)col_atoms * 512};
-    cuuint32_t box[3] = {256, (cuuint32_t)(2 * box_atoms), (cuuint32_t)box_tiles};
-    cuuint32_t estr[3] = {1, 1, 1};
-    CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(base), dims, strides, box, estr,
-                          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
-                          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-    return r == CUDA_SUCCESS ? W4A4_OK : W4A4_ERR_CUDA;
-}
-
 // 3-D byte tensor map over codes[rows][row_bytes] (row_bytes a multiple of 128)
 // seen as (128-byte K-block, row, K-block): a box of box_rows rows x box_kb
 // consecutive K-blocks lands as box_kb 128-byte-swizzled [box_rows][128] tiles.
@@ -103,6 +90,21 @@ int make_map_kblocks(CUtensorMap* map, const void* base, int rows, int row_bytes
     cuuint32_t estr[3] = {1, 1, 1};
     CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(base), dims, strides, box, estr,
                           CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? W4A4_OK : W4A4_ERR_CUDA;
+}
+
+// 5-D byte tensor map over scale atoms [row_tiles][col_atoms][512 bytes] that
+// repeats every atom 4 times: (256-byte half, half, repeat [stride 0], atom,
+// row tile).  A box of box_atoms atoms x box_tiles row tiles lands as
+// [tile][atom][repeat][512].
+int make_map_sf_rep(CUtensorMap* map, const void* base, int row_tiles, int col_atoms, int box_atoms, int box_tiles) {
+    cuuint64_t dims[5] = {256, 2, 4, (cuuint64_t)col_atoms, (cuuint64_t)row_tiles};
+    cuuint64_t strides[4] = {256, 0, 512, (cuuint64_t)col_atoms * 512};
+    cuuint32_t box[5] = {256, 2, 4, (cuuint32_t)box_atoms, (cuuint32_t)box_tiles};
+    cuuint32_t estr[5] = {1, 1, 1, 1, 1};
+    CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 5, const_cast<void*>(base), dims, strides, box, estr,
+                          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
                           CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS ? W4A4_OK : W4A4_ERR_CUDA;
 }
@@ -200,9 +202,9 @@ int setup_gemm(const w4a4_qtensor* A, const w4a4_qtensor* B, uint16_t* Y, int ld
         rc = make_map(&s->ta, A->codes, A->rows, row_bytes, 128, kBM, true);
         if (rc == W4A4_OK) rc = make_map(&s->tb, B->codes, B->rows, row_bytes, 128, kBM, true);
         if (rc == W4A4_OK)
-            rc = make_map_sf(&s->tsa, A->scales, pad128(A->rows) / 128, g.sf_col_atoms, atoms_ps, 1);
+            rc = make_map_sf_rep(&s->tsa, A->scales, pad128(A->rows) / 128, g.sf_col_atoms, atoms_ps, 1);
         if (rc == W4A4_OK)
-            rc = make_map_sf(&s->tsb, B->scales, pad128(B->rows) / 128, g.sf_col_atoms, atoms_ps, 2);
+            rc = make_map_sf_rep(&s->tsb, B->scales, pad128(B->rows) / 128, g.sf_col_atoms, atoms_ps, 2);
     } else if (!decode) {
         rc = make_map(&s->ta, A->codes, A->rows, row_bytes, 128, kBM, true);
         if (rc == W4A4_OK) rc = make_map(&s->tb, B->codes, B->rows, row_bytes, 128, kBN, true);

@@ -14,17 +14,24 @@
 //     128..255 in the odd CTA's;
 //   - one pair scale-factor copy fills both CTAs' tensor memory, each from
 //     its own shared memory: A's scales are per CTA, B's (all 256 rows) are
-//     staged by both, so a pair issues 3 copies per K = 64 where two one-CTA
-//     tiles of the same work would issue 6.
+//     staged by both.  The MMA reads row r's scales from TMEM lane r, column
+//     base + r/32, so every lane quarter needs the whole 32 x 16-byte atom:
+//     the atoms arrive already repeated four times (a TMA box over a
+//     zero-stride dimension), and one 128 x 256-bit copy then fills the
+//     columns of two atoms -- 6 copies per 256-wide K stage instead of 12
+//     replicating 32 x 128-bit ones.
+//   - the MMA thread issues each stage's copies itself, interleaved with its
+//     4 MMAs (one thread's tcgen05 operations execute in order, so no barrier
+//     sits between a copy and the MMA that reads it, and the tensor pipe
+//     overlaps each copy with the MMA before it).
 // All loads are tiled TMA copies without multicast; the odd CTA's copies
 // count their bytes on the even CTA's stage barrier (cta_group::2 form),
-// whose expected byte count covers both CTAs.  Scale atoms arrive as 3-D
-// boxes, so out-of-range row tiles and K tails are zero-filled by the copy.
+// whose expected byte count covers both CTAs.  Out-of-range row tiles and K
+// tails are zero-filled by the copies.
 // Warp roles (384 threads per CTA):
-//   warp 0 lane 0   TMA producer (both CTAs), 5-stage ring
+//   warp 0 lane 0   TMA producer (both CTAs), 4-stage (NVFP4) / 5-stage (MXFP4) ring
 //   warp 1          TMEM allocation (both CTAs, together); even CTA lane 0
-//                   issues the MMAs
-//   warp 2 lane 0   even CTA: scale-factor copies
+//                   issues the scale copies and the MMAs
 //   warps 4..11     epilogue (both CTAs): TMEM -> registers -> bf16 stores,
 //                   two warps per lane quarter so the accumulator drains fast
 // Every wait is bounded; on expiry the kernel records a timeout, drains its
@@ -41,23 +48,29 @@ namespace pp {
 constexpr int BM = 256;                       // pair tile rows of A (128 per CTA)
 constexpr int BN = 256;                       // pair tile rows of B
 constexpr int HALF = 128;                     // rows of A and of B staged by one CTA
-constexpr int STAGES = 5;
 constexpr int A_BYTES = HALF * 128;           // 16 KB of A codes (K = 256 per stage)
 constexpr int B_BYTES = HALF * 128;           // 16 KB of B codes
 constexpr int ATOM = 512;                     // 128 rows x 4 scales
-constexpr int SFA_C = 4 * ATOM;               // this CTA's A scale atoms of a stage
-constexpr int SFB_C = 2 * 4 * ATOM;           // B scale atoms of both row halves
-constexpr int STAGE = A_BYTES + B_BYTES + SFA_C + SFB_C;
-constexpr int BAR_OFF = STAGES * STAGE;
-constexpr int SMEM = BAR_OFF + 256 + 1024;
+constexpr int REP = 4;                        // each atom staged 4 times (the TMEM lane quarters)
 constexpr int SF_COLS = 48;                   // TMEM per stage: A 16 + B 32 columns
 constexpr int SF_COL0 = BN;                   // after the accumulator
 constexpr int TMEM_COLS = 512;
 constexpr int THREADS = 384;
 constexpr int EPI_WARPS = 8;                  // two per TMEM lane quarter, 128 columns each
-static_assert(STAGE % 1024 == 0, "stages keep the 1024-byte alignment of swizzled tiles");
-static_assert(SF_COL0 + STAGES * SF_COLS <= TMEM_COLS, "tensor memory holds 512 columns");
-static_assert(SMEM <= 232448, "shared memory per block");
+// Per format: NVFP4 stages 4 scale atoms per 128 rows and K-stage, MXFP4 2.
+template <bool NV>
+struct Cfg {
+    static constexpr int ATOMS = NV ? 4 : 2;
+    static constexpr int SFA_C = ATOMS * REP * ATOM;      // this CTA's A scale atoms of a stage
+    static constexpr int SFB_C = 2 * ATOMS * REP * ATOM;  // B scale atoms of both row halves
+    static constexpr int STAGE = A_BYTES + B_BYTES + SFA_C + SFB_C;
+    static constexpr int STAGES = NV ? 4 : 5;
+    static constexpr int BAR_OFF = STAGES * STAGE;
+    static constexpr int SMEM = BAR_OFF + 256 + 1024;
+    static_assert(STAGE % 1024 == 0, "stages keep the 1024-byte alignment of swizzled tiles");
+    static_assert(SF_COL0 + STAGES * SF_COLS <= TMEM_COLS, "tensor memory holds 512 columns");
+    static_assert(SMEM <= 232448, "shared memory per block");
+};
 }  // namespace pp
 
 template <bool NV>
@@ -66,6 +79,8 @@ __global__ void __launch_bounds__(pp::THREADS, 1)
                          const __grid_constant__ CUtensorMap tmSA, const __grid_constant__ CUtensorMap tmSB,
                          GemmArgs g) {
     using namespace pp;
+    using C = Cfg<NV>;
+    constexpr int STAGES = C::STAGES, STAGE = C::STAGE, SFA_C = C::SFA_C, BAR_OFF = C::BAR_OFF;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint64_t* full = reinterpret_cast<uint64_t*>(smem + BAR_OFF);
@@ -86,7 +101,7 @@ __global__ void __launch_bounds__(pp::THREADS, 1)
     const int num_a = (g.M + BM - 1) / BM, num_b = (g.N + BN - 1) / BN;
     const int ntiles = num_a * num_b;
     const uint64_t limit = g.wait_limit_ns;
-    const int atoms_ps = NV ? 4 : 2;  // scale atoms per 256-wide K stage and 128 rows
+    constexpr int atoms_ps = C::ATOMS;  // scale atoms per 256-wide K stage and 128 rows
     // grouped raster: a group of A tiles (about 40 MB of A codes and scales, so
     // it stays in L2) is swept against every B tile, so B is read from HBM once
     // per group
@@ -134,7 +149,7 @@ __global__ void __launch_bounds__(pp::THREADS, 1)
     if (warp == 0) {
         if (lane == 0) {
             // ------------------------------ producer ------------------------------
-            const uint32_t stage_tx = 2u * (A_BYTES + B_BYTES + 3u * atoms_ps * ATOM);
+            const uint32_t stage_tx = 2u * (A_BYTES + B_BYTES + 3u * atoms_ps * REP * ATOM);
             int it = 0;
             for (int t = pair; t < ntiles && !*abort_flag; t += npairs) {
                 int at, bt;
@@ -149,8 +164,8 @@ __global__ void __launch_bounds__(pp::THREADS, 1)
                     const int atom_k0 = kt * atoms_ps;
                     tma_load_2d_pair(st, &tmA, kt * 128, at * BM + (int)rank * HALF, bar);
                     tma_load_2d_pair(st + A_BYTES, &tmB, kt * 128, bt * BN + (int)rank * HALF, bar);
-                    tma_load_3d_pair(st + A_BYTES + B_BYTES, &tmSA, 0, 2 * atom_k0, at * 2 + (int)rank, bar);
-                    tma_load_3d_pair(st + A_BYTES + B_BYTES + SFA_C, &tmSB, 0, 2 * atom_k0, bt * 2, bar);
+                    tma_load_5d_pair(st + A_BYTES + B_BYTES, &tmSA, 0, 0, 0, atom_k0, at * 2 + (int)rank, bar);
+                    tma_load_5d_pair(st + A_BYTES + B_BYTES + SFA_C, &tmSB, 0, 0, 0, atom_k0, bt * 2, bar);
                 }
                 if (*abort_flag) break;
             }
@@ -200,9 +215,10 @@ __global__ void __launch_bounds__(pp::THREADS, 1)
     } else if (warp == 2) {
         if (lane == 0 && leader) {
             // ------------------------- scale-factor copies -------------------------
-            // The tensor pipe overlaps these copies with the MMAs only when they
-            // come from another thread than the MMAs (a thread's tcgen05
-            // instructions block for about their execution time).
+            // From another thread than the MMAs (a thread's tcgen05 instructions
+            // block for about their execution time, and the pipe overlaps copies
+            // with MMAs of other threads).  A: atoms 2p, 2p+1 (4 repeats each, 2 KB
+            // apart) -> columns 8p .. 8p+7; B: atom j of row halves 0 and 1 -> 8j .. 8j+7.
             bool ok = true;
             int it = 0;
             for (int t = pair; t < ntiles && ok; t += npairs) {
@@ -217,11 +233,11 @@ __global__ void __launch_bounds__(pp::THREADS, 1)
                     const uint32_t sfa_t = tmem + SF_COL0 + s * SF_COLS, sfb_t = sfa_t + 16;
                     const int nk = min(4, (g.K - kt * kBK_FP4) / 64);
                     const int atoms = NV ? nk : (nk + 1) / 2;
-                    for (int j = 0; j < atoms; ++j) {
-                        tc_cp_pair_32x128b_x4(sfa_t + 4 * j, desc_sf_32x16(ca + j * ATOM));
-                        tc_cp_pair_32x128b_x4(sfb_t + 8 * j, desc_sf_32x16(cb + j * ATOM));
-                        tc_cp_pair_32x128b_x4(sfb_t + 8 * j + 4, desc_sf_32x16(cb + (atoms_ps + j) * ATOM));
-                    }
+                    for (int pa = 0; pa < (atoms + 1) / 2; ++pa)
+                        tc_cp_pair_128x256b(sfa_t + 8 * pa, smem_desc(ca + pa * 2 * REP * ATOM, REP * ATOM, 128, 0));
+                    for (int j = 0; j < atoms; ++j)
+                        tc_cp_pair_128x256b(sfb_t + 8 * j,
+                                            smem_desc(cb + j * REP * ATOM, atoms_ps * REP * ATOM, 128, 0));
                     tc_commit_pair(sfull + s);
                 }
             }
@@ -284,7 +300,8 @@ cudaError_t launch_gemm_fp4_pair(bool nvfp4, const CUtensorMap& tmA, const CUten
     auto kern = nvfp4 ? gemm_fp4_pair_kernel<true> : gemm_fp4_pair_kernel<false>;
     static bool attr_set[2] = {false, false};
     if (!attr_set[nvfp4]) {
-        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, pp::SMEM);
+        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             nvfp4 ? pp::Cfg<true>::SMEM : pp::Cfg<false>::SMEM);
         if (e != cudaSuccess) return e;
         attr_set[nvfp4] = true;
     }
@@ -295,7 +312,7 @@ cudaError_t launch_gemm_fp4_pair(bool nvfp4, const CUtensorMap& tmA, const CUten
         cudaLaunchConfig_t q = {};
         q.gridDim = dim3(2 * (num_sms / 2));
         q.blockDim = dim3(pp::THREADS);
-        q.dynamicSmemBytes = pp::SMEM;
+        q.dynamicSmemBytes = nvfp4 ? pp::Cfg<true>::SMEM : pp::Cfg<false>::SMEM;
         cudaLaunchAttribute ca[1];
         ca[0].id = cudaLaunchAttributeClusterDimension;
         ca[0].val.clusterDim.x = 2;
@@ -315,7 +332,7 @@ cudaError_t launch_gemm_fp4_pair(bool nvfp4, const CUtensorMap& tmA, const CUten
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(2 * pairs);
     cfg.blockDim = dim3(pp::THREADS);
-    cfg.dynamicSmemBytes = pp::SMEM;
+    cfg.dynamicSmemBytes = nvfp4 ? pp::Cfg<true>::SMEM : pp::Cfg<false>::SMEM;
     cfg.stream = st;
     cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeClusterDimension;

@@ -73,8 +73,8 @@ cudaError_t launch_gemm_fp4(bool nvfp4, const CUtensorMap& tmA, const CUtensorMa
                             int num_sms, bool pdl, cudaStream_t st);
 // The same product on clusters of two CTAs (tcgen05 cta_group::2), 256 x 256
 // output tiles: tmA/tmB boxes of 128 x 128 bytes (each CTA stages its half of
-// A and of B), tmSA/tmSB 3-D maps over the scale atoms (boxes of one stage's
-// atoms for 1 (A) and 2 (B) row tiles).
+// A and of B), tmSA/tmSB 5-D maps over the scale atoms that repeat each atom
+// four times (boxes of one stage's atoms for 1 (A) and 2 (B) row tiles).
 cudaError_t launch_gemm_fp4_pair(bool nvfp4, const CUtensorMap& tmA, const CUtensorMap& tmB, const CUtensorMap& tmSA,
                                  const CUtensorMap& tmSB, const GemmArgs& g, int num_sms, bool pdl, cudaStream_t st);
 // Small-M variant (M <= 16): weights take the MMA's M side (128 rows per tile),

@@ -39,6 +39,23 @@ FP4_PER_BF16 = 4.0        # nominal dense FP4 / BF16 tensor throughput (9 / 2.25
 INT8_PER_BF16 = 2.0       # nominal dense INT8 / BF16 (4.5 / 2.25)
 
 
+# DRAM traffic (dram__bytes_read.sum + dram__bytes_write.sum) per launch of the
+# dominant kernel, averaged over the five GEMM launches of one step, from the ncu
+# launch list summarised in profiles/launch_list_llama70b_layer_m4096.md; valid
+# only for the kernel source it was measured on (else reported as null).
+PROFILED_TRAFFIC = {"sources": ("gemm_fp4_pair.cu", "ptx.cuh"), "sha256_16": "06a561793d232171",
+                    "bytes_per_launch": 294.9e6}
+
+
+def profiled_traffic():
+    import hashlib
+    h = hashlib.sha256()
+    for f in PROFILED_TRAFFIC["sources"]:
+        with open(os.path.join(ROOT, "w4a4_quantized_gemm_token_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return PROFILED_TRAFFIC["bytes_per_launch"] if h.hexdigest()[:16] == PROFILED_TRAFFIC["sha256_16"] else None
+
+
 def peaks():
     try:
         p = json.load(open(PEAKS_FILE))
@@ -302,7 +319,7 @@ def run_ours(args, rank, world):
         del Xq
     gemm_tflops = gemm_flops / (gemm_ms * 1e-3) / 1e12
     roofline = {"bound": "tensor", "achieved": round(gemm_tflops, 1), "peak": round(fp4_peak, 1),
-                "unit": "TFLOP/s", "frac": round(gemm_tflops / fp4_peak, 4), "traffic": None,
+                "unit": "TFLOP/s", "frac": round(gemm_tflops / fp4_peak, 4), "traffic": profiled_traffic(),
                 "peak_src": f"{P['src']} bf16 burst x {FP4_PER_BF16:g} (nominal fp4/bf16)",
                 "kernel": "gemm_fp4_pair_kernel (NVFP4, 256x256 tile on a CTA pair)", "per_shape_tflops": per_shape}
 

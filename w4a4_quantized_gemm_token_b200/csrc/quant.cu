@@ -551,14 +551,14 @@ __global__ void __launch_bounds__(1024) compact_kernel(const int* selected, int 
 template <int J>
 __global__ void __launch_bounds__(J <= 2 ? 1024 : 768) quant_nvfp4_token_kernel(QuantArgs a, int nb) {
     pdl_launch_dependents();
-    extern __shared__ __align__(128) uint8_t qsm[];
+    extern __shared__ __align__(128) uint8_t qring[];
     __shared__ float wmax[32];
     __shared__ float2 tab[128];  // (d_c, RN(1/d_c)) for E4M3 codes c (sign 0)
     const int t = threadIdx.x, T = blockDim.x;
     const int lane = t & 31, warp = t >> 5, nwarps = T >> 5;
     const int items = a.K / 16;
     const int row_bytes = a.K * 2;
-    uint64_t* bars = reinterpret_cast<uint64_t*>(qsm + (size_t)nb * row_bytes);
+    uint64_t* bars = reinterpret_cast<uint64_t*>(qring + (size_t)nb * row_bytes);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + nb);
     const int G = gridDim.x;
     // rows of this CTA that are loaded: blockIdx.x + i*G < M
@@ -566,7 +566,7 @@ __global__ void __launch_bounds__(J <= 2 ? 1024 : 768) quant_nvfp4_token_kernel(
     auto issue = [&](int i) {
         const int b = i % nb, r = blockIdx.x + i * G;
         mbar_arrive_expect_tx(&bars[b], (uint32_t)row_bytes);
-        bulk_load(qsm + (size_t)b * row_bytes, a.X + (size_t)r * a.ldx, row_bytes, &bars[b]);
+        bulk_load(qring + (size_t)b * row_bytes, a.X + (size_t)r * a.ldx, row_bytes, &bars[b]);
     };
     if (t == 0) {
         for (int b = 0; b < nb; ++b) mbar_init(&bars[b], 1);
@@ -578,7 +578,7 @@ __global__ void __launch_bounds__(J <= 2 ? 1024 : 768) quant_nvfp4_token_kernel(
     for (int i = 0; i < nlive; ++i) {
         const int b = i % nb, r = blockIdx.x + i * G;
         if (!mbar_wait(&bars[b], (i / nb) & 1, 2000000000ull, abort_flag)) break;
-        const uint4* xr = reinterpret_cast<const uint4*>(qsm + (size_t)b * row_bytes);
+        const uint4* xr = reinterpret_cast<const uint4*>(qring + (size_t)b * row_bytes);
         uint32_t w[J][8];
 #pragma unroll
         for (int j = 0; j < J; ++j) {

@@ -297,9 +297,13 @@ __global__ void __launch_bounds__(Dec<KB>::THREADS, 1)
 }
 
 // Y[m, n] = bf16(alpha_m * sum of the tile's segment partials, in owner order).
+// One CTA per weight tile, one thread per (token, 4 adjacent rows): each
+// thread issues the float4 loads of all the tile's segments before adding
+// them, so the kernel costs one memory latency instead of one per segment.
 template <bool NV>
-__global__ void __launch_bounds__(256) decode_reduce_kernel(GemmArgs g, int grid_g) {
+__global__ void __launch_bounds__(512) decode_reduce_kernel(GemmArgs g, int grid_g) {
     pdl_wait();
+    constexpr int MAX_OWNERS = 16;
     const int KT = (g.K + kBK_FP4 - 1) / kBK_FP4;
     const int KG = (KT + decode_kb(g.K) - 1) / decode_kb(g.K);
     const int ntiles = (g.N + kBM - 1) / kBM;
@@ -307,17 +311,37 @@ __global__ void __launch_bounds__(256) decode_reduce_kernel(GemmArgs g, int grid
     const int nt = blockIdx.x;
     const int first = unit_owner((long long)nt * KG, U, grid_g);
     const int last = unit_owner((long long)(nt + 1) * KG - 1, U, grid_g);
-    for (int idx = threadIdx.x; idx < kBN_DEC * kBM; idx += blockDim.x) {
-        const int t = idx / kBM, row = idx % kBM;
-        const int n = nt * kBM + row;
-        if (t >= g.M || n >= g.N) continue;
-        float acc = 0.0f;
-        for (int c = first; c <= last; ++c)
-            acc += g.partial[((size_t)nt * g.splits + (c - first)) * (kBN_DEC * kBM) + idx];
-        const float alpha = NV ? __fmul_rn(g.s2a[g.s2a_per_row ? t : 0], g.s2b[0]) : 1.0f;
-        __nv_bfloat16 h = __float2bfloat16_rn(__fmul_rn(acc, alpha));
-        g.Y[(size_t)t * g.ldy + n] = *reinterpret_cast<uint16_t*>(&h);
+    const int t = threadIdx.x >> 5, r4 = (threadIdx.x & 31) * 4;  // token, first of 4 rows
+    if (t >= g.M) return;
+    const float4* slot = reinterpret_cast<const float4*>(g.partial + (size_t)nt * g.splits * (kBN_DEC * kBM) +
+                                                         t * kBM + r4);
+    const int owners = last - first + 1;
+    float4 v[MAX_OWNERS];
+#pragma unroll
+    for (int c = 0; c < MAX_OWNERS; ++c)
+        if (c < owners) v[c] = slot[(size_t)c * (kBN_DEC * kBM / 4)];
+    float4 acc = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+#pragma unroll
+    for (int c = 0; c < MAX_OWNERS; ++c)
+        if (c < owners) {
+            acc.x += v[c].x;
+            acc.y += v[c].y;
+            acc.z += v[c].z;
+            acc.w += v[c].w;
+        }
+    for (int c = MAX_OWNERS; c < owners; ++c) {  // more segments than the unrolled ones (many SMs, short K)
+        const float4 w = slot[(size_t)c * (kBN_DEC * kBM / 4)];
+        acc.x += w.x;
+        acc.y += w.y;
+        acc.z += w.z;
+        acc.w += w.w;
     }
+    const float alpha = NV ? __fmul_rn(g.s2a[g.s2a_per_row ? t : 0], g.s2b[0]) : 1.0f;
+    const int n = nt * kBM + r4;
+    __nv_bfloat162 h0 = __floats2bfloat162_rn(__fmul_rn(acc.x, alpha), __fmul_rn(acc.y, alpha));
+    __nv_bfloat162 h1 = __floats2bfloat162_rn(__fmul_rn(acc.z, alpha), __fmul_rn(acc.w, alpha));
+    *reinterpret_cast<uint2*>(g.Y + (size_t)t * g.ldy + n) =
+        make_uint2(*reinterpret_cast<uint32_t*>(&h0), *reinterpret_cast<uint32_t*>(&h1));
 }
 
 static cudaError_t launch_pdl(const void* kern, dim3 grid, dim3 block, size_t smem, cudaStream_t st, void** args) {
@@ -374,7 +398,7 @@ static cudaError_t launch_dec_t(const CUtensorMap& tmW, const CUtensorMap& tmX, 
     int gg = G;
     void* rargs[] = {&g, &gg};
     return launch_pdl(reinterpret_cast<const void*>(decode_reduce_kernel<NV>), dim3((g.N + kBM - 1) / kBM),
-                      dim3(256), 0, st, rargs);
+                      dim3(kBN_DEC * kBM / 4), 0, st, rargs);
 }
 
 int decode_k_blocks(int K) { return decode_kb(K); }

@@ -129,8 +129,10 @@ int cuda_status(cudaError_t e) { return e == cudaSuccess ? W4A4_OK : W4A4_ERR_CU
 
 // Quantize rows [0, M) of X into the first K columns of q (q->cols >= K).
 int quantize_rows(const uint16_t* X, int M, int K, int ldx, const int32_t* S, int K_src, const float* static_s2,
-                  w4a4_qtensor* q, int num_sms, cudaStream_t st) {
+                  w4a4_qtensor* q, int num_sms, cudaStream_t st, int* zero_words = nullptr, int zero_count = 0) {
     QuantArgs a{};
+    a.zero_words = zero_words;
+    a.zero_count = zero_count;
     a.X = X;
     a.M = M;
     a.K = K;
@@ -222,7 +224,7 @@ int setup_gemm(const w4a4_qtensor* A, const w4a4_qtensor* B, uint16_t* Y, int ld
 }
 
 int run_gemm(const w4a4_qtensor* A, const w4a4_qtensor* B, uint16_t* Y, int ldy, float* partial, int num_sms,
-             bool pdl, cudaStream_t st) {
+             bool pdl, cudaStream_t st, int* tile_count = nullptr) {
     const bool decode = A->format != W4A4_INT4 && partial != nullptr;
     GemmSetup s;
     int rc = setup_gemm(A, B, Y, ldy, decode, &s);
@@ -232,6 +234,7 @@ int run_gemm(const w4a4_qtensor* A, const w4a4_qtensor* B, uint16_t* Y, int ldy,
         e = launch_gemm_int4(s.ta, s.tb, s.g, num_sms, pdl, st);
     } else if (decode) {
         s.g.partial = partial;
+        s.g.tile_count = tile_count;
         e = launch_gemm_fp4_decode(A->format == W4A4_NVFP4, s.ta, s.tb, s.g, num_sms, st);
     } else if (use_pair(A)) {
         e = launch_gemm_fp4_pair(A->format == W4A4_NVFP4, s.ta, s.tb, s.tsa, s.tsb, s.g, num_sms, pdl, st);
@@ -244,7 +247,7 @@ int run_gemm(const w4a4_qtensor* A, const w4a4_qtensor* B, uint16_t* Y, int ldy,
 // Workspace layout of w4a4_linear: quantized activation (codes, scales, s2),
 // then the split-K partial sums of the small-M variant.
 struct WsLayout {
-    size_t codes, scales, s2, partial, total;
+    size_t codes, scales, s2, partial, counters, total;
 };
 
 WsLayout ws_layout(int M, int N, int K, int fmt, int nS) {
@@ -264,7 +267,9 @@ WsLayout ws_layout(int M, int N, int K, int fmt, int nS) {
         const int ntiles = (N + kBM - 1) / kBM;
         pb = (size_t)ntiles * decode_max_owners(N, cols, 1024) * kBN_DEC * kBM * sizeof(float);
     }
-    w.total = w.partial + align256(pb);
+    w.counters = w.partial + align256(pb);
+    const size_t nb = (fmt != W4A4_INT4 && M <= 16) ? (size_t)((N + kBM - 1) / kBM) * sizeof(int) : 0;
+    w.total = w.counters + align256(nb);
     return w;
 }
 
@@ -394,15 +399,18 @@ int w4a4_linear(const uint16_t* X, int M, int K, int ldx, const w4a4_qtensor* Wq
     xq.codes = base + L.codes;
     xq.scales = base + L.scales;
     xq.s2 = reinterpret_cast<float*>(base + L.s2);
-    rc = quantize_rows(X, M, K, ldx, nullptr, K, nullptr, &xq, sms, st);
+    const bool small_m = fmt != W4A4_INT4 && M <= 16;
+    int* counters = small_m ? reinterpret_cast<int*>(base + L.counters) : nullptr;
+    // the quantizer clears the decode GEMM's per-tile counters on its way
+    rc = quantize_rows(X, M, K, ldx, nullptr, K, nullptr, &xq, sms, st, counters, small_m ? (N + kBM - 1) / kBM : 0);
     if (rc != W4A4_OK) return rc;
     if (nS) {
         ResidualArgs r{X, M, K, ldx, pad128(M), S, nS, static_cast<uint8_t*>(xq.codes), xq.cols / 2,
                        static_cast<uint8_t*>(xq.scales), xq.cols / 16 / 4, xq.s2, xq.scale_mode};
         if (launch_residual(r, st) != cudaSuccess) return W4A4_ERR_CUDA;
     }
-    float* partial = (fmt != W4A4_INT4 && M <= 16) ? reinterpret_cast<float*>(base + L.partial) : nullptr;
-    return run_gemm(&xq, Wq, Y, ldy, partial, sms, true, st);
+    float* partial = small_m ? reinterpret_cast<float*>(base + L.partial) : nullptr;
+    return run_gemm(&xq, Wq, Y, ldy, partial, sms, true, st, counters);
 }
 
 int w4a4_augment_residual(const uint16_t* X, int M, int K, int ldx, const int32_t* S, int nS, w4a4_qtensor* Xaug,

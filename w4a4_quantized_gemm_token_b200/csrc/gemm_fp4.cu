@@ -11,8 +11,9 @@
 // much faster, and the box still lands as standard 128-byte-swizzled tiles.
 // A CTA accumulates in TMEM while its range stays in one weight tile and
 // writes an FP32 partial sum per tile segment (double-buffered
-// accumulators); a second kernel adds the segments of each tile in a fixed
-// order (deterministic), applies alpha and rounds to bf16.  Launched as a
+// accumulators); the CTA that writes a tile's last segment adds the tile's
+// segments in a fixed order (deterministic), applies alpha and rounds to
+// bf16.  Launched as a
 // programmatic dependent, the kernel starts streaming weights while the
 // activation quantizer still runs and waits only before its first activation
 // load.
@@ -61,6 +62,10 @@ __device__ __forceinline__ void tmem_ld_32x32b_x16(uint32_t taddr, uint32_t (&r)
         : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
           "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
         : "r"(taddr));
+}
+
+__device__ __forceinline__ void named_bar_sync(int id, int n) {
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
 }
 
 // First unit of CTA c when U units are split into G equal contiguous ranges.
@@ -140,7 +145,7 @@ __global__ void __launch_bounds__(Dec<KB>::THREADS, 1)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_holder;
-    pdl_launch_dependents();  // the reduction kernel may be scheduled; it waits for this grid
+    pdl_launch_dependents();  // the next launch may be scheduled; it waits for this grid
 
     if (warp == 0) {
         if (lane == 0) {
@@ -263,27 +268,95 @@ __global__ void __launch_bounds__(Dec<KB>::THREADS, 1)
         }
     } else if (warp >= 4) {
         // ------------------------------ epilogue ------------------------------
-        // segment partial sums -> workspace slot (tile, owner offset): [16 tokens][128 rows] FP32
+        // Segment partial sums -> workspace slot (tile, owner offset) [16 tokens][128
+        // rows] FP32.  The CTA whose segment completes a tile (a per-tile counter)
+        // adds all the tile's slots in owner order -- the same order whichever CTA
+        // arrives last -- applies alpha, writes Y and clears the counter.
         const int q = warp & 3;
+        const int row = q * 32 + lane;
+        __shared__ int last_flag;
+        // Every epilogue warp runs the same segments and named barriers; after a
+        // failed (timed-out) wait a warp only skips its TMEM read and stores.
         int seg = 0;
         long long u = u0;
+        bool waited = false, ok = true;
         while (u < u1) {
             const int nt = (int)(u / KG);
             const long long send = min(u1, (long long)(nt + 1) * KG);
             const int buf = seg & 1;
-            if (!mbar_wait(&accf[buf], (seg >> 1) & 1, limit, abort_flag, 20000)) break;
-            tc_fence_after();
-            uint32_t r[16];
-            tmem_ld_32x32b_x16(tmem + ((uint32_t)(q * 32) << 16) + buf * BN, r);
-            tmem_ld_wait();
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&acce[buf]);
             const int first = unit_owner((long long)nt * KG, U, G);
-            float* slot = g.partial + ((size_t)nt * g.splits + (blockIdx.x - first)) * (BN * kBM);
-            const int row = q * 32 + lane;
+            const int last = unit_owner((long long)(nt + 1) * KG - 1, U, G);
+            float* tile = g.partial + (size_t)nt * g.splits * (BN * kBM);
+            if (ok) ok = mbar_wait(&accf[buf], (seg >> 1) & 1, limit, abort_flag, 20000);
+            if (ok) {
+                tc_fence_after();
+                uint32_t r[16];
+                tmem_ld_32x32b_x16(tmem + ((uint32_t)(q * 32) << 16) + buf * BN, r);
+                tmem_ld_wait();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&acce[buf]);
+                float* slot = tile + (size_t)(blockIdx.x - first) * (BN * kBM);
 #pragma unroll
-            for (int t = 0; t < BN; ++t) slot[t * kBM + row] = __uint_as_float(r[t]);
+                for (int t = 0; t < BN; ++t) slot[t * kBM + row] = __uint_as_float(r[t]);
+            }
+            __threadfence();
+            named_bar_sync(1, 128);  // the four epilogue warps wrote their rows
+            if (threadIdx.x == 128) {
+                if (!waited) pdl_wait();  // the counters were cleared by the preceding launch
+                waited = true;
+                last_flag = !*abort_flag && atomicAdd(&g.tile_count[nt], 1) == last - first;
+            }
+            named_bar_sync(1, 128);
+            if (last_flag) {
+                __threadfence();
+                // thread e of the 128 takes positions (token, 4 rows) p = e, e+128, ...:
+                // the float4 loads of all its positions and segments are issued
+                // before any addition, so the tile costs about one memory latency
+                const int owners = last - first + 1, e = threadIdx.x - 128;
+                constexpr int PMAX = BN * kBM / 4 / 128, OMAX = 4;
+                float4 v[PMAX][OMAX];
+#pragma unroll
+                for (int pi = 0; pi < PMAX; ++pi) {
+                    const int p = e + 128 * pi, t = p >> 5, r4 = (p & 31) * 4;
+                    const float4* src = reinterpret_cast<const float4*>(tile + t * kBM + r4);
+#pragma unroll
+                    for (int c = 0; c < OMAX; ++c)
+                        if (t < g.M && c < owners) v[pi][c] = src[(size_t)c * (BN * kBM / 4)];
+                }
+#pragma unroll
+                for (int pi = 0; pi < PMAX; ++pi) {
+                    const int p = e + 128 * pi, t = p >> 5, r4 = (p & 31) * 4;
+                    if (t >= g.M) continue;
+                    const float4* src = reinterpret_cast<const float4*>(tile + t * kBM + r4);
+                    float4 acc = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+                    // fixed order: owner offset 0, 1, ...
+#pragma unroll
+                    for (int c = 0; c < OMAX; ++c)
+                        if (c < owners) {
+                            acc.x += v[pi][c].x;
+                            acc.y += v[pi][c].y;
+                            acc.z += v[pi][c].z;
+                            acc.w += v[pi][c].w;
+                        }
+                    for (int c = OMAX; c < owners; ++c) {
+                        const float4 w = src[(size_t)c * (BN * kBM / 4)];
+                        acc.x += w.x;
+                        acc.y += w.y;
+                        acc.z += w.z;
+                        acc.w += w.w;
+                    }
+                    const float alpha = NV ? __fmul_rn(g.s2a[g.s2a_per_row ? t : 0], g.s2b[0]) : 1.0f;
+                    const int n = nt * kBM + r4;
+                    __nv_bfloat162 h0 = __floats2bfloat162_rn(__fmul_rn(acc.x, alpha), __fmul_rn(acc.y, alpha));
+                    __nv_bfloat162 h1 = __floats2bfloat162_rn(__fmul_rn(acc.z, alpha), __fmul_rn(acc.w, alpha));
+                    if (n < g.N)
+                        *reinterpret_cast<uint2*>(g.Y + (size_t)t * g.ldy + n) =
+                            make_uint2(*reinterpret_cast<uint32_t*>(&h0), *reinterpret_cast<uint32_t*>(&h1));
+                }
+                if (threadIdx.x == 128) g.tile_count[nt] = 0;  // ready for the next call
+            }
+            named_bar_sync(1, 128);  // last_flag is rewritten for the next segment
             u = send;
             ++seg;
         }
@@ -294,54 +367,6 @@ __global__ void __launch_bounds__(Dec<KB>::THREADS, 1)
         tc_fence_after();
         tmem_dealloc(tmem, D::TMEM_COLS);
     }
-}
-
-// Y[m, n] = bf16(alpha_m * sum of the tile's segment partials, in owner order).
-// One CTA per weight tile, one thread per (token, 4 adjacent rows): each
-// thread issues the float4 loads of all the tile's segments before adding
-// them, so the kernel costs one memory latency instead of one per segment.
-template <bool NV>
-__global__ void __launch_bounds__(512) decode_reduce_kernel(GemmArgs g, int grid_g) {
-    pdl_wait();
-    constexpr int MAX_OWNERS = 16;
-    const int KT = (g.K + kBK_FP4 - 1) / kBK_FP4;
-    const int KG = (KT + decode_kb(g.K) - 1) / decode_kb(g.K);
-    const int ntiles = (g.N + kBM - 1) / kBM;
-    const long long U = (long long)ntiles * KG;
-    const int nt = blockIdx.x;
-    const int first = unit_owner((long long)nt * KG, U, grid_g);
-    const int last = unit_owner((long long)(nt + 1) * KG - 1, U, grid_g);
-    const int t = threadIdx.x >> 5, r4 = (threadIdx.x & 31) * 4;  // token, first of 4 rows
-    if (t >= g.M) return;
-    const float4* slot = reinterpret_cast<const float4*>(g.partial + (size_t)nt * g.splits * (kBN_DEC * kBM) +
-                                                         t * kBM + r4);
-    const int owners = last - first + 1;
-    float4 v[MAX_OWNERS];
-#pragma unroll
-    for (int c = 0; c < MAX_OWNERS; ++c)
-        if (c < owners) v[c] = slot[(size_t)c * (kBN_DEC * kBM / 4)];
-    float4 acc = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
-#pragma unroll
-    for (int c = 0; c < MAX_OWNERS; ++c)
-        if (c < owners) {
-            acc.x += v[c].x;
-            acc.y += v[c].y;
-            acc.z += v[c].z;
-            acc.w += v[c].w;
-        }
-    for (int c = MAX_OWNERS; c < owners; ++c) {  // more segments than the unrolled ones (many SMs, short K)
-        const float4 w = slot[(size_t)c * (kBN_DEC * kBM / 4)];
-        acc.x += w.x;
-        acc.y += w.y;
-        acc.z += w.z;
-        acc.w += w.w;
-    }
-    const float alpha = NV ? __fmul_rn(g.s2a[g.s2a_per_row ? t : 0], g.s2b[0]) : 1.0f;
-    const int n = nt * kBM + r4;
-    __nv_bfloat162 h0 = __floats2bfloat162_rn(__fmul_rn(acc.x, alpha), __fmul_rn(acc.y, alpha));
-    __nv_bfloat162 h1 = __floats2bfloat162_rn(__fmul_rn(acc.z, alpha), __fmul_rn(acc.w, alpha));
-    *reinterpret_cast<uint2*>(g.Y + (size_t)t * g.ldy + n) =
-        make_uint2(*reinterpret_cast<uint32_t*>(&h0), *reinterpret_cast<uint32_t*>(&h1));
 }
 
 static cudaError_t launch_pdl(const void* kern, dim3 grid, dim3 block, size_t smem, cudaStream_t st, void** args) {
@@ -392,13 +417,8 @@ static cudaError_t launch_dec_t(const CUtensorMap& tmW, const CUtensorMap& tmX, 
     g.splits = decode_max_owners(g.N, g.K, num_sms);  // slots per weight tile in the workspace
     CUtensorMap a = tmW, b = tmX;
     void* args[] = {&a, &b, &g};
-    cudaError_t e =
-        launch_pdl(reinterpret_cast<const void*>(kern), dim3(G), dim3(Dec<KB>::THREADS), Dec<KB>::SMEM, st, args);
-    if (e != cudaSuccess) return e;
-    int gg = G;
-    void* rargs[] = {&g, &gg};
-    return launch_pdl(reinterpret_cast<const void*>(decode_reduce_kernel<NV>), dim3((g.N + kBM - 1) / kBM),
-                      dim3(kBN_DEC * kBM / 4), 0, st, rargs);
+    return launch_pdl(reinterpret_cast<const void*>(kern), dim3(G), dim3(Dec<KB>::THREADS), Dec<KB>::SMEM, st,
+                      args);
 }
 
 int decode_k_blocks(int K) { return decode_kb(K); }

@@ -27,6 +27,8 @@ struct QuantArgs {
     float* s2_out;           // NVFP4 s2 ([1] or [M])
     const float* tensor_amax;  // NVFP4 tensor mode without static s2
     int rows_pad;              // pad128(M): rows of the scale atoms (set by the launcher)
+    int* zero_words;           // nullable: words the first CTA clears (a later kernel's counters)
+    int zero_count;
 };
 
 struct ResidualArgs {
@@ -54,6 +56,7 @@ struct GemmArgs {
     uint16_t* Y;
     int ldy;
     float* partial;            // split-K partial sums (decode variant)
+    int* tile_count;           // decode variant: per weight tile, segments written so far (start at 0)
     int splits;                // split-K factor (decode variant)
     int k_tiles_per_split;
     int skip_k_tile;           // debug: never load this k-tile (-1 = off)
@@ -79,8 +82,9 @@ cudaError_t launch_gemm_fp4_pair(bool nvfp4, const CUtensorMap& tmA, const CUten
                                  const CUtensorMap& tmSB, const GemmArgs& g, int num_sms, bool pdl, cudaStream_t st);
 // Small-M variant (M <= 16): weights take the MMA's M side (128 rows per tile),
 // the tokens its N side; the (tile, K-stage) units are split evenly over the
-// SMs, FP32 segment partials go to g.partial and a second kernel reduces them
-// into Y.  Both kernels are programmatic dependents of the preceding launch.
+// SMs, FP32 segment partials go to g.partial and the CTA that writes a tile's
+// last segment adds them into Y (g.tile_count[N/128] must be zero on entry and
+// is zero again on exit).  A programmatic dependent of the preceding launch.
 cudaError_t launch_gemm_fp4_decode(bool nvfp4, const CUtensorMap& tmW, const CUtensorMap& tmX, const GemmArgs& g,
                                    int num_sms, cudaStream_t st);
 // Partial-sum slots per weight tile of the small-M variant on `num_sms` SMs.

@@ -187,6 +187,8 @@ struct RowConsts {
 template <int FMT, bool GATHER>
 __global__ void __launch_bounds__(256, 4) quant_rows_kernel(QuantArgs a, int rows_per_cta, int nbuf) {
     pdl_launch_dependents();
+    if (blockIdx.x == 0)
+        for (int i = threadIdx.x; i < a.zero_count; i += blockDim.x) a.zero_words[i] = 0;
     extern __shared__ __align__(16) uint8_t qsm[];
     const int row_bytes = a.K_src * 2;                        // bf16 source row in shared memory
     const size_t buf_bytes = (size_t)rows_per_cta * row_bytes;
@@ -551,6 +553,8 @@ __global__ void __launch_bounds__(1024) compact_kernel(const int* selected, int 
 template <int J>
 __global__ void __launch_bounds__(J <= 2 ? 1024 : 768) quant_nvfp4_token_kernel(QuantArgs a, int nb) {
     pdl_launch_dependents();
+    if (blockIdx.x == 0)
+        for (int i = threadIdx.x; i < a.zero_count; i += blockDim.x) a.zero_words[i] = 0;
     extern __shared__ __align__(128) uint8_t qring[];
     __shared__ float wmax[32];
     __shared__ float2 tab[128];  // (d_c, RN(1/d_c)) for E4M3 codes c (sign 0)

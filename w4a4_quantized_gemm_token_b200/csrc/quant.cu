@@ -187,6 +187,7 @@ struct RowConsts {
 template <int FMT, bool GATHER>
 __global__ void __launch_bounds__(256, 4) quant_rows_kernel(QuantArgs a, int rows_per_cta, int nbuf) {
     pdl_launch_dependents();
+    pdl_wait();  // X and the words to clear may belong to the preceding launch
     if (blockIdx.x == 0)
         for (int i = threadIdx.x; i < a.zero_count; i += blockDim.x) a.zero_words[i] = 0;
     extern __shared__ __align__(16) uint8_t qsm[];
@@ -553,6 +554,7 @@ __global__ void __launch_bounds__(1024) compact_kernel(const int* selected, int 
 template <int J>
 __global__ void __launch_bounds__(J <= 2 ? 1024 : 768) quant_nvfp4_token_kernel(QuantArgs a, int nb) {
     pdl_launch_dependents();
+    pdl_wait();  // X and the words to clear may belong to the preceding launch
     if (blockIdx.x == 0)
         for (int i = threadIdx.x; i < a.zero_count; i += blockDim.x) a.zero_words[i] = 0;
     extern __shared__ __align__(128) uint8_t qring[];
@@ -656,6 +658,24 @@ __global__ void __launch_bounds__(J <= 2 ? 1024 : 768) quant_nvfp4_token_kernel(
             *reinterpret_cast<uint32_t*>(a.sf + sf_offset(r, 4 * c4, a.sf_col_atoms)) = 0u;
 }
 
+// Launch as a programmatic dependent of the preceding launch (the kernels wait
+// for it before touching memory it may write).
+template <typename... Args>
+static cudaError_t launch_dep(void (*kern)(Args...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                              Args... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kern, args...);
+}
+
 static cudaError_t launch_nvfp4_token(const QuantArgs& a, int rows_pad, int num_sms, cudaStream_t st) {
     // J items (32 J bytes of the row) per thread: two, so that the resident
     // CTAs bring enough warps to hide the per-item latency (at most 1024
@@ -685,15 +705,15 @@ static cudaError_t launch_nvfp4_token(const QuantArgs& a, int rows_pad, int num_
     if (J == 1) {
         static size_t attr = 0;
         if (smem > 48 * 1024 && smem > attr) e = cudaFuncSetAttribute(quant_nvfp4_token_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem), attr = smem;
-        if (e == cudaSuccess) quant_nvfp4_token_kernel<1><<<grid, T, smem, st>>>(b, nb);
+        if (e == cudaSuccess) e = launch_dep(quant_nvfp4_token_kernel<1>, dim3(grid), dim3(T), smem, st, b, nb);
     } else if (J == 2) {
         static size_t attr = 0;
         if (smem > 48 * 1024 && smem > attr) e = cudaFuncSetAttribute(quant_nvfp4_token_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem), attr = smem;
-        if (e == cudaSuccess) quant_nvfp4_token_kernel<2><<<grid, T, smem, st>>>(b, nb);
+        if (e == cudaSuccess) e = launch_dep(quant_nvfp4_token_kernel<2>, dim3(grid), dim3(T), smem, st, b, nb);
     } else {
         static size_t attr = 0;
         if (smem > 48 * 1024 && smem > attr) e = cudaFuncSetAttribute(quant_nvfp4_token_kernel<4>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem), attr = smem;
-        if (e == cudaSuccess) quant_nvfp4_token_kernel<4><<<grid, T, smem, st>>>(b, nb);
+        if (e == cudaSuccess) e = launch_dep(quant_nvfp4_token_kernel<4>, dim3(grid), dim3(T), smem, st, b, nb);
     }
     return e != cudaSuccess ? e : cudaGetLastError();
 }
@@ -724,8 +744,7 @@ static cudaError_t launch_quant_fmt(const QuantArgs& a, int rows_pad, int num_sm
     (void)num_sms;
     QuantArgs b = a;
     b.rows_pad = rows_pad;
-    kern<<<grid, T, smem, st>>>(b, rpc, nbuf);
-    return cudaGetLastError();
+    return launch_dep(kern, dim3(grid), dim3(T), smem, st, b, rpc, nbuf);
 }
 
 cudaError_t launch_quant(int fmt, bool gather, const QuantArgs& a, int rows_pad, int num_sms, cudaStream_t st) {

@@ -1,7 +1,7 @@
 // INT4-g128 W4A4 GEMM on the sm_100a 8-bit integer MMA (tcgen05.mma kind::i8).
 //
 // sm_100's tensor cores have no 4-bit integer kind, so the packed nibbles are
-// widened to int8 in shared memory.  Per 128-element K group g the MMA
+// widened to int8 in shared memory (as 16 * q, see widen8_x16).  Per 128-element K group g the MMA
 // produces the exact int32 partial sum P_g[m,n] = sum_{k in g} qa qw into one
 // of two TMEM buffers; CUDA-core warps rescale it,
 //     acc[m,n] += float(P_g[m,n]) * (sa[m,g] * sw[n,g])    (FP32),
@@ -36,16 +36,15 @@ constexpr int THREADS = 14 * 32;
 constexpr int TMEM_COLS = 256;                      // two int32 buffers of 128 columns
 }  // namespace i4
 
-// Sign-extend the 8 nibbles of w (element i in nibble i) into 8 int8 bytes,
-// returned as two words (elements 0-3, 4-7).
-__device__ __forceinline__ void widen8(uint32_t w, uint32_t& o0, uint32_t& o1) {
-    uint32_t lo = w & 0x0F0F0F0Fu;          // elements 0,2,4,6
-    uint32_t hi = (w >> 4) & 0x0F0F0F0Fu;   // elements 1,3,5,7
-    // per byte: n in [0,15] -> ((n ^ 8) + 0x78) ^ 0x80 = n - 16*(n >= 8), no carries between bytes
-    lo = ((lo ^ 0x08080808u) + 0x78787878u) ^ 0x80808080u;
-    hi = ((hi ^ 0x08080808u) + 0x78787878u) ^ 0x80808080u;
-    o0 = __byte_perm(lo, hi, 0x5140);  // e0 e1 e2 e3
-    o1 = __byte_perm(lo, hi, 0x7362);  // e4 e5 e6 e7
+// The 8 nibbles of w (element i in nibble i) as 8 int8 bytes holding 16 * q:
+// each nibble moves to the high half of its byte, whose sign bit is then the
+// nibble's, so no sign extension is needed (5 integer operations per 8
+// elements).  The MMA then yields 256 * P exactly (|256 P| <= 256 * 128 * 64).
+__device__ __forceinline__ void widen8_x16(uint32_t w, uint32_t& o0, uint32_t& o1) {
+    const uint32_t lo = (w << 4) & 0xF0F0F0F0u;  // elements 0,2,4,6
+    const uint32_t hi = w & 0xF0F0F0F0u;         // elements 1,3,5,7
+    o0 = __byte_perm(lo, hi, 0x5140);             // e0 e1 e2 e3
+    o1 = __byte_perm(lo, hi, 0x7362);             // e4 e5 e6 e7
 }
 
 __device__ __forceinline__ uint64_t pack2(float v) {
@@ -186,10 +185,10 @@ __global__ void __launch_bounds__(i4::THREADS, 1)
                     const int seg = lane & 3;
                     const uint4 w = *reinterpret_cast<const uint4*>(pk + row * 64 + seg * 16);
                     uint32_t o[8];
-                    widen8(w.x, o[0], o[1]);
-                    widen8(w.y, o[2], o[3]);
-                    widen8(w.z, o[4], o[5]);
-                    widen8(w.w, o[6], o[7]);
+                    widen8_x16(w.x, o[0], o[1]);
+                    widen8_x16(w.y, o[2], o[3]);
+                    widen8_x16(w.z, o[4], o[5]);
+                    widen8_x16(w.w, o[6], o[7]);
                     // 16-byte chunk c of the 128-byte row lands at chunk c ^ (row % 8)
                     const int c0 = 2 * seg, c1 = 2 * seg + 1;
                     *reinterpret_cast<uint4*>(un + row * 128 + ((c0 ^ (row & 7)) << 4)) = make_uint4(o[0], o[1], o[2], o[3]);
@@ -214,8 +213,10 @@ __global__ void __launch_bounds__(i4::THREADS, 1)
         for (int i = 0; i < 64; ++i) acc[i] = 0.0f;
         // the scales of group gi+1 are fetched while group gi is rescaled, so no
         // global-memory latency sits between two groups
+        // the MMA sums 16 qa * 16 qw = 256 P: scaling sa by 2^-8 (exact) gives
+        // float(256 P) * RN(2^-8 sa * sw) = float(P) * RN(sa * sw)
         const int mrow = min(m, g.sfa_ld - 1);
-        float sa_next = sfa[mrow];
+        float sa_next = sfa[mrow] * 0.00390625f;
         float sb_next = rt < 128 ? sfb[n_tile * kBN_I4 + rt] : 0.0f;
         // After a failed wait the loop keeps running (without waiting or reading
         // TMEM) so that every rescale thread passes the same named barriers.
@@ -226,7 +227,7 @@ __global__ void __launch_bounds__(i4::THREADS, 1)
             if (rt < 128) sbb[rt] = sb_next;
             const float sa = sa_next;
             if (gi + 1 < G) {
-                sa_next = sfa[(size_t)(gi + 1) * g.sfa_ld + mrow];
+                sa_next = sfa[(size_t)(gi + 1) * g.sfa_ld + mrow] * 0.00390625f;
                 if (rt < 128) sb_next = sfb[(size_t)(gi + 1) * g.sfb_ld + n_tile * kBN_I4 + rt];
             }
             named_bar(1, 256);

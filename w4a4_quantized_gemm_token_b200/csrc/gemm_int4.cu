@@ -9,7 +9,9 @@
 // is the cost the APEX4 paragraph ("Depth Registers..." thelatestinai page,
 // para 2) analyses through the tensor-core / CUDA-core throughput ratio.
 //
-// One CTA per 128 x 128 output tile, 14 warps:
+// Persistent (one CTA per SM, 128 x 128 output tiles in turn), 14 warps; the
+// MMA and unpack warps run ahead into the next tile while the rescale warps
+// finish and store the previous one:
 //   warp 0 lane 0   TMA producer: packed codes of A and B (64-byte rows).
 //   warp 1          TMEM owner; lane 0 issues 4 MMAs (K=32) per group.
 //   warps 2..5      unpack: nibbles -> int8, written in the 128-byte swizzled
@@ -89,12 +91,16 @@ __global__ void __launch_bounds__(i4::THREADS, 1)
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int G = g.K / 128;
     const uint64_t limit = g.wait_limit_ns;
-    // grouped raster over (m tile, n tile)
+    // persistent: tiles t = blockIdx.x, +gridDim.x, ...; grouped raster over (m tile, n tile)
     const int num_m = (g.M + 127) / 128, num_n = (g.N + kBN_I4 - 1) / kBN_I4;
-    const int GR = 8, per_group = GR * num_n;
-    const int grp = blockIdx.x / per_group, first = grp * GR, gsz = min(GR, num_m - first);
-    const int in = blockIdx.x - grp * per_group;
-    const int m_tile = first + in % gsz, n_tile = in / gsz;
+    const int ntiles = num_m * num_n;
+    auto coords = [&](int t, int& m_tile, int& n_tile) {
+        const int GR = 8, per_group = GR * num_n;
+        const int grp = t / per_group, first = grp * GR, gsz = min(GR, num_m - first);
+        const int in = t - grp * per_group;
+        m_tile = first + in % gsz;
+        n_tile = in / gsz;
+    };
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < STAGES; ++s) {
@@ -124,53 +130,59 @@ __global__ void __launch_bounds__(i4::THREADS, 1)
     const uint32_t tmem = *tmem_holder;
     pdl_wait();
 
+    // gi counts the groups of every tile this CTA processes, in order
     if (warp == 0) {
         if (lane == 0) {
             int gi = 0;
-            for (; gi < G; ++gi) {
-                const int s = gi % STAGES, n = gi / STAGES;
-                if (gi >= STAGES && !mbar_wait(&empty[s], (n - 1) & 1, limit, abort_flag)) break;
-                if (gi == g.skip_k_tile) continue;
-                uint8_t* st = smem + s * STAGE;
-                mbar_arrive_expect_tx(&full[s], 2 * PK_BYTES);
-                tma_load_2d(st + 2 * UN_BYTES, &tmA, gi * 64, m_tile * 128, &full[s]);
-                tma_load_2d(st + 2 * UN_BYTES + PK_BYTES, &tmB, gi * 64, n_tile * kBN_I4, &full[s]);
+            bool stop = false;
+            for (int t = blockIdx.x; t < ntiles && !stop; t += gridDim.x) {
+                int m_tile, n_tile;
+                coords(t, m_tile, n_tile);
+                for (int k = 0; k < G; ++k, ++gi) {
+                    const int s = gi % STAGES, n = gi / STAGES;
+                    if (gi >= STAGES && !mbar_wait(&empty[s], (n - 1) & 1, limit, abort_flag)) {
+                        stop = true;
+                        break;
+                    }
+                    if (k == g.skip_k_tile) continue;
+                    uint8_t* st = smem + s * STAGE;
+                    mbar_arrive_expect_tx(&full[s], 2 * PK_BYTES);
+                    tma_load_2d(st + 2 * UN_BYTES, &tmA, k * 64, m_tile * 128, &full[s]);
+                    tma_load_2d(st + 2 * UN_BYTES + PK_BYTES, &tmB, k * 64, n_tile * kBN_I4, &full[s]);
+                }
             }
             if (*abort_flag)
-                for (int j = max(0, gi - STAGES); j < gi; ++j)
-                    if (j != g.skip_k_tile) {
-                        const uint64_t t0 = globaltimer();
-                        while (!mbar_try_wait(&full[j % STAGES], (j / STAGES) & 1) && globaltimer() - t0 < 100000000ull) {
-                        }
-                    }
+                for (int j = max(0, gi - STAGES); j < gi; ++j) mbar_wait_drain(&full[j % STAGES], (j / STAGES) & 1, 100000000ull);
         }
     } else if (warp == 1) {
         if (lane == 0) {
             bool ok = true;
-            for (int gi = 0; gi < G; ++gi) {
-                const int s = gi % STAGES, n = gi / STAGES, buf = gi & 1;
-                if (!mbar_wait(&conv[s], n & 1, limit, abort_flag)) { ok = false; break; }
-                if (gi >= 2 && !mbar_wait(&tfree[buf], ((gi >> 1) - 1) & 1, limit, abort_flag)) { ok = false; break; }
-                tc_fence_after();
-                const uint32_t sA = smem_u32(smem + s * STAGE), sB = sA + UN_BYTES;
+            int gi = 0;
+            for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x) {
+                for (int k = 0; k < G; ++k, ++gi) {
+                    const int s = gi % STAGES, n = gi / STAGES, buf = gi & 1;
+                    if (!mbar_wait(&conv[s], n & 1, limit, abort_flag)) { ok = false; break; }
+                    if (gi >= 2 && !mbar_wait(&tfree[buf], ((gi >> 1) - 1) & 1, limit, abort_flag)) { ok = false; break; }
+                    tc_fence_after();
+                    const uint32_t sA = smem_u32(smem + s * STAGE), sB = sA + UN_BYTES;
 #pragma unroll
-                for (int j = 0; j < 4; ++j)
-                    mma_i8(tmem + buf * 128, desc_kmajor_sw128(sA + 32 * j), desc_kmajor_sw128(sB + 32 * j),
-                           idesc_i8(128, kBN_I4), j > 0 ? 1u : 0u);
-                tc_commit(&empty[s]);
-                tc_commit(&accf[buf]);
+                    for (int j = 0; j < 4; ++j)
+                        mma_i8(tmem + buf * 128, desc_kmajor_sw128(sA + 32 * j), desc_kmajor_sw128(sB + 32 * j),
+                               idesc_i8(128, kBN_I4), j > 0 ? 1u : 0u);
+                    tc_commit(&empty[s]);
+                    tc_commit(&accf[buf]);
+                }
             }
             if (!ok) {
                 tc_commit(drain);
-                const uint64_t t0 = globaltimer();
-                while (!mbar_try_wait(drain, 0) && globaltimer() - t0 < 100000000ull) {
-                }
+                mbar_wait_drain(drain, 0, 100000000ull);
             }
         }
     } else if (warp < 6) {
         // ------------------------------ unpack ------------------------------
         const int uw = warp - 2;  // 0..3
-        for (int gi = 0; gi < G; ++gi) {
+        const int total = ((ntiles - (int)blockIdx.x + (int)gridDim.x - 1) / (int)gridDim.x) * G;
+        for (int gi = 0; gi < total; ++gi) {
             const int s = gi % STAGES, n = gi / STAGES;
             if (!mbar_wait(&full[s], n & 1, limit, abort_flag)) break;
             uint8_t* st = smem + s * STAGE;
@@ -204,67 +216,74 @@ __global__ void __launch_bounds__(i4::THREADS, 1)
         const int q = warp & 3, half = (warp - 6) >> 2;
         const int rt = (warp - 6) * 32 + lane;  // 0..255
         const int row = q * 32 + lane;
-        const int m = m_tile * 128 + row;
-        const int ncol0 = n_tile * kBN_I4 + 64 * half;
         const float* sfa = reinterpret_cast<const float*>(g.sfa);
         const float* sfb = reinterpret_cast<const float*>(g.sfb);
-        float acc[64];
-#pragma unroll
-        for (int i = 0; i < 64; ++i) acc[i] = 0.0f;
-        // the scales of group gi+1 are fetched while group gi is rescaled, so no
-        // global-memory latency sits between two groups
-        // the MMA sums 16 qa * 16 qw = 256 P: scaling sa by 2^-8 (exact) gives
-        // float(256 P) * RN(2^-8 sa * sw) = float(P) * RN(sa * sw)
-        const int mrow = min(m, g.sfa_ld - 1);
-        float sa_next = sfa[mrow] * 0.00390625f;
-        float sb_next = rt < 128 ? sfb[n_tile * kBN_I4 + rt] : 0.0f;
+        // the scales of group gi+1 (possibly the next tile's first) are fetched
+        // while group gi is rescaled; the MMA sums 16 qa * 16 qw = 256 P, and
+        // scaling sa by 2^-8 (exact) gives float(256 P) * RN(2^-8 sa * sw) = float(P) * RN(sa * sw)
+        auto scales_of = [&](int t, int k, float& sa, float& sb) {
+            int m_tile, n_tile;
+            coords(t, m_tile, n_tile);
+            sa = sfa[(size_t)k * g.sfa_ld + min(m_tile * 128 + row, g.sfa_ld - 1)] * 0.00390625f;
+            sb = rt < 128 ? sfb[(size_t)k * g.sfb_ld + n_tile * kBN_I4 + rt] : 0.0f;
+        };
+        float sa_next = 0.0f, sb_next = 0.0f;
+        if ((int)blockIdx.x < ntiles) scales_of(blockIdx.x, 0, sa_next, sb_next);
         // After a failed wait the loop keeps running (without waiting or reading
         // TMEM) so that every rescale thread passes the same named barriers.
         bool ok = true;
-        for (int gi = 0; gi < G; ++gi) {
-            const int buf = gi & 1;
-            float* sbb = sb_smem + buf * 128;
-            if (rt < 128) sbb[rt] = sb_next;
-            const float sa = sa_next;
-            if (gi + 1 < G) {
-                sa_next = sfa[(size_t)(gi + 1) * g.sfa_ld + mrow] * 0.00390625f;
-                if (rt < 128) sb_next = sfb[(size_t)(gi + 1) * g.sfb_ld + n_tile * kBN_I4 + rt];
-            }
-            named_bar(1, 256);
-            if (ok) ok = mbar_wait(&accf[buf], (gi >> 1) & 1, limit, abort_flag);
-            if (!ok) continue;
-            tc_fence_after();
-            const uint64_t sa2 = pack2(sa);
+        int gi = 0;
+        for (int t = blockIdx.x; t < ntiles; t += gridDim.x) {
+            int m_tile, n_tile;
+            coords(t, m_tile, n_tile);
+            const int m = m_tile * 128 + row;
+            const int ncol0 = n_tile * kBN_I4 + 64 * half;
+            float acc[64];
 #pragma unroll
-            for (int ch = 0; ch < 2; ++ch) {
-                uint32_t r[32];
-                tmem_ld_32x32b_x32(tmem + ((uint32_t)(q * 32) << 16) + buf * 128 + 64 * half + 32 * ch, r);
-                tmem_ld_wait();
-                const float4* sb4 = reinterpret_cast<const float4*>(sbb + 64 * half + 32 * ch);
+            for (int i = 0; i < 64; ++i) acc[i] = 0.0f;
+            for (int k = 0; k < G; ++k, ++gi) {
+                const int buf = gi & 1;
+                float* sbb = sb_smem + buf * 128;
+                if (rt < 128) sbb[rt] = sb_next;
+                const float sa = sa_next;
+                if (k + 1 < G) scales_of(t, k + 1, sa_next, sb_next);
+                else if (t + (int)gridDim.x < ntiles) scales_of(t + gridDim.x, 0, sa_next, sb_next);
+                named_bar(1, 256);
+                if (ok) ok = mbar_wait(&accf[buf], (gi >> 1) & 1, limit, abort_flag);
+                if (!ok) continue;
+                tc_fence_after();
+                const uint64_t sa2 = pack2(sa);
 #pragma unroll
-                for (int i = 0; i < 8; ++i) {
-                    const float4 b = sb4[i];
-                    // acc += float(P) * (sa * sb), two columns per packed FP32 operation
-                    rescale2(acc[32 * ch + 4 * i], acc[32 * ch + 4 * i + 1], r[4 * i], r[4 * i + 1], sa2, b.x, b.y);
-                    rescale2(acc[32 * ch + 4 * i + 2], acc[32 * ch + 4 * i + 3], r[4 * i + 2], r[4 * i + 3], sa2, b.z,
-                             b.w);
+                for (int ch = 0; ch < 2; ++ch) {
+                    uint32_t r[32];
+                    tmem_ld_32x32b_x32(tmem + ((uint32_t)(q * 32) << 16) + buf * 128 + 64 * half + 32 * ch, r);
+                    tmem_ld_wait();
+                    const float4* sb4 = reinterpret_cast<const float4*>(sbb + 64 * half + 32 * ch);
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) {
+                        const float4 b = sb4[i];
+                        // acc += float(P) * (sa * sb), two columns per packed FP32 operation
+                        rescale2(acc[32 * ch + 4 * i], acc[32 * ch + 4 * i + 1], r[4 * i], r[4 * i + 1], sa2, b.x, b.y);
+                        rescale2(acc[32 * ch + 4 * i + 2], acc[32 * ch + 4 * i + 3], r[4 * i + 2], r[4 * i + 3], sa2,
+                                 b.z, b.w);
+                    }
                 }
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&tfree[buf]);
             }
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&tfree[buf]);
-        }
-        if (ok && m < g.M && ncol0 < g.N) {
-            uint16_t* dst = g.Y + (size_t)m * g.ldy + ncol0;
+            if (ok && m < g.M && ncol0 < g.N) {
+                uint16_t* dst = g.Y + (size_t)m * g.ldy + ncol0;
 #pragma unroll
-            for (int v = 0; v < 8; ++v) {
-                uint32_t pk[4];
+                for (int v = 0; v < 8; ++v) {
+                    uint32_t pk[4];
 #pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    __nv_bfloat162 h = __floats2bfloat162_rn(acc[8 * v + 2 * e], acc[8 * v + 2 * e + 1]);
-                    pk[e] = *reinterpret_cast<uint32_t*>(&h);
+                    for (int e = 0; e < 4; ++e) {
+                        __nv_bfloat162 h = __floats2bfloat162_rn(acc[8 * v + 2 * e], acc[8 * v + 2 * e + 1]);
+                        pk[e] = *reinterpret_cast<uint32_t*>(&h);
+                    }
+                    *reinterpret_cast<uint4*>(dst + 8 * v) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
                 }
-                *reinterpret_cast<uint4*>(dst + 8 * v) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
             }
         }
     }
@@ -276,7 +295,7 @@ __global__ void __launch_bounds__(i4::THREADS, 1)
     }
 }
 
-cudaError_t launch_gemm_int4(const CUtensorMap& tmA, const CUtensorMap& tmB, const GemmArgs& g, int /*num_sms*/,
+cudaError_t launch_gemm_int4(const CUtensorMap& tmA, const CUtensorMap& tmB, const GemmArgs& g, int num_sms,
                              bool pdl, cudaStream_t st) {
     static bool attr_set = false;
     if (!attr_set) {
@@ -286,7 +305,7 @@ cudaError_t launch_gemm_int4(const CUtensorMap& tmA, const CUtensorMap& tmB, con
     }
     const int tiles = ((g.M + 127) / 128) * ((g.N + kBN_I4 - 1) / kBN_I4);
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(tiles);
+    cfg.gridDim = dim3(tiles < num_sms ? tiles : num_sms);  // persistent: one CTA per SM
     cfg.blockDim = dim3(i4::THREADS);
     cfg.dynamicSmemBytes = i4::SMEM;
     cfg.stream = st;

@@ -144,28 +144,52 @@ __global__ void __launch_bounds__(pp::THREADS, 1)
     const uint32_t tmem = *tmem_holder;
     const uint32_t full_leader = mapa_shared(smem_u32(full), 0);
     const uint32_t acce_leader = mapa_shared(smem_u32(acce), 0);
-    pdl_wait();  // operands written by the preceding kernel are visible from here on
+    // operands written by the preceding kernel (A, its scales, s2a) are visible
+    // after this wait; the producer waits only before its first A load, so the
+    // weights of the first stages stream in while the quantizer finishes
+    if (!(warp == 0 && lane == 0)) pdl_wait();
 
     if (warp == 0) {
         if (lane == 0) {
             // ------------------------------ producer ------------------------------
             const uint32_t stage_tx = 2u * (A_BYTES + B_BYTES + 3u * atoms_ps * REP * ATOM);
+            auto load_b = [&](int s, int bt, int kt) {  // weights: independent of the preceding kernel
+                uint8_t* st = smem + s * STAGE;
+                const uint32_t bar = full_leader + 8u * s;
+                if (leader) mbar_arrive_expect_tx(&full[s], stage_tx);
+                tma_load_2d_pair(st + A_BYTES, &tmB, kt * 128, bt * BN + (int)rank * HALF, bar);
+                tma_load_5d_pair(st + A_BYTES + B_BYTES + SFA_C, &tmSB, 0, 0, 0, kt * atoms_ps, bt * 2, bar);
+            };
+            auto load_a = [&](int s, int at, int kt) {
+                uint8_t* st = smem + s * STAGE;
+                const uint32_t bar = full_leader + 8u * s;
+                tma_load_2d_pair(st, &tmA, kt * 128, at * BM + (int)rank * HALF, bar);
+                tma_load_5d_pair(st + A_BYTES + B_BYTES, &tmSA, 0, 0, 0, kt * atoms_ps, at * 2 + (int)rank, bar);
+            };
+            // the first stages' weights before the wait for the preceding kernel
+            int pre = 0;
+            if (pair < ntiles) {
+                int at, bt;
+                coords(pair, at, bt);
+                for (; pre < STAGES && pre < KT; ++pre)
+                    if (pre != g.skip_k_tile) load_b(pre, bt, pre);
+                pdl_wait();
+                for (int j = 0; j < pre; ++j)
+                    if (j != g.skip_k_tile) load_a(j, at, j);
+            } else {
+                pdl_wait();
+            }
             int it = 0;
             for (int t = pair; t < ntiles && !*abort_flag; t += npairs) {
                 int at, bt;
                 coords(t, at, bt);
                 for (int kt = 0; kt < KT; ++kt, ++it) {
+                    if (it < pre) continue;  // loaded above
                     const int s = it % STAGES, n = it / STAGES;
                     if (it >= STAGES && !mbar_wait(&empty[s], (n - 1) & 1, limit, abort_flag)) break;
                     if (kt == g.skip_k_tile) continue;  // test hook: this stage never fills
-                    uint8_t* st = smem + s * STAGE;
-                    const uint32_t bar = full_leader + 8u * s;
-                    if (leader) mbar_arrive_expect_tx(&full[s], stage_tx);
-                    const int atom_k0 = kt * atoms_ps;
-                    tma_load_2d_pair(st, &tmA, kt * 128, at * BM + (int)rank * HALF, bar);
-                    tma_load_2d_pair(st + A_BYTES, &tmB, kt * 128, bt * BN + (int)rank * HALF, bar);
-                    tma_load_5d_pair(st + A_BYTES + B_BYTES, &tmSA, 0, 0, 0, atom_k0, at * 2 + (int)rank, bar);
-                    tma_load_5d_pair(st + A_BYTES + B_BYTES + SFA_C, &tmSB, 0, 0, 0, atom_k0, bt * 2, bar);
+                    load_b(s, bt, kt);
+                    load_a(s, at, kt);
                 }
                 if (*abort_flag) break;
             }

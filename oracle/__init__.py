@@ -64,6 +64,9 @@ def _declare(L):
     L.orc_f64_to_bf16.argtypes = [C.c_double]; L.orc_f64_to_bf16.restype = C.c_uint16
     L.orc_nvfp4_s2_from_amax.argtypes = [C.c_float]; L.orc_nvfp4_s2_from_amax.restype = C.c_float
     L.orc_quant_nvfp4.argtypes = [_u16p, C.c_int, C.c_int, C.c_int, C.c_int, _f32p, _u8p, _u8p, _f32p]
+    L.orc_quant_nvfp4_segments.argtypes = [_u16p, C.c_int, C.c_int, C.c_int, _i32p, C.c_int, _u8p, _u8p, _f32p]
+    L.orc_gemm_nvfp4_wrows.argtypes = [_u8p, _u8p, _f32p, C.c_int, _u8p, _u8p, _f32p, C.c_int,
+                                       C.c_int, C.c_int, C.c_int, _u16p, _f64p, _f64p]
     L.orc_quant_mxfp4.argtypes = [_u16p, C.c_int, C.c_int, C.c_int, _u8p, _u8p]
     L.orc_quant_int4.argtypes = [_u16p, C.c_int, C.c_int, C.c_int, _u8p, _f32p]
     L.orc_dequant_nvfp4.argtypes = [_u8p, _u8p, _f32p, C.c_int, C.c_int, C.c_int, _f64p]
@@ -147,6 +150,20 @@ def quant_nvfp4(X, mode: int, static_s2=None):
     return codes, scales, s2
 
 
+def quant_nvfp4_segments(X, seg):
+    """Row segments [seg[i], seg[i+1]) quantized as separate NVFP4 tensors.
+    Returns (codes, scales, s2 per row [M])."""
+    X = _bf16(X)
+    M, K = X.shape
+    seg = np.ascontiguousarray(seg, np.int32)
+    codes = np.zeros((M, K // 2), np.uint8)
+    scales = np.zeros((M, K // 16), np.uint8)
+    s2 = np.zeros(M, np.float32)
+    _check(lib().orc_quant_nvfp4_segments(_p(X, _u16p), M, K, K, _p(seg, _i32p), len(seg) - 1, _p(codes, _u8p),
+                                          _p(scales, _u8p), _p(s2, _f32p)), "quant_nvfp4_segments")
+    return codes, scales, s2
+
+
 def quant_mxfp4(X):
     """Returns (codes [M, K/2] u8, scales [M, K/32] u8 (E8M0))."""
     X = _bf16(X)
@@ -202,14 +219,17 @@ def _gemm_out(M, N, want_ref):
 
 
 def gemm_nvfp4(ca, sa, s2a, a_mode, cw, sw, s2w, want_ref=True):
-    """Returns (Y bf16 bits [M,N], exact value [M,N], |alpha|*sum|a w| [M,N])."""
+    """Returns (Y bf16 bits [M,N], exact value [M,N], |alpha|*sum|a w| [M,N]).
+    s2w: one weight scale ([1]) or one per output row ([N])."""
     M, K = ca.shape[0], ca.shape[1] * 2
     N = cw.shape[0]
     Y, yref, absd = _gemm_out(M, N, want_ref)
     c = np.ascontiguousarray
-    _check(lib().orc_gemm_nvfp4(_p(c(ca), _u8p), _p(c(sa), _u8p), _p(c(s2a, np.float32), _f32p), a_mode,
-                                _p(c(cw), _u8p), _p(c(sw), _u8p), _p(c(s2w, np.float32), _f32p),
-                                M, N, K, _p(Y, _u16p), _p(yref, _f64p), _p(absd, _f64p)), "gemm_nvfp4")
+    s2w = c(s2w, np.float32)
+    w_mode = 1 if s2w.size == N and N > 1 else 0
+    _check(lib().orc_gemm_nvfp4_wrows(_p(c(ca), _u8p), _p(c(sa), _u8p), _p(c(s2a, np.float32), _f32p), a_mode,
+                                      _p(c(cw), _u8p), _p(c(sw), _u8p), _p(s2w, _f32p), w_mode,
+                                      M, N, K, _p(Y, _u16p), _p(yref, _f64p), _p(absd, _f64p)), "gemm_nvfp4")
     return Y, yref, absd
 
 

@@ -228,6 +228,25 @@ static void mxfp4_block(const float* x, uint8_t* codes16 /* 16 bytes */, uint8_t
     *scale = (uint8_t)c;
 }
 
+/* Fused modules ("Daily Papers", para 4): each row segment is quantized as
+ * its own NVFP4 tensor (the tensor rule over the segment's rows), and every
+ * row records its segment's second-level scale. */
+int orc_quant_nvfp4_segments(const uint16_t* X, int M, int K, int ldx,
+                             const int32_t* seg, int nseg, uint8_t* codes,
+                             uint8_t* scales, float* s2_rows) {
+    if (nseg < 1 || seg[0] != 0 || seg[nseg] != M || K % 16) return -1;
+    for (int i = 0; i < nseg; ++i) {
+        const int r0 = seg[i], r1 = seg[i + 1];
+        if (r1 < r0) return -1;
+        float s2 = 1.0f;
+        if (orc_quant_nvfp4(X + (size_t)r0 * ldx, r1 - r0, K, ldx, 0, NULL, codes + (size_t)r0 * (K / 2),
+                            scales + (size_t)r0 * (K / 16), &s2))
+            return -1;
+        for (int r = r0; r < r1; ++r) s2_rows[r] = s2;
+    }
+    return 0;
+}
+
 int orc_quant_mxfp4(const uint16_t* X, int M, int K, int ldx, uint8_t* codes, uint8_t* scales) {
     if (M < 0 || K % 32 || ldx < K) return -1;
     float x[32];
@@ -319,12 +338,18 @@ static int e2m1_x2(uint8_t c) {
 int orc_gemm_nvfp4(const uint8_t* ca, const uint8_t* sa, const float* s2a, int a_mode,
                    const uint8_t* cw, const uint8_t* sw, const float* s2w,
                    int M, int N, int K, uint16_t* Y, double* yref, double* absdot) {
+    return orc_gemm_nvfp4_wrows(ca, sa, s2a, a_mode, cw, sw, s2w, 0, M, N, K, Y, yref, absdot);
+}
+
+int orc_gemm_nvfp4_wrows(const uint8_t* ca, const uint8_t* sa, const float* s2a, int a_mode,
+                         const uint8_t* cw, const uint8_t* sw, const float* s2w, int w_mode,
+                         int M, int N, int K, uint16_t* Y, double* yref, double* absdot) {
     if (K % 16) return -1;
     const int KB = K / 16;
     for (int m = 0; m < M; ++m) {
         double s2m = (double)(a_mode == 1 ? s2a[m] : s2a[0]);
-        double alpha = s2m * (double)s2w[0];
         for (int n = 0; n < N; ++n) {
+            double alpha = s2m * (double)(w_mode == 1 ? s2w[n] : s2w[0]);
             __int128 acc = 0, aacc = 0;
             for (int b = 0; b < KB; ++b) {
                 long long p = 0, ap = 0;

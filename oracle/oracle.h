@@ -58,6 +58,14 @@ float orc_nvfp4_s2_from_amax(float amax);
 int orc_quant_nvfp4(const uint16_t* X, int M, int K, int ldx, int mode,
                     const float* static_s2, uint8_t* codes, uint8_t* scales,
                     float* s2);
+/* Fused modules ("Daily Papers", para 4 (Minima): a global-scale mismatch
+ * when modules quantized with their own global scales are fused into one
+ * GEMM): rows [seg[i], seg[i+1]) form module i, quantized as its own tensor
+ * (one FP32 scale from the module's amax); s2_rows[M] receives every row's
+ * module scale.  seg: nseg+1 ascending boundaries, seg[0] = 0, seg[nseg] = M. */
+int orc_quant_nvfp4_segments(const uint16_t* X, int M, int K, int ldx,
+                             const int32_t* seg, int nseg, uint8_t* codes,
+                             uint8_t* scales, float* s2_rows);
 /* codes [M][K/2], scales [M][K/32] E8M0 bytes                             */
 int orc_quant_mxfp4(const uint16_t* X, int M, int K, int ldx,
                     uint8_t* codes, uint8_t* scales);
@@ -79,6 +87,11 @@ void orc_dequant_int4(const uint8_t* codes, const float* scales,
 int orc_gemm_nvfp4(const uint8_t* ca, const uint8_t* sa, const float* s2a, int a_mode,
                    const uint8_t* cw, const uint8_t* sw, const float* s2w,
                    int M, int N, int K, uint16_t* Y, double* yref, double* absdot);
+/* The same with the weights' second-level scale per output row (w_mode 1:
+ * s2w[N], alpha = s2a * s2w[n]) or per tensor (w_mode 0).                  */
+int orc_gemm_nvfp4_wrows(const uint8_t* ca, const uint8_t* sa, const float* s2a, int a_mode,
+                         const uint8_t* cw, const uint8_t* sw, const float* s2w, int w_mode,
+                         int M, int N, int K, uint16_t* Y, double* yref, double* absdot);
 int orc_gemm_mxfp4(const uint8_t* ca, const uint8_t* sa,
                    const uint8_t* cw, const uint8_t* sw,
                    int M, int N, int K, uint16_t* Y, double* yref, double* absdot);

@@ -370,3 +370,49 @@ def test_select_channels_vs_sort(orc):
         np.testing.assert_array_equal(S, np.sort(order[:nS]))
     S = orc.select_channels(Xb, 1)
     assert list(S) == [10]
+
+
+# ---- fused modules: per-segment weight scales ------------------------------------
+def test_segments_single_segment_is_the_tensor_rule(orc):
+    X = bf16(synth.normal((40, 64), 0.02, 40, 1))
+    c, s, s2 = orc.quant_nvfp4_segments(X, [0, 40])
+    c0, s0, t0 = orc.quant_nvfp4(X, mode=0)
+    np.testing.assert_array_equal(c, c0)
+    np.testing.assert_array_equal(s, s0)
+    assert np.all(s2 == t0[0])
+
+
+def test_segments_are_separate_tensors(orc):
+    # rows of very different magnitude, as in fused q/k/v modules
+    X = bf16(synth.normal((48, 64), 1.0, 41, 1) * np.repeat([1.0, 3000.0, 0.001], 16)[:, None])
+    seg = [0, 16, 32, 48]
+    c, s, s2 = orc.quant_nvfp4_segments(X, seg)
+    for i in range(3):
+        r0, r1 = seg[i], seg[i + 1]
+        ci, si, ti = orc.quant_nvfp4(X[r0:r1], mode=0)
+        np.testing.assert_array_equal(c[r0:r1], ci)
+        np.testing.assert_array_equal(s[r0:r1], si)
+        assert np.all(s2[r0:r1] == ti[0])
+    # one scale for the whole fused tensor puts the small module's block scales below
+    # E4M3's smallest subnormal: every code of it is 0, while its own scale keeps it
+    ct, _, _ = orc.quant_nvfp4(X, mode=0)
+    assert (unpack(ct[32:]) & 7 == 0).mean() == 1.0
+    assert (unpack(c[32:]) & 7 == 0).mean() < 0.2
+
+
+def test_gemm_per_row_weight_scale(orc):
+    M, N, K = 9, 48, 128
+    A = bf16(synth.normal((M, K), 1.0, 42, 1))
+    W = bf16(synth.normal((N, K), 0.02, 42, 2) * np.repeat([1.0, 50.0, 0.02], 16)[:, None])
+    ca, sa, s2a = orc.quant_nvfp4(A, mode=1)
+    cw, sw, s2w = orc.quant_nvfp4_segments(W, [0, 16, 32, 48])
+    Y, yref, absd = orc.gemm_nvfp4(ca, sa, s2a, 1, cw, sw, s2w)
+    # brute force on the dequantized operands (library conversions, fp64)
+    naive = _nvfp4_lib_dequant(ca, sa, s2a, 1) @ _nvfp4_lib_dequant(cw, sw, s2w, 1).T
+    assert np.all(np.abs(yref - naive) <= 1e-12 * np.abs(naive) + 1e-300)
+    # all rows sharing one scale reduces to the per-tensor form
+    cw0, sw0, t0 = orc.quant_nvfp4(W, mode=0)
+    Y1, y1, _ = orc.gemm_nvfp4(ca, sa, s2a, 1, cw0, sw0, np.full(N, t0[0], np.float32))
+    Y0, y0, _ = orc.gemm_nvfp4(ca, sa, s2a, 1, cw0, sw0, t0)
+    np.testing.assert_array_equal(Y1, Y0)
+    np.testing.assert_array_equal(y1, y0)

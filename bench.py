@@ -462,6 +462,36 @@ def extra_rows(args, dev, stream, P):
     if tot_ms > 0:
         out["aug_nvfp4_qwen25_3b_m8192"] = {"TFLOPS_exec": round(tot_f / (tot_ms * 1e-3) / 1e12, 1),
                                             "TFLOPS_effective_K": round(tot_fk / (tot_ms * 1e-3) / 1e12, 1)}
+    # fused qkv with one weight scale per module (q | k | v segments): the
+    # linear at M = 4096 and the M = 1 decode, beside the one-scale weights
+    if want("segments"):
+        K = 8192
+        rows, gains = synth.FUSED["llama2_70b"]["qkv"]
+        Wb, seg = synth.fused_weights(rows, gains, K, seed=0, tensor_id=100)
+        Wd = to_dev(Wb, dev)
+        del Wb
+        N = seg[-1]
+        variants = {"segments": w4.quantize_weight_segments(Wd, seg), "one_scale": w4.quantize_weight(Wd, w4.NVFP4)}
+        del Wd
+        fl = l2_flush_buffer(dev)  # the M = 1 weights (47 MB) would stay in L2
+        for Ms in (args.tokens, 1):
+            X = to_dev(synth.activations("llama2_70b", Ms, K, seed=9), dev)
+            Y = torch.empty(Ms, N, dtype=torch.bfloat16, device=dev)
+            ws = torch.empty(w4.linear_workspace(Ms, N, K, w4.NVFP4), dtype=torch.uint8, device=dev)
+            for vname, Wq in variants.items():
+                f = lambda: w4.linear(X, Wq, w4.SCALE_TOKEN, Y=Y, ws=ws)
+                for _ in range(max(3, args.warmup)):
+                    f()
+                ms = time_loop(f, it, stream, None if Ms > 16 else fl)
+                if Ms > 16:
+                    out[f"qkv_{vname}_m{Ms}"] = {"TFLOPS": round(2.0 * Ms * N * K / (ms * 1e-3) / 1e12, 1),
+                                                 "us": round(ms * 1e3, 2)}
+                else:
+                    byts = N * K * 0.5625 + 2 * Ms * K + 2 * Ms * N + (4 * N if vname == "segments" else 0)
+                    out[f"qkv_{vname}_m{Ms}"] = {"GB/s": round(byts / ms / 1e6, 1), "us": round(ms * 1e3, 2)}
+            del X, Y, ws
+        del variants, fl
+
     if not want("mxfp4"):
         torch.cuda.synchronize()
         assert w4.device_status() == w4.OK
@@ -494,7 +524,7 @@ def main():
     ap.add_argument("--cpu-rows", type=int, default=8, help="cpu_baseline sample: tokens")
     ap.add_argument("--cpu-cols", type=int, default=4096, help="cpu_baseline sample: output columns")
     ap.add_argument("--no-rows", action="store_true", help="skip the secondary rows")
-    ap.add_argument("--only", choices=["gemm", "quant", "decode", "int4", "aug", "mxfp4"], default=None,
+    ap.add_argument("--only", choices=["gemm", "quant", "decode", "int4", "aug", "mxfp4", "segments"], default=None,
                     help="run only one secondary row (for profiling) and print it")
     ap.add_argument("--no-cpu", action="store_true", help="skip the oracle CPU baseline")
     ap.add_argument("--shape", default=None, help="--only gemm: one Llama linear (qkv, o, w1, w3, w2)")

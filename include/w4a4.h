@@ -132,8 +132,9 @@ int w4a4_quantize_act(const uint16_t* X, int M, int K, int ldx,
 
 /*
  * Quantize weights W[N,K] (bf16, row stride ldw) once, offline.  Same block
- * rules as w4a4_quantize_act; NVFP4 weights always use one tensor scale
- * (out->scale_mode must be TENSOR).  With S (device int32[nS], strictly
+ * rules as w4a4_quantize_act; NVFP4 weights here use one tensor scale
+ * (out->scale_mode must be TENSOR; w4a4_quantize_weight_segments gives one
+ * scale per row segment).  With S (device int32[nS], strictly
  * ascending channel indices in [0,K), nS a multiple of 128) the quantized
  * tensor is [W | W[:,S]] with cols = K + nS: the weight side of the
  * dual-stage residual augmentation ("APEX4..." page, para 2, ARCQuant).
@@ -143,10 +144,36 @@ int w4a4_quantize_weight(const uint16_t* W, int N, int K, int ldw,
                          w4a4_qtensor* out, void* stream);
 
 /*
+ * NVFP4 weights of a fused module (q/k/v, gate/up stacked along N) with one
+ * global scale per constituent module ("Daily Papers" page, para 4, Minima:
+ * one NVFP4 global scale per module, calibrated separately).  Row segment i
+ * is rows [seg[i], seg[i+1]) of W[N,K]; it is quantized exactly as
+ * w4a4_quantize_weight quantizes that slice alone (tensor scale
+ * s2_i = amax(segment)/2688), and every row of it stores s2_i.
+ *   seg: HOST int32[nseg+1], seg[0] = 0 < seg[1] < ... < seg[nseg] = N, every
+ *     boundary a multiple of 128 (so each segment owns whole scale atoms);
+ *     nseg >= 1.  nseg = 1 gives the tensor rule with the scale repeated.
+ *   S, nS: as w4a4_quantize_weight (cols = K + nS; the appended channels use
+ *     their segment's scale).
+ *   out: format NVFP4, scale_mode W4A4_SCALE_TOKEN (s2 holds one scale per
+ *     row, N floats, 16-byte aligned), rows = N, cols = K + nS.
+ * The GEMM and the linear layer read s2[n] for output column n; with the
+ * same rows in one segment the result equals a tensor-scale weight's.
+ * Returns W4A4_ERR_INVALID_ARG on a bad segment list, W4A4_ERR_MISALIGNED on
+ * an unaligned s2; nothing is launched then.
+ */
+int w4a4_quantize_weight_segments(const uint16_t* W, int N, int K, int ldw,
+                                  const int32_t* seg, int nseg,
+                                  const int32_t* S, int nS,
+                                  w4a4_qtensor* out, void* stream);
+
+/*
  * Y[M,N] = A * B^T for quantized A (activations, rows = M) and B (weights,
  * rows = N) of the same format and the same cols (= K, or K + nS).
  *   NVFP4/MXFP4: block-scaled tensor-core MMA, FP32 accumulation;
- *     NVFP4 result multiplied by alpha = s2_A(row or tensor) * s2_B.
+ *     NVFP4 result of (m, n) multiplied by alpha = s2_A (row m, or the
+ *     tensor's) * s2_B (the tensor's, or row n's when B->scale_mode is
+ *     TOKEN, e.g. per-segment weights; B->s2 must then be 16-byte aligned).
  *   INT4: exact int32 partial sum per 128-group, rescaled by
  *     scale_A[m,g]*scale_B[n,g] and accumulated in FP32 ("Depth
  *     Registers..." thelatestinai page, para 2: group dequantization).

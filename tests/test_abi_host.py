@@ -88,9 +88,9 @@ def test_argument_errors_before_any_device_work(L):
     assert L.w4a4_gemm(C.byref(a), C.byref(b), C.c_void_p(16), 256, None) == w4.ERR_INVALID_ARG
     b = _qt(w4.NVFP4, 200, 256, w4.SCALE_TENSOR)
     assert L.w4a4_gemm(C.byref(a), C.byref(b), C.c_void_p(16), 256, None) == w4.ERR_INVALID_ARG
-    # NVFP4 weights must carry a tensor scale
-    b = _qt(w4.NVFP4, 256, 256, w4.SCALE_TOKEN)
-    assert L.w4a4_gemm(C.byref(a), C.byref(b), C.c_void_p(16), 256, None) == w4.ERR_INVALID_ARG
+    # NVFP4 weights with one scale per row need those scales 16-byte aligned
+    b = _qt(w4.NVFP4, 256, 256, w4.SCALE_TOKEN, s2=20)
+    assert L.w4a4_gemm(C.byref(a), C.byref(b), C.c_void_p(16), 256, None) == w4.ERR_MISALIGNED
     # linear: workspace too small, residual channels with a non-NVFP4 weight
     W = _qt(w4.NVFP4, 256, 256, w4.SCALE_TENSOR)
     assert L.w4a4_linear(C.c_void_p(16), 4, 256, 256, C.byref(W), 1, None, 0, C.c_void_p(16), 256,
@@ -120,3 +120,28 @@ def test_no_device_means_error_not_fallback(L):
     q = _qt(w4.NVFP4, 4, 256, w4.SCALE_TOKEN)
     rc = L.w4a4_quantize_act(C.c_void_p(16), 4, 256, 256, 0, 16, 1, None, C.byref(q), None)
     assert rc in (w4.ERR_CUDA, w4.ERR_ARCH)
+
+
+def test_segment_weight_arguments(L):
+    """Per-segment weight scales: the segment list, the output's scale mode and
+    the alignment of its per-row scales are checked on the host."""
+    def seg_call(seg, out, N=512, K=256, S=None, nS=0):
+        arr = (C.c_int32 * len(seg))(*seg)
+        return L.w4a4_quantize_weight_segments(C.c_void_p(16), N, K, K, arr, len(seg) - 1, S, nS,
+                                               C.byref(out), None)
+    out = _qt(w4.NVFP4, 512, 256, w4.SCALE_TOKEN)
+    for bad in ([0, 256, 256, 512],   # empty segment
+                [0, 200, 512],        # boundary not a multiple of 128
+                [0, 256, 384],        # does not end at N
+                [128, 512],           # does not start at 0
+                [0],                  # no segment
+                [0, 384, 256, 512]):  # not ascending
+        assert seg_call(bad, out) == w4.ERR_INVALID_ARG, bad
+    # the output must be NVFP4 with one s2 per row
+    assert seg_call([0, 512], _qt(w4.NVFP4, 512, 256, w4.SCALE_TENSOR)) == w4.ERR_INVALID_ARG
+    assert seg_call([0, 512], _qt(w4.MXFP4, 512, 256)) == w4.ERR_INVALID_ARG
+    assert seg_call([0, 512], _qt(w4.NVFP4, 512, 256, w4.SCALE_TOKEN, s2=20)) == w4.ERR_MISALIGNED
+    # residual channels: cols must be K + nS, nS a multiple of 128
+    assert seg_call([0, 512], out, S=C.c_void_p(16), nS=128) == w4.ERR_INVALID_ARG
+    aug = _qt(w4.NVFP4, 512, 384, w4.SCALE_TOKEN)
+    assert seg_call([0, 512], aug, S=C.c_void_p(16), nS=64) == w4.ERR_INVALID_ARG

@@ -25,7 +25,8 @@ OK, ERR_INVALID_ARG, ERR_MISALIGNED, ERR_WORKSPACE, ERR_ARCH, ERR_CUDA, ERR_DEVI
 # every entry point declared in include/w4a4.h
 EXPORTS = ("w4a4_qtensor_bytes", "w4a4_quantize_act", "w4a4_quantize_weight", "w4a4_gemm",
            "w4a4_linear_workspace", "w4a4_linear", "w4a4_augment_residual", "w4a4_select_channels",
-           "w4a4_device_status", "w4a4_debug_set", "w4a4_status_string", "w4a4_linear_noalloc")
+           "w4a4_device_status", "w4a4_debug_set", "w4a4_status_string", "w4a4_linear_noalloc",
+           "w4a4_quantize_weight_segments")
 
 
 class W4A4Error(RuntimeError):
@@ -56,6 +57,7 @@ def lib():
         L.w4a4_qtensor_bytes.argtypes = [i, i, i, i, C.POINTER(sz), C.POINTER(sz), C.POINTER(sz)]
         L.w4a4_quantize_act.argtypes = [vp, i, i, i, i, i, i, vp, qp, vp]
         L.w4a4_quantize_weight.argtypes = [vp, i, i, i, i, i, vp, i, qp, vp]
+        L.w4a4_quantize_weight_segments.argtypes = [vp, i, i, i, C.POINTER(C.c_int32), i, vp, i, qp, vp]
         L.w4a4_gemm.argtypes = [qp, qp, vp, i, vp]
         L.w4a4_linear_workspace.argtypes = [i, i, i, i, i]
         L.w4a4_linear_workspace.restype = sz
@@ -70,7 +72,7 @@ def lib():
         L.w4a4_status_string.restype = C.c_char_p
         for name in ("w4a4_qtensor_bytes", "w4a4_quantize_act", "w4a4_quantize_weight", "w4a4_gemm",
                      "w4a4_linear", "w4a4_augment_residual", "w4a4_select_channels", "w4a4_device_status",
-                     "w4a4_linear_noalloc"):
+                     "w4a4_linear_noalloc", "w4a4_quantize_weight_segments"):
             getattr(L, name).restype = i
         _lib = L
     return _lib
@@ -139,6 +141,24 @@ def quantize_weight(W, fmt: int, S=None, out: QTensor | None = None) -> QTensor:
         out = QTensor(fmt, N, K + nS, SCALE_TENSOR, W.device)
     _check(lib().w4a4_quantize_weight(_ptr(W), N, K, W.stride(0), fmt, GROUP[fmt], _ptr(S), nS, out.ref,
                                       _stream()), "w4a4_quantize_weight")
+    return out
+
+
+def quantize_weight_segments(W, seg, S=None, out: QTensor | None = None) -> QTensor:
+    """NVFP4 weights of a fused module, one global scale per row segment.
+
+    W: bf16 [N, K]; seg: host sequence of N-row boundaries [0, ..., N], each a
+    multiple of 128 (e.g. [0, q_rows, q_rows + k_rows, N] for fused q/k/v);
+    S: optional int32 CUDA tensor of augmented channels.  The result stores
+    one s2 per row (scale_mode TOKEN)."""
+    N, K = W.shape
+    nS = 0 if S is None else S.numel()
+    seg = [int(v) for v in seg]
+    if out is None:
+        out = QTensor(NVFP4, N, K + nS, SCALE_TOKEN, W.device)
+    arr = (C.c_int32 * len(seg))(*seg)
+    _check(lib().w4a4_quantize_weight_segments(_ptr(W), N, K, W.stride(0), arr, len(seg) - 1, _ptr(S), nS,
+                                               out.ref, _stream()), "w4a4_quantize_weight_segments")
     return out
 
 

@@ -159,6 +159,13 @@ int quantize_rows(const uint16_t* X, int M, int K, int ldx, const int32_t* S, in
     return cuda_status(launch_quant(q->format, S != nullptr, a, pad128(M), num_sms, st));
 }
 
+// NVFP4 weights with one s2 per row (per-segment scales): the GEMM epilogues
+// read four consecutive row scales at a time.
+int check_weight_s2(const w4a4_qtensor* B) {
+    if (B->format == W4A4_NVFP4 && B->scale_mode == W4A4_SCALE_TOKEN && !aligned16(B->s2)) return W4A4_ERR_MISALIGNED;
+    return W4A4_OK;
+}
+
 int check_S_args(const int32_t* S, int nS, int K) {
     if (nS < 0 || (nS > 0 && (!S || nS % 128 || nS > K))) return W4A4_ERR_INVALID_ARG;
     if (nS == 0 && S) return W4A4_ERR_INVALID_ARG;
@@ -189,6 +196,7 @@ int setup_gemm(const w4a4_qtensor* A, const w4a4_qtensor* B, uint16_t* Y, int ld
     g.s2a = A->s2;
     g.s2a_per_row = A->scale_mode == W4A4_SCALE_TOKEN ? 1 : 0;
     g.s2b = B->s2;
+    g.s2b_per_row = B->format == W4A4_NVFP4 && B->scale_mode == W4A4_SCALE_TOKEN ? 1 : 0;
     g.Y = Y;
     g.ldy = ldy;
     g.skip_k_tile = g_skip_k_tile;
@@ -343,13 +351,52 @@ int w4a4_quantize_weight(const uint16_t* W, int N, int K, int ldw, int format, i
     return quantize_rows(W, N, K + nS, ldw, nS ? S : nullptr, K, nullptr, out, sms, as_stream(stream));
 }
 
+int w4a4_quantize_weight_segments(const uint16_t* W, int N, int K, int ldw, const int32_t* seg, int nseg,
+                                  const int32_t* S, int nS, w4a4_qtensor* out, void* stream) {
+    if (N < 0 || K < 128 || K % 128 || K > kMaxK || ldw < K) return W4A4_ERR_INVALID_ARG;
+    if (!seg || nseg < 1 || seg[0] != 0 || seg[nseg] != N) return W4A4_ERR_INVALID_ARG;
+    for (int i = 0; i < nseg; ++i)
+        if (seg[i + 1] <= seg[i] || seg[i + 1] % 128) return W4A4_ERR_INVALID_ARG;
+    int rc = check_S_args(S, nS, K);
+    if (rc != W4A4_OK) return rc;
+    rc = check_qtensor(out);
+    if (rc != W4A4_OK) return rc;
+    if (out->format != W4A4_NVFP4 || out->scale_mode != W4A4_SCALE_TOKEN || out->rows != N || out->cols != K + nS)
+        return W4A4_ERR_INVALID_ARG;
+    rc = check_weight_s2(out);
+    if (rc != W4A4_OK) return rc;
+    if (!W) return W4A4_ERR_INVALID_ARG;
+    if (!aligned16(W) || ldw % 8) return W4A4_ERR_MISALIGNED;
+    int sms = 0;
+    rc = device_check(&sms);
+    if (rc != W4A4_OK) return rc;
+    cudaStream_t st = as_stream(stream);
+    const int cols = K + nS;
+    for (int i = 0; i < nseg; ++i) {
+        // the segment as a tensor of its own: rows r0..r1 of codes, its 128-row
+        // scale atoms, and s2[r0] as its tensor scale (s2[r0 + 1] holds its amax)
+        const int r0 = seg[i], rows = seg[i + 1] - seg[i];
+        w4a4_qtensor q = *out;
+        q.rows = rows;
+        q.scale_mode = W4A4_SCALE_TENSOR;
+        q.codes = static_cast<uint8_t*>(out->codes) + (size_t)r0 * (cols / 2);
+        q.scales = static_cast<uint8_t*>(out->scales) + (size_t)(r0 / 128) * (cols / 16 / 4) * 512;
+        q.s2 = out->s2 + r0;
+        rc = quantize_rows(W + (size_t)r0 * ldw, rows, cols, ldw, nS ? S : nullptr, K, nullptr, &q, sms, st);
+        if (rc != W4A4_OK) return rc;
+        if (launch_spread_first(q.s2, rows, st) != cudaSuccess) return W4A4_ERR_CUDA;
+    }
+    return W4A4_OK;
+}
+
 int w4a4_gemm(const w4a4_qtensor* A, const w4a4_qtensor* B, uint16_t* Y, int ldy, void* stream) {
     int rc = check_qtensor(A);
     if (rc == W4A4_OK) rc = check_qtensor(B);
     if (rc != W4A4_OK) return rc;
     if (A->format != B->format || A->cols != B->cols || B->rows < 128 || B->rows % 128 || ldy < B->rows)
         return W4A4_ERR_INVALID_ARG;
-    if (A->format == W4A4_NVFP4 && B->scale_mode != W4A4_SCALE_TENSOR) return W4A4_ERR_INVALID_ARG;
+    rc = check_weight_s2(B);
+    if (rc != W4A4_OK) return rc;
     if (A->rows == 0) return W4A4_OK;
     if (!Y) return W4A4_ERR_INVALID_ARG;
     if (!aligned16(Y) || ldy % 8) return W4A4_ERR_MISALIGNED;
@@ -375,9 +422,10 @@ int w4a4_linear(const uint16_t* X, int M, int K, int ldx, const w4a4_qtensor* Wq
     if (rc != W4A4_OK) return rc;
     if (nS && fmt != W4A4_NVFP4) return W4A4_ERR_INVALID_ARG;
     if (Wq->cols != K + nS || Wq->rows < 128 || Wq->rows % 128 || ldy < Wq->rows) return W4A4_ERR_INVALID_ARG;
-    if (fmt == W4A4_NVFP4 && (Wq->scale_mode != W4A4_SCALE_TENSOR ||
-                              (scale_mode != W4A4_SCALE_TENSOR && scale_mode != W4A4_SCALE_TOKEN)))
+    if (fmt == W4A4_NVFP4 && scale_mode != W4A4_SCALE_TENSOR && scale_mode != W4A4_SCALE_TOKEN)
         return W4A4_ERR_INVALID_ARG;
+    rc = check_weight_s2(Wq);
+    if (rc != W4A4_OK) return rc;
     if (M == 0) return W4A4_OK;
     if (!X || !Y) return W4A4_ERR_INVALID_ARG;
     if (!aligned16(X) || ldx % 8 || !aligned16(Y) || ldy % 8) return W4A4_ERR_MISALIGNED;

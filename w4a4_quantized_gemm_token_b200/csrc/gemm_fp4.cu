@@ -346,10 +346,19 @@ __global__ void __launch_bounds__(Dec<KB>::THREADS, 1)
                         acc.z += w.z;
                         acc.w += w.w;
                     }
-                    const float alpha = NV ? __fmul_rn(g.s2a[g.s2a_per_row ? t : 0], g.s2b[0]) : 1.0f;
                     const int n = nt * kBM + r4;
-                    __nv_bfloat162 h0 = __floats2bfloat162_rn(__fmul_rn(acc.x, alpha), __fmul_rn(acc.y, alpha));
-                    __nv_bfloat162 h1 = __floats2bfloat162_rn(__fmul_rn(acc.z, alpha), __fmul_rn(acc.w, alpha));
+                    // alpha per output column: s2 of token t times s2 of weight row n
+                    // (one weight scale, or one per row for per-segment weights)
+                    float4 al = make_float4(1.0f, 1.0f, 1.0f, 1.0f);
+                    if (NV) {
+                        const float sa = g.s2a[g.s2a_per_row ? t : 0];
+                        const float4 sb = g.s2b_per_row ? *reinterpret_cast<const float4*>(g.s2b + min(n, g.N - 4))
+                                                        : make_float4(g.s2b[0], g.s2b[0], g.s2b[0], g.s2b[0]);
+                        al = make_float4(__fmul_rn(sa, sb.x), __fmul_rn(sa, sb.y), __fmul_rn(sa, sb.z),
+                                         __fmul_rn(sa, sb.w));
+                    }
+                    __nv_bfloat162 h0 = __floats2bfloat162_rn(__fmul_rn(acc.x, al.x), __fmul_rn(acc.y, al.y));
+                    __nv_bfloat162 h1 = __floats2bfloat162_rn(__fmul_rn(acc.z, al.z), __fmul_rn(acc.w, al.w));
                     if (n < g.N)
                         *reinterpret_cast<uint2*>(g.Y + (size_t)t * g.ldy + n) =
                             make_uint2(*reinterpret_cast<uint32_t*>(&h0), *reinterpret_cast<uint32_t*>(&h1));

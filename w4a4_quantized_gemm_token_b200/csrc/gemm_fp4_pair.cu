@@ -73,7 +73,9 @@ struct Cfg {
 };
 }  // namespace pp
 
-template <bool NV>
+// PB: B (the weights) carries one second-level scale per row (per output
+// column of Y), as NVFP4 weights of fused modules quantized per segment do.
+template <bool NV, bool PB>
 __global__ void __launch_bounds__(pp::THREADS, 1)
     gemm_fp4_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                          const __grid_constant__ CUtensorMap tmSA, const __grid_constant__ CUtensorMap tmSB,
@@ -279,11 +281,22 @@ __global__ void __launch_bounds__(pp::THREADS, 1)
         for (int t = pair; t < ntiles; t += npairs, ++ti) {
             int at, bt;
             coords(t, at, bt);
+            // per-row B scales of these 128 columns, lane l holding column
+            // 32 * ch + l, fetched before the accumulator is ready (N is a
+            // multiple of 128: a half tile is wholly inside N or wholly past it)
+            float sbl[4];
+            if constexpr (PB) {
+#pragma unroll
+                for (int ch = 0; ch < 4; ++ch) sbl[ch] = g.s2b[min(bt * BN + half * 128, g.N - 128) + 32 * ch + lane];
+            }
             if (!mbar_wait(accf, ti & 1, limit, abort_flag, 100000)) break;
             tc_fence_after();
             const int m = at * BM + (int)rank * HALF + q * 32 + lane;
-            float alpha = 1.0f;
-            if (NV && m < g.M) alpha = __fmul_rn(g.s2a[g.s2a_per_row ? m : 0], g.s2b[0]);
+            float alpha = 1.0f, sa = 0.0f;
+            if (NV && m < g.M) {
+                sa = g.s2a[g.s2a_per_row ? m : 0];
+                alpha = __fmul_rn(sa, g.s2b[0]);
+            }
             uint32_t pk[64];
 #pragma unroll
             for (int ch = 0; ch < 4; ++ch) {
@@ -292,8 +305,13 @@ __global__ void __launch_bounds__(pp::THREADS, 1)
                 tmem_ld_wait();
 #pragma unroll
                 for (int e = 0; e < 16; ++e) {
-                    __nv_bfloat162 h = __floats2bfloat162_rn(__fmul_rn(__uint_as_float(r[2 * e]), alpha),
-                                                             __fmul_rn(__uint_as_float(r[2 * e + 1]), alpha));
+                    float a0 = alpha, a1 = alpha;
+                    if constexpr (PB) {
+                        a0 = __fmul_rn(sa, __shfl_sync(0xffffffffu, sbl[ch], 2 * e));
+                        a1 = __fmul_rn(sa, __shfl_sync(0xffffffffu, sbl[ch], 2 * e + 1));
+                    }
+                    __nv_bfloat162 h = __floats2bfloat162_rn(__fmul_rn(__uint_as_float(r[2 * e]), a0),
+                                                             __fmul_rn(__uint_as_float(r[2 * e + 1]), a1));
                     pk[16 * ch + e] = *reinterpret_cast<uint32_t*>(&h);
                 }
             }
@@ -321,18 +339,21 @@ __global__ void __launch_bounds__(pp::THREADS, 1)
 
 cudaError_t launch_gemm_fp4_pair(bool nvfp4, const CUtensorMap& tmA, const CUtensorMap& tmB, const CUtensorMap& tmSA,
                                  const CUtensorMap& tmSB, const GemmArgs& g, int num_sms, bool pdl, cudaStream_t st) {
-    auto kern = nvfp4 ? gemm_fp4_pair_kernel<true> : gemm_fp4_pair_kernel<false>;
-    static bool attr_set[2] = {false, false};
-    if (!attr_set[nvfp4]) {
+    // variants: MXFP4, NVFP4 with one B scale, NVFP4 with per-row B scales
+    const int v = !nvfp4 ? 0 : g.s2b_per_row ? 2 : 1;
+    auto kern = v == 0 ? gemm_fp4_pair_kernel<false, false>
+                       : v == 1 ? gemm_fp4_pair_kernel<true, false> : gemm_fp4_pair_kernel<true, true>;
+    static bool attr_set[3] = {false, false, false};
+    if (!attr_set[v]) {
         cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                              nvfp4 ? pp::Cfg<true>::SMEM : pp::Cfg<false>::SMEM);
         if (e != cudaSuccess) return e;
-        attr_set[nvfp4] = true;
+        attr_set[v] = true;
     }
     const int tiles = ((g.M + pp::BM - 1) / pp::BM) * ((g.N + pp::BN - 1) / pp::BN);
     // as many pairs as can be resident at once (a persistent grid must not queue)
-    static int resident[2] = {0, 0};
-    if (!resident[nvfp4]) {
+    static int resident[3] = {0, 0, 0};
+    if (!resident[v]) {
         cudaLaunchConfig_t q = {};
         q.gridDim = dim3(2 * (num_sms / 2));
         q.blockDim = dim3(pp::THREADS);
@@ -349,10 +370,10 @@ cudaError_t launch_gemm_fp4_pair(bool nvfp4, const CUtensorMap& tmA, const CUten
             cudaGetLastError();
             n = num_sms / 2;
         }
-        resident[nvfp4] = n;
+        resident[v] = n;
     }
     int pairs = tiles < num_sms / 2 ? tiles : num_sms / 2;
-    if (pairs > resident[nvfp4]) pairs = resident[nvfp4];
+    if (pairs > resident[v]) pairs = resident[v];
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(2 * pairs);
     cfg.blockDim = dim3(pp::THREADS);

@@ -55,7 +55,9 @@ static_assert(SF_COL0 + STAGES * SF_COLS <= TMEM_COLS, "tensor memory holds 512 
 static_assert(SMEM <= 232448, "shared memory per block");
 }  // namespace pf
 
-template <bool NV>
+// PB: B (the weights) carries one second-level scale per row (per output
+// column of Y), as NVFP4 weights of fused modules quantized per segment do.
+template <bool NV, bool PB>
 __global__ void __launch_bounds__(pf::THREADS, 1)
     gemm_fp4_persistent_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                                GemmArgs g) {
@@ -223,11 +225,22 @@ __global__ void __launch_bounds__(pf::THREADS, 1)
         for (int t = blockIdx.x; t < ntiles; t += gridDim.x, ++ti) {
             int at, bt;
             coords(t, at, bt);
+            // per-row B scales of the tile's columns, lane l holding column
+            // 32 * ch + l, fetched before the accumulator is ready (clamped
+            // inside N past its end, which is a multiple of 128)
+            float sbl[8];
+            if constexpr (PB) {
+#pragma unroll
+                for (int ch = 0; ch < 8; ++ch) sbl[ch] = g.s2b[min(bt * BN + 32 * ch, g.N - 32) + lane];
+            }
             if (!mbar_wait(accf, ti & 1, limit, abort_flag, 100000)) break;
             tc_fence_after();
             const int m = at * kBM + q * 32 + lane;
-            float alpha = 1.0f;
-            if (NV && m < g.M) alpha = __fmul_rn(g.s2a[g.s2a_per_row ? m : 0], g.s2b[0]);
+            float alpha = 1.0f, sa = 0.0f;
+            if (NV && m < g.M) {
+                sa = g.s2a[g.s2a_per_row ? m : 0];
+                alpha = __fmul_rn(sa, g.s2b[0]);
+            }
             uint32_t pk[128];
 #pragma unroll
             for (int ch = 0; ch < 8; ++ch) {
@@ -236,8 +249,13 @@ __global__ void __launch_bounds__(pf::THREADS, 1)
                 tmem_ld_wait();
 #pragma unroll
                 for (int e = 0; e < 16; ++e) {
-                    __nv_bfloat162 h = __floats2bfloat162_rn(__fmul_rn(__uint_as_float(r[2 * e]), alpha),
-                                                             __fmul_rn(__uint_as_float(r[2 * e + 1]), alpha));
+                    float a0 = alpha, a1 = alpha;
+                    if constexpr (PB) {
+                        a0 = __fmul_rn(sa, __shfl_sync(0xffffffffu, sbl[ch], 2 * e));
+                        a1 = __fmul_rn(sa, __shfl_sync(0xffffffffu, sbl[ch], 2 * e + 1));
+                    }
+                    __nv_bfloat162 h = __floats2bfloat162_rn(__fmul_rn(__uint_as_float(r[2 * e]), a0),
+                                                             __fmul_rn(__uint_as_float(r[2 * e + 1]), a1));
                     pk[16 * ch + e] = *reinterpret_cast<uint32_t*>(&h);
                 }
             }
@@ -264,12 +282,15 @@ __global__ void __launch_bounds__(pf::THREADS, 1)
 
 cudaError_t launch_gemm_fp4(bool nvfp4, const CUtensorMap& tmA, const CUtensorMap& tmB, const GemmArgs& g,
                             int num_sms, bool pdl, cudaStream_t st) {
-    auto kern = nvfp4 ? gemm_fp4_persistent_kernel<true> : gemm_fp4_persistent_kernel<false>;
-    static bool attr_set[2] = {false, false};
-    if (!attr_set[nvfp4]) {
+    // variants: MXFP4, NVFP4 with one B scale, NVFP4 with per-row B scales
+    const int v = !nvfp4 ? 0 : g.s2b_per_row ? 2 : 1;
+    auto kern = v == 0 ? gemm_fp4_persistent_kernel<false, false>
+                       : v == 1 ? gemm_fp4_persistent_kernel<true, false> : gemm_fp4_persistent_kernel<true, true>;
+    static bool attr_set[3] = {false, false, false};
+    if (!attr_set[v]) {
         cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, pf::SMEM);
         if (e != cudaSuccess) return e;
-        attr_set[nvfp4] = true;
+        attr_set[v] = true;
     }
     const int tiles = ((g.M + kBM - 1) / kBM) * ((g.N + pf::BN - 1) / pf::BN);
     const int grid = tiles < num_sms ? tiles : num_sms;

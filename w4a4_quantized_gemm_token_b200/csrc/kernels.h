@@ -52,7 +52,8 @@ struct GemmArgs {
     int sfa_ld, sfb_ld;        // INT4: pad128(M), pad128(N)
     const float* s2a;          // NVFP4 alpha parts (nullable for MXFP4)
     int s2a_per_row;
-    const float* s2b;
+    const float* s2b;          // NVFP4: [1], or [N] (16-byte aligned) when s2b_per_row
+    int s2b_per_row;
     uint16_t* Y;
     int ldy;
     float* partial;            // split-K partial sums (decode variant)
@@ -66,6 +67,8 @@ struct GemmArgs {
 cudaError_t launch_quant(int fmt, bool gather, const QuantArgs& a, int rows_pad, int num_sms, cudaStream_t st);
 cudaError_t launch_amax(const uint16_t* X, int M, int K, int ldx, float* out, int num_sms, cudaStream_t st);
 cudaError_t launch_residual(const ResidualArgs& a, cudaStream_t st);
+// p[1 .. n) = p[0] (device floats)
+cudaError_t launch_spread_first(float* p, int n, cudaStream_t st);
 cudaError_t launch_select(const uint16_t* X, int Mc, int K, int ldx, int nS, int32_t* S, float* amax, int* sel,
                           cudaStream_t st);
 

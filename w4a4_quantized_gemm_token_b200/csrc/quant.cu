@@ -767,6 +767,19 @@ cudaError_t launch_amax(const uint16_t* X, int M, int K, int ldx, float* out, in
     return cudaGetLastError();
 }
 
+// p[1 .. n) = p[0]: spreads a segment's tensor scale over its rows.
+__global__ void spread_first_kernel(float* p, int n) {
+    const float v = p[0];
+    for (int i = 1 + blockIdx.x * blockDim.x + threadIdx.x; i < n; i += gridDim.x * blockDim.x) p[i] = v;
+}
+
+cudaError_t launch_spread_first(float* p, int n, cudaStream_t st) {
+    if (n <= 1) return cudaSuccess;
+    const int grid = (n + 255) / 256 < 64 ? (n + 255) / 256 : 64;
+    spread_first_kernel<<<grid, 256, 0, st>>>(p, n);
+    return cudaGetLastError();
+}
+
 cudaError_t launch_residual(const ResidualArgs& a, cudaStream_t st) {
     long long n = (long long)a.rows_pad * (a.nS / 16);
     residual_kernel<<<(unsigned)((n + 127) / 128), 128, 0, st>>>(a);

@@ -141,6 +141,28 @@ def weights(model: str, N: int, K: int, seed: int = 0, tensor_id: int = 2) -> np
     return normal((N, K), sigma, seed, tensor_id, bf16=True)
 
 
+# Fused projection modules stacked along N: rows of each part and the spread of
+# its weights relative to the model's weight sigma (synthetic; the parts of a
+# fused module differ in magnitude, which is why each gets its own scale).
+FUSED = {
+    "llama2_70b": {"qkv": ((8192, 1024, 1024), (1.0, 4.0, 0.25)),
+                   "w1w3": ((28672, 28672), (1.0, 0.5))},
+}
+
+
+def fused_weights(seg_rows, gains, K: int, model: str = "llama2_70b", seed: int = 0,
+                  tensor_id: int = 2):
+    """W [sum(seg_rows), K] as bf16 bits, part i drawn with sigma * gains[i];
+    returns (bits, row boundaries [0, ..., N])."""
+    sigma = 0.01 if model == "llama2_70b" else 0.02
+    N = int(sum(seg_rows))
+    w = normal((N, K), sigma, seed, tensor_id)
+    bounds = np.concatenate([[0], np.cumsum(seg_rows)]).astype(np.int64)
+    for i, gain in enumerate(gains):
+        w[bounds[i]:bounds[i + 1]] *= np.float32(gain)
+    return f32_to_bf16_bits(w), [int(b) for b in bounds]
+
+
 def calibration(model: str, K: int, rows: int = 512) -> np.ndarray:
     """Calibration batch (seed 1) with the same outlier channels as the run data."""
     return activations(model, rows, K, seed=1, tensor_id=7)

@@ -20,18 +20,20 @@
 //     zero-stride dimension), and one 128 x 256-bit copy then fills the
 //     columns of two atoms -- 6 copies per 256-wide K stage instead of 12
 //     replicating 32 x 128-bit ones.
-//   - the MMA thread issues each stage's copies itself, interleaved with its
-//     4 MMAs (one thread's tcgen05 operations execute in order, so no barrier
-//     sits between a copy and the MMA that reads it, and the tensor pipe
-//     overlaps each copy with the MMA before it).
+//   - a warp of its own issues each stage's copies and signals the MMA warp
+//     through a per-stage barrier (one thread's tcgen05 operations block for
+//     about their execution time; those of two threads overlap in part).
 // All loads are tiled TMA copies without multicast; the odd CTA's copies
 // count their bytes on the even CTA's stage barrier (cta_group::2 form),
 // whose expected byte count covers both CTAs.  Out-of-range row tiles and K
 // tails are zero-filled by the copies.
 // Warp roles (384 threads per CTA):
-//   warp 0 lane 0   TMA producer (both CTAs), 4-stage (NVFP4) / 5-stage (MXFP4) ring
+//   warp 0 lane 0   TMA producer (both CTAs), 4-stage (NVFP4) / 5-stage (MXFP4) ring;
+//                   each stage (56 KB NVFP4) is near the rate at which TMA fills
+//                   shared memory (~64 B per cycle per SM), the bound of this kernel
 //   warp 1          TMEM allocation (both CTAs, together); even CTA lane 0
-//                   issues the scale copies and the MMAs
+//                   issues the MMAs
+//   warp 2          even CTA lane 0 issues the scale-factor copies
 //   warps 4..11     epilogue (both CTAs): TMEM -> registers -> bf16 stores,
 //                   two warps per lane quarter so the accumulator drains fast
 // Every wait is bounded; on expiry the kernel records a timeout, drains its

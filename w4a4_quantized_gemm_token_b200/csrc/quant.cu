@@ -541,11 +541,12 @@ __global__ void __launch_bounds__(1024) compact_kernel(const int* selected, int 
 // NB-1 rows in flight as bulk copies into a ring of shared-memory row
 // buffers, so each SM has its loads outstanding while it computes.  For the
 // current row every thread takes J chunks of 16 elements (items t, t+T, ...)
-// into registers, the CTA reduces the row amax, and the threads tabulate for
-// the row d_c = E4M3(c) * s2 and RN(1/d_c) for all 128 scale codes, so a
-// block needs no reciprocal of its own.  Each item is then quantized from
-// registers: block scale by two refined divisions, codes by refined division
-// with the tabulated reciprocal.  The refined division is exact here whenever
+// into registers and the CTA reduces the row amax: the only CTA barrier of a
+// row (the per-warp maxima alternate between two buffers, so no barrier is
+// needed before the next row rewrites them).  Each item is then quantized
+// from registers: block scale by two refined divisions, codes by refined
+// division with RN(1/d) of its own divisor d = E4M3(scale) * s2.  The refined
+// division is exact here whenever
 // s2 >= 2^-100 (the block quotients are then either below 2^-10, which
 // encodes to zero either way, or normal and at most about 12); a row below
 // that takes IEEE division throughout (a CTA-uniform branch).  Rows
@@ -558,8 +559,7 @@ __global__ void __launch_bounds__(J <= 2 ? 1024 : 768) quant_nvfp4_token_kernel(
     if (blockIdx.x == 0)
         for (int i = threadIdx.x; i < a.zero_count; i += blockDim.x) a.zero_words[i] = 0;
     extern __shared__ __align__(128) uint8_t qring[];
-    __shared__ float wmax[32];
-    __shared__ float2 tab[128];  // (d_c, RN(1/d_c)) for E4M3 codes c (sign 0)
+    __shared__ float wmax[2][32];  // per-warp row maxima, alternating rows
     const int t = threadIdx.x, T = blockDim.x;
     const int lane = t & 31, warp = t >> 5, nwarps = T >> 5;
     const int items = a.K / 16;
@@ -604,18 +604,13 @@ __global__ void __launch_bounds__(J <= 2 ? 1024 : 768) quant_nvfp4_token_kernel(
             m = fmaxf(m, bm[j]);
         }
         m = warp_max(m);
-        if (lane == 0) wmax[warp] = m;
+        if (lane == 0) wmax[i & 1][warp] = m;
         __syncthreads();  // (also: every thread has its row data in registers)
         if (t == 0 && i + nb < nlive) issue(i + nb);  // the buffer is free again
-        const float amax = warp_max(lane < nwarps ? wmax[lane] : 0.0f);
+        const float amax = warp_max(lane < nwarps ? wmax[i & 1][lane] : 0.0f);
         const float s2 = nvfp4_s2(amax);
         const bool fast = s2 >= 0x1p-100f;  // the same for the whole CTA
-        for (int c = t; c < 128; c += T) {
-            const float d = c ? __fmul_rn(e4m3_value((uint8_t)c), s2) : 1.0f;
-            tab[c] = make_float2(d, __frcp_rn(d));
-        }
         if (t == 0) a.s2_out[r] = s2;
-        __syncthreads();
         const float rinv = __frcp_rn(s2);
 #pragma unroll
         for (int j = 0; j < J; ++j) {
@@ -624,12 +619,13 @@ __global__ void __launch_bounds__(J <= 2 ? 1024 : 768) quant_nvfp4_token_kernel(
             if (fast) {
                 const float u = div_refined(bm[j], 6.0f, 0x1.555556p-3f);  // RN(1/6)
                 sb = e4m3_rn_sat(div_refined(u, s2, rinv));
-                const float2 dy = tab[sb];
-                w0 = e2m1x8_fast(w[j], pack2(-dy.y), pack2(dy.x));
-                w1 = e2m1x8_fast(w[j] + 4, pack2(-dy.y), pack2(dy.x));
+                const float d = sb ? __fmul_rn(e4m3_value((uint8_t)sb), s2) : 1.0f;
+                const float y = __frcp_rn(d);
+                w0 = e2m1x8_fast(w[j], pack2(-y), pack2(d));
+                w1 = e2m1x8_fast(w[j] + 4, pack2(-y), pack2(d));
             } else {
                 sb = e4m3_rn_sat(__fdiv_rn(__fdiv_rn(bm[j], 6.0f), s2));
-                const float d = tab[sb].x;
+                const float d = sb ? __fmul_rn(e4m3_value((uint8_t)sb), s2) : 1.0f;
                 w0 = e2m1x8_exact(make_uint4(w[j][0], w[j][1], w[j][2], w[j][3]), d);
                 w1 = e2m1x8_exact(make_uint4(w[j][4], w[j][5], w[j][6], w[j][7]), d);
             }
@@ -648,7 +644,6 @@ __global__ void __launch_bounds__(J <= 2 ? 1024 : 768) quant_nvfp4_token_kernel(
                 *reinterpret_cast<uint2*>(a.codes + (size_t)r * a.ldc + 8 * it) = make_uint2(w0, w1);
             }
         }
-        __syncthreads();  // wmax and tab are rewritten for the next row
     }
     if (*abort_flag && t == 0)  // wait for the copies still in flight
         for (int b = 0; b < nb; ++b) mbar_wait_drain(&bars[b], 0, 100000000ull);

@@ -68,6 +68,7 @@ def _declare(L):
     L.orc_gemm_nvfp4_wrows.argtypes = [_u8p, _u8p, _f32p, C.c_int, _u8p, _u8p, _f32p, C.c_int,
                                        C.c_int, C.c_int, C.c_int, _u16p, _f64p, _f64p]
     L.orc_quant_mxfp4.argtypes = [_u16p, C.c_int, C.c_int, C.c_int, _u8p, _u8p]
+    L.orc_quant_mxfp4_msd.argtypes = [_u16p, C.c_int, C.c_int, C.c_int, C.c_int, _u8p, _u8p]
     L.orc_quant_int4.argtypes = [_u16p, C.c_int, C.c_int, C.c_int, _u8p, _f32p]
     L.orc_dequant_nvfp4.argtypes = [_u8p, _u8p, _f32p, C.c_int, C.c_int, C.c_int, _f64p]
     L.orc_dequant_mxfp4.argtypes = [_u8p, _u8p, C.c_int, C.c_int, _f64p]
@@ -172,6 +173,19 @@ def quant_mxfp4(X):
     scales = np.zeros((M, K // 32), np.uint8)
     _check(lib().orc_quant_mxfp4(_p(X, _u16p), M, K, K, _p(codes, _u8p), _p(scales, _u8p)),
            "quant_mxfp4")
+    return codes, scales
+
+
+def quant_mxfp4_msd(X, passes=2):
+    """Multi-pass MXFP4: pass p quantizes the residual of passes 0..p-1 into
+    columns [p*K, (p+1)*K).  Returns (codes [M, passes*K/2], scales
+    [M, passes*K/32])."""
+    X = _bf16(X)
+    M, K = X.shape
+    codes = np.zeros((M, passes * K // 2), np.uint8)
+    scales = np.zeros((M, passes * K // 32), np.uint8)
+    _check(lib().orc_quant_mxfp4_msd(_p(X, _u16p), M, K, K, passes, _p(codes, _u8p), _p(scales, _u8p)),
+           "quant_mxfp4_msd")
     return codes, scales
 
 

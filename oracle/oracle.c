@@ -258,6 +258,46 @@ int orc_quant_mxfp4(const uint16_t* X, int M, int K, int ldx, uint8_t* codes, ui
     return 0;
 }
 
+/* Multi-pass MXFP4 decomposition ("APEX4: Efficient Pure W4A4 LLM Inference
+ * via Intra-SM Compute Rebalancing" page, para 1, MSD: the activation becomes
+ * a sum of low-precision components, each multiplied with the quantized
+ * weights).  Per 32-element block: pass 0 quantizes x by the MXFP4 rule;
+ * pass p quantizes the residual x - (sum of the earlier passes' values), again
+ * by the MXFP4 rule with its own shared exponent.  The residual is formed in
+ * FP32 and is exact: it is x minus x rounded to a grid at least as coarse as
+ * x's own, so it keeps at most 8 significant bits and is a bf16 value (the
+ * function returns -2 if that ever failed, which would break this reading).
+ * Pass p fills columns [p*K, (p+1)*K): codes [M][passes*K/2], scales
+ * [M][passes*K/32]. */
+int orc_quant_mxfp4_msd(const uint16_t* X, int M, int K, int ldx, int passes, uint8_t* codes,
+                        uint8_t* scales) {
+    if (M < 0 || K % 32 || ldx < K || passes < 1) return -1;
+    const size_t cb = (size_t)passes * (K / 2), sb = (size_t)passes * (K / 32);
+    float x[32];
+    for (int m = 0; m < M; ++m)
+        for (int b = 0; b < K / 32; ++b) {
+            for (int i = 0; i < 32; ++i) x[i] = orc_bf16_to_f32(X[(size_t)m * ldx + 32 * b + i]);
+            for (int p = 0; p < passes; ++p) {
+                uint8_t* c16 = codes + (size_t)m * cb + (size_t)p * (K / 2) + 16 * b;
+                uint8_t* sc = scales + (size_t)m * sb + (size_t)p * (K / 32) + b;
+                mxfp4_block(x, c16, sc);
+                if (p + 1 == passes) break;
+                const float unit = orc_e8m0_decode(*sc);
+                for (int i = 0; i < 32; ++i) {
+                    const uint8_t q = (i & 1) ? (c16[i / 2] >> 4) : (c16[i / 2] & 15);
+                    const float v = orc_e2m1_decode(q) * unit; /* exact: 3 significant bits */
+                    const float r = x[i] - v;
+                    if ((double)r != (double)x[i] - (double)v) return -2;
+                    uint32_t u;
+                    memcpy(&u, &r, 4);
+                    if (u & 0xFFFFu) return -2; /* not a bf16 value */
+                    x[i] = r;
+                }
+            }
+        }
+    return 0;
+}
+
 void orc_dequant_mxfp4(const uint8_t* codes, const uint8_t* scales, int M, int K, double* out) {
     for (int m = 0; m < M; ++m)
         for (int k = 0; k < K; ++k) {

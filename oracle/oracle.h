@@ -69,6 +69,13 @@ int orc_quant_nvfp4_segments(const uint16_t* X, int M, int K, int ldx,
 /* codes [M][K/2], scales [M][K/32] E8M0 bytes                             */
 int orc_quant_mxfp4(const uint16_t* X, int M, int K, int ldx,
                     uint8_t* codes, uint8_t* scales);
+/* Multi-pass MXFP4 ("APEX4: Efficient Pure W4A4..." page, para 1, MSD): pass
+ * p quantizes the residual left by passes 0..p-1 (exact, a bf16 value) with
+ * its own shared exponents into columns [p*K, (p+1)*K).  codes
+ * [M][passes*K/2], scales [M][passes*K/32].  Returns -2 if a residual were
+ * not exact (never, under the MXFP4 rule above).                           */
+int orc_quant_mxfp4_msd(const uint16_t* X, int M, int K, int ldx, int passes,
+                        uint8_t* codes, uint8_t* scales);
 /* codes [M][K/2] two's-complement nibbles, scales [M][K/128] FP32          */
 int orc_quant_int4(const uint16_t* X, int M, int K, int ldx,
                    uint8_t* codes, float* scales);

@@ -416,3 +416,87 @@ def test_gemm_per_row_weight_scale(orc):
     Y0, y0, _ = orc.gemm_nvfp4(ca, sa, s2a, 1, cw0, sw0, t0)
     np.testing.assert_array_equal(Y1, Y0)
     np.testing.assert_array_equal(y1, y0)
+
+
+# ---- multi-pass MXFP4 (MSD) -------------------------------------------------
+def _mx_values(codes, scales, K):
+    """Values of MXFP4 codes by the ml_dtypes decoder and 2^(c-127)."""
+    return lib_e2m1(unpack(codes)) * np.repeat(np.exp2(scales.astype(np.float64) - 127), 32, axis=-1)[..., :K]
+
+
+def _msd_inputs():
+    X = np.concatenate([synth.normal((6, 256), 1.0, 51, 1),
+                        synth.student_t((6, 256), 4.0, 0.5, 51, 2) * np.exp2(np.array([-30, -3, 0, 5, 20, 60]))[:, None]])
+    X[0, :32] = 0.0                       # an all-zero block
+    X[1, 32:64] = -0.0                    # negative zeros
+    X[2, 64:96] = 1e-38                   # tiny values
+    X[3, 100] = 3e38                      # near the top of the range
+    return bf16(X)
+
+
+def test_msd_one_pass_is_mxfp4(orc):
+    Xb = _msd_inputs()
+    c1, s1 = orc.quant_mxfp4_msd(Xb, passes=1)
+    c, s = orc.quant_mxfp4(Xb)
+    np.testing.assert_array_equal(c1, c)
+    np.testing.assert_array_equal(s1, s)
+
+
+def test_msd_exact_inputs_leave_no_residual(orc):
+    """Blocks already on the MXFP4 grid (block maximum 4 or 6 times 2^e) are
+    reproduced by the first pass; the second pass sees zeros only."""
+    M, K = 4, 256
+    V = synth.e2m1_grid_values((M, K), 52, 1)
+    V[:, ::32] = 6.0
+    V[1, ::32] = -4.0
+    V *= np.exp2(np.arange(M) * 7 - 10)[:, None]
+    c, s = orc.quant_mxfp4_msd(bf16(V), passes=2)
+    np.testing.assert_array_equal(_mx_values(c[:, :K // 2], s[:, :K // 32], K), V)
+    assert np.all(unpack(c[:, K // 2:]) & 7 == 0) and np.all(s[:, K // 32:] == 0)
+
+
+@pytest.mark.parametrize("passes", [2, 3])
+def test_msd_passes_follow_the_rule_on_the_residual(orc, passes):
+    """Each later pass is the MXFP4 rule (restated here with frexp and the
+    brute-force grid search) applied to the exact residual of the earlier
+    passes; the residual is a bf16 value; every pass shrinks every element's
+    error; a pass's error is at most twice its block unit (once without
+    saturation)."""
+    Xb = _msd_inputs()
+    M, K = Xb.shape
+    c, s = orc.quant_mxfp4_msd(Xb, passes=passes)
+    x = synth.bf16_bits_to_f32(Xb).astype(np.float64)
+    r = x.copy()
+    prev = np.abs(r)
+    for p in range(passes):
+        cp, sp = c[:, p * K // 2:(p + 1) * K // 2], s[:, p * K // 32:(p + 1) * K // 32]
+        # the rule on this pass's input r
+        for m in range(M):
+            for b in range(K // 32):
+                blk = r[m, 32 * b:32 * b + 32]
+                a = np.abs(blk).max()
+                e = 0 if a == 0 else int(np.clip(np.frexp(a)[1] - 1 - 2 + 127, 0, 254))
+                assert sp[m, b] == e, (p, m, b)
+                want = [0] * 32 if a == 0 else [brute_e2m1(v * 2.0 ** (127 - e)) for v in blk]
+                np.testing.assert_array_equal(unpack(cp)[m, 32 * b:32 * b + 32], want)
+        v = _mx_values(cp, sp, K)
+        unit = np.repeat(np.exp2(sp.astype(np.float64) - 127), 32, axis=-1)
+        sat = np.abs(r) > 6 * unit
+        r = r - v
+        assert np.all(np.abs(r) <= np.where(sat, 2.0, 1.0) * unit)
+        assert np.all(np.abs(r) <= prev)
+        prev = np.abs(r)
+        # the residual is exact in bf16
+        np.testing.assert_array_equal(synth.bf16_bits_to_f32(bf16(r)).astype(np.float64), r)
+
+
+def test_msd_two_passes_cut_the_error(orc):
+    """On the Llama-like activations two passes cut the RMS error by more than
+    4x (each pass has the resolution of one E2M1 grid under its own unit)."""
+    Xb = synth.activations("llama2_70b", 64, 1024, seed=53)
+    x = synth.bf16_bits_to_f32(Xb).astype(np.float64)
+    c1, s1 = orc.quant_mxfp4(Xb)
+    c2, s2 = orc.quant_mxfp4_msd(Xb, passes=2)
+    e1 = x - _mx_values(c1, s1, 1024)
+    e2 = x - _mx_values(c2[:, :512], s2[:, :32], 1024) - _mx_values(c2[:, 512:], s2[:, 32:], 1024)
+    assert np.sqrt((e2 ** 2).mean()) < np.sqrt((e1 ** 2).mean()) / 4

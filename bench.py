@@ -492,6 +492,35 @@ def extra_rows(args, dev, stream, P):
             del X, Y, ws
         del variants, fl
 
+    # multi-pass MXFP4 (two passes) on the Llama qkv shape: the quantizer alone
+    # (L2 flushed before each launch) and the linear, beside one-pass MXFP4
+    if want("msd"):
+        K, N, M = 8192, 10240, args.tokens
+        Wd = to_dev(synth.weights("llama2_70b", N, K, tensor_id=100), dev)
+        W1, W2 = w4.quantize_weight(Wd, w4.MXFP4), w4.quantize_weight_msd(Wd, 2)
+        del Wd
+        X = to_dev(synth.activations("llama2_70b", M, K, seed=7), dev)
+        q = w4.QTensor(w4.MXFP4, M, 2 * K, 0, dev)
+        fl = l2_flush_buffer(dev)
+        f = lambda: w4.quantize_act_msd(X, 2, out=q)
+        for _ in range(max(3, args.warmup)):
+            f()
+        ms = time_loop(f, it, stream, fl)
+        byts = 2 * M * K + 2 * (M * K / 2 + M * K / 32)
+        out["msd2_quant_llama_qkv_in"] = {"GB/s": round(byts / ms / 1e6, 1), "frac_hbm": round(byts / ms / 1e6 / hbm, 3),
+                                          "us": round(ms * 1e3, 2)}
+        del fl
+        Y = torch.empty(M, N, dtype=torch.bfloat16, device=dev)
+        for name, fn, passes in (("mxfp4_1pass", lambda: w4.linear(X, W1, 0, Y=Y), 1),
+                                 ("msd2", lambda: w4.linear_msd(X, W2, 2, Y=Y), 2)):
+            for _ in range(max(3, args.warmup)):
+                fn()
+            ms = time_loop(fn, it, stream)
+            out[f"{name}_linear_llama_qkv_m{M}"] = {
+                "TFLOPS_exec": round(2.0 * M * N * K * passes / (ms * 1e-3) / 1e12, 1),
+                "TFLOPS_effective_K": round(2.0 * M * N * K / (ms * 1e-3) / 1e12, 1), "us": round(ms * 1e3, 2)}
+        del W1, W2, X, q, Y
+
     if not want("mxfp4"):
         torch.cuda.synchronize()
         assert w4.device_status() == w4.OK
@@ -524,7 +553,7 @@ def main():
     ap.add_argument("--cpu-rows", type=int, default=8, help="cpu_baseline sample: tokens")
     ap.add_argument("--cpu-cols", type=int, default=4096, help="cpu_baseline sample: output columns")
     ap.add_argument("--no-rows", action="store_true", help="skip the secondary rows")
-    ap.add_argument("--only", choices=["gemm", "quant", "decode", "int4", "aug", "mxfp4", "segments"], default=None,
+    ap.add_argument("--only", choices=["gemm", "quant", "decode", "int4", "aug", "mxfp4", "segments", "msd"], default=None,
                     help="run only one secondary row (for profiling) and print it")
     ap.add_argument("--no-cpu", action="store_true", help="skip the oracle CPU baseline")
     ap.add_argument("--shape", default=None, help="--only gemm: one Llama linear (qkv, o, w1, w3, w2)")

@@ -168,6 +168,31 @@ int w4a4_quantize_weight_segments(const uint16_t* W, int N, int K, int ldw,
                                   w4a4_qtensor* out, void* stream);
 
 /*
+ * Multi-pass MXFP4 decomposition of activations ("APEX4: Efficient Pure W4A4
+ * LLM Inference via Intra-SM Compute Rebalancing" page, para 1, MSD: the
+ * activation is split into several low-precision components, each multiplied
+ * directly with the quantized weights).  Pass 0 is w4a4_quantize_act's MXFP4
+ * rule on X; pass p applies the same rule, with its own shared exponents, to
+ * the residual X - (values of passes 0..p-1), formed exactly in FP32 (it is
+ * always a bf16 value).  Pass p fills columns [p*K, (p+1)*K) of `out`.
+ *   passes: 1 .. 4 (1 is plain MXFP4).
+ *   out: format MXFP4, rows = M, cols = passes * K.
+ * Multiplied with w4a4_quantize_weight_msd's [W | W | ...] (one GEMM over
+ * passes * K), the product is sum_p X_p W^T.
+ */
+int w4a4_quantize_act_msd(const uint16_t* X, int M, int K, int ldx, int passes,
+                          w4a4_qtensor* out, void* stream);
+
+/*
+ * The weight side of the multi-pass product: W[N,K] quantized to MXFP4 once
+ * and repeated `passes` times along K (cols = passes * K), so that one GEMM
+ * multiplies every activation pass with the same weights.
+ *   out: format MXFP4, rows = N, cols = passes * K.
+ */
+int w4a4_quantize_weight_msd(const uint16_t* W, int N, int K, int ldw, int passes,
+                             w4a4_qtensor* out, void* stream);
+
+/*
  * Y[M,N] = A * B^T for quantized A (activations, rows = M) and B (weights,
  * rows = N) of the same format and the same cols (= K, or K + nS).
  *   NVFP4/MXFP4: block-scaled tensor-core MMA, FP32 accumulation;
@@ -221,6 +246,17 @@ int w4a4_linear_noalloc(const uint16_t* X, int M, int K, int ldx,
                         const w4a4_qtensor* Wq, int scale_mode,
                         const int32_t* S, int nS,
                         uint16_t* Y, int ldy, void* stream);
+
+/*
+ * The multi-pass MXFP4 linear layer: w4a4_quantize_act_msd of X[M,K] into the
+ * workspace, then one MXFP4 GEMM over passes * K columns with Wq (made by
+ * w4a4_quantize_weight_msd with the same passes), Y[M,N] bf16.  ws: at least
+ * w4a4_linear_workspace(M, N, K, W4A4_MXFP4, (passes - 1) * K) bytes,
+ * 256-byte aligned.  M <= 16 takes the split-K decode variant.
+ */
+int w4a4_linear_msd(const uint16_t* X, int M, int K, int ldx,
+                    const w4a4_qtensor* Wq, int passes,
+                    uint16_t* Y, int ldy, void* ws, size_t ws_bytes, void* stream);
 
 /*
  * Second stage of the dual-stage NVFP4 quantization ("APEX4..." page,

@@ -145,3 +145,21 @@ def test_segment_weight_arguments(L):
     assert seg_call([0, 512], out, S=C.c_void_p(16), nS=128) == w4.ERR_INVALID_ARG
     aug = _qt(w4.NVFP4, 512, 384, w4.SCALE_TOKEN)
     assert seg_call([0, 512], aug, S=C.c_void_p(16), nS=64) == w4.ERR_INVALID_ARG
+
+
+def test_msd_arguments(L):
+    """Multi-pass MXFP4: pass count, output format and width are checked on the host."""
+    out = _qt(w4.MXFP4, 4, 512)
+    X = C.c_void_p(16)
+    assert L.w4a4_quantize_act_msd(X, 4, 256, 256, 0, C.byref(out), None) == w4.ERR_INVALID_ARG   # passes < 1
+    assert L.w4a4_quantize_act_msd(X, 4, 256, 256, 5, C.byref(out), None) == w4.ERR_INVALID_ARG   # passes > 4
+    assert L.w4a4_quantize_act_msd(X, 4, 256, 256, 3, C.byref(out), None) == w4.ERR_INVALID_ARG   # cols != 3K
+    nv = _qt(w4.NVFP4, 4, 512, w4.SCALE_TOKEN)
+    assert L.w4a4_quantize_act_msd(X, 4, 256, 256, 2, C.byref(nv), None) == w4.ERR_INVALID_ARG    # not MXFP4
+    assert L.w4a4_quantize_act_msd(C.c_void_p(18), 4, 256, 256, 2, C.byref(out), None) == w4.ERR_MISALIGNED
+    W = _qt(w4.MXFP4, 256, 512)
+    assert L.w4a4_quantize_weight_msd(X, 256, 256, 256, 3, C.byref(W), None) == w4.ERR_INVALID_ARG
+    assert L.w4a4_linear_msd(X, 4, 256, 256, C.byref(W), 3, C.c_void_p(16), 256, C.c_void_p(256), 1 << 20,
+                             None) == w4.ERR_INVALID_ARG
+    assert L.w4a4_linear_msd(X, 4, 256, 256, C.byref(W), 2, C.c_void_p(16), 256, C.c_void_p(256), 16,
+                             None) == w4.ERR_WORKSPACE

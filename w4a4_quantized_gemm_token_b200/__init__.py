@@ -26,7 +26,8 @@ OK, ERR_INVALID_ARG, ERR_MISALIGNED, ERR_WORKSPACE, ERR_ARCH, ERR_CUDA, ERR_DEVI
 EXPORTS = ("w4a4_qtensor_bytes", "w4a4_quantize_act", "w4a4_quantize_weight", "w4a4_gemm",
            "w4a4_linear_workspace", "w4a4_linear", "w4a4_augment_residual", "w4a4_select_channels",
            "w4a4_device_status", "w4a4_debug_set", "w4a4_status_string", "w4a4_linear_noalloc",
-           "w4a4_quantize_weight_segments")
+           "w4a4_quantize_weight_segments", "w4a4_quantize_act_msd", "w4a4_quantize_weight_msd",
+           "w4a4_linear_msd")
 
 
 class W4A4Error(RuntimeError):
@@ -59,6 +60,9 @@ def lib():
         L.w4a4_quantize_weight.argtypes = [vp, i, i, i, i, i, vp, i, qp, vp]
         L.w4a4_quantize_weight_segments.argtypes = [vp, i, i, i, C.POINTER(C.c_int32), i, vp, i, qp, vp]
         L.w4a4_gemm.argtypes = [qp, qp, vp, i, vp]
+        L.w4a4_quantize_act_msd.argtypes = [vp, i, i, i, i, qp, vp]
+        L.w4a4_quantize_weight_msd.argtypes = [vp, i, i, i, i, qp, vp]
+        L.w4a4_linear_msd.argtypes = [vp, i, i, i, qp, i, vp, i, vp, sz, vp]
         L.w4a4_linear_workspace.argtypes = [i, i, i, i, i]
         L.w4a4_linear_workspace.restype = sz
         L.w4a4_linear.argtypes = [vp, i, i, i, qp, i, vp, i, vp, i, vp, sz, vp]
@@ -72,7 +76,8 @@ def lib():
         L.w4a4_status_string.restype = C.c_char_p
         for name in ("w4a4_qtensor_bytes", "w4a4_quantize_act", "w4a4_quantize_weight", "w4a4_gemm",
                      "w4a4_linear", "w4a4_augment_residual", "w4a4_select_channels", "w4a4_device_status",
-                     "w4a4_linear_noalloc", "w4a4_quantize_weight_segments"):
+                     "w4a4_linear_noalloc", "w4a4_quantize_weight_segments", "w4a4_quantize_act_msd",
+                     "w4a4_quantize_weight_msd", "w4a4_linear_msd"):
             getattr(L, name).restype = i
         _lib = L
     return _lib
@@ -160,6 +165,41 @@ def quantize_weight_segments(W, seg, S=None, out: QTensor | None = None) -> QTen
     _check(lib().w4a4_quantize_weight_segments(_ptr(W), N, K, W.stride(0), arr, len(seg) - 1, _ptr(S), nS,
                                                out.ref, _stream()), "w4a4_quantize_weight_segments")
     return out
+
+
+def quantize_act_msd(X, passes: int = 2, out: QTensor | None = None) -> QTensor:
+    """Multi-pass MXFP4 activations: pass p (the residual of the earlier
+    passes) in columns [p*K, (p+1)*K)."""
+    M, K = X.shape
+    if out is None:
+        out = QTensor(MXFP4, M, passes * K, SCALE_TENSOR, X.device)
+    _check(lib().w4a4_quantize_act_msd(_ptr(X), M, K, X.stride(0), passes, out.ref, _stream()),
+           "w4a4_quantize_act_msd")
+    return out
+
+
+def quantize_weight_msd(W, passes: int = 2, out: QTensor | None = None) -> QTensor:
+    """MXFP4 weights repeated `passes` times along K, for the multi-pass product."""
+    N, K = W.shape
+    if out is None:
+        out = QTensor(MXFP4, N, passes * K, SCALE_TENSOR, W.device)
+    _check(lib().w4a4_quantize_weight_msd(_ptr(W), N, K, W.stride(0), passes, out.ref, _stream()),
+           "w4a4_quantize_weight_msd")
+    return out
+
+
+def linear_msd(X, Wq: QTensor, passes: int = 2, Y=None, ws=None):
+    """The multi-pass MXFP4 linear layer (Wq from quantize_weight_msd)."""
+    import torch
+    M, K = X.shape
+    if Y is None:
+        Y = torch.empty(M, Wq.rows, dtype=torch.bfloat16, device=X.device)
+    need = linear_workspace(M, Wq.rows, K, MXFP4, (passes - 1) * K)
+    if ws is None:
+        ws = torch.empty(max(need, 256), dtype=torch.uint8, device=X.device)
+    _check(lib().w4a4_linear_msd(_ptr(X), M, K, X.stride(0), Wq.ref, passes, _ptr(Y), Y.stride(0), _ptr(ws),
+                                 ws.numel(), _stream()), "w4a4_linear_msd")
+    return Y
 
 
 def gemm(A: QTensor, B: QTensor, Y=None):

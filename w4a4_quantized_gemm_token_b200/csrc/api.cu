@@ -20,6 +20,7 @@ namespace {
 
 constexpr int kMaxDevices = 64;
 constexpr int kMaxK = 65536;
+constexpr int kMaxPasses = 4;  // multi-pass MXFP4 decomposition
 
 struct DevInfo {
     bool init = false;
@@ -113,7 +114,7 @@ int check_qtensor(const w4a4_qtensor* q) {
     if (!q || !q->codes || !q->scales) return W4A4_ERR_INVALID_ARG;
     if (q->format < 0 || q->format > 2 || q->group != group_of(q->format) || q->reserved != 0)
         return W4A4_ERR_INVALID_ARG;
-    if (q->rows < 0 || q->cols < 128 || q->cols % 128 || q->cols > kMaxK + 32768) return W4A4_ERR_INVALID_ARG;
+    if (q->rows < 0 || q->cols < 128 || q->cols % 128 || q->cols > kMaxPasses * kMaxK) return W4A4_ERR_INVALID_ARG;
     if (q->format == W4A4_NVFP4) {
         if (!q->s2) return W4A4_ERR_INVALID_ARG;
         if (q->scale_mode != W4A4_SCALE_TENSOR && q->scale_mode != W4A4_SCALE_TOKEN) return W4A4_ERR_INVALID_ARG;
@@ -129,8 +130,10 @@ int cuda_status(cudaError_t e) { return e == cudaSuccess ? W4A4_OK : W4A4_ERR_CU
 
 // Quantize rows [0, M) of X into the first K columns of q (q->cols >= K).
 int quantize_rows(const uint16_t* X, int M, int K, int ldx, const int32_t* S, int K_src, const float* static_s2,
-                  w4a4_qtensor* q, int num_sms, cudaStream_t st, int* zero_words = nullptr, int zero_count = 0) {
+                  w4a4_qtensor* q, int num_sms, cudaStream_t st, int* zero_words = nullptr, int zero_count = 0,
+                  int passes = 1) {
     QuantArgs a{};
+    a.passes = passes;
     a.zero_words = zero_words;
     a.zero_count = zero_count;
     a.X = X;
@@ -389,6 +392,53 @@ int w4a4_quantize_weight_segments(const uint16_t* W, int N, int K, int ldw, cons
     return W4A4_OK;
 }
 
+int w4a4_quantize_act_msd(const uint16_t* X, int M, int K, int ldx, int passes, w4a4_qtensor* out, void* stream) {
+    if (M < 0 || K < 128 || K % 128 || K > kMaxK || ldx < K || passes < 1 || passes > kMaxPasses)
+        return W4A4_ERR_INVALID_ARG;
+    int rc = check_qtensor(out);
+    if (rc != W4A4_OK) return rc;
+    if (out->format != W4A4_MXFP4 || out->rows != M || out->cols != passes * K) return W4A4_ERR_INVALID_ARG;
+    if (M == 0) return W4A4_OK;
+    if (!X) return W4A4_ERR_INVALID_ARG;
+    if (!aligned16(X) || ldx % 8) return W4A4_ERR_MISALIGNED;
+    int sms = 0;
+    rc = device_check(&sms);
+    if (rc != W4A4_OK) return rc;
+    return quantize_rows(X, M, K, ldx, nullptr, K, nullptr, out, sms, as_stream(stream), nullptr, 0, passes);
+}
+
+// The weight side of the multi-pass product: W quantized once into the first
+// K columns, then copied into the other passes' columns (codes row by row,
+// scale atoms row tile by row tile).
+int w4a4_quantize_weight_msd(const uint16_t* W, int N, int K, int ldw, int passes, w4a4_qtensor* out, void* stream) {
+    if (N < 0 || K < 128 || K % 128 || K > kMaxK || ldw < K || passes < 1 || passes > kMaxPasses)
+        return W4A4_ERR_INVALID_ARG;
+    int rc = check_qtensor(out);
+    if (rc != W4A4_OK) return rc;
+    if (out->format != W4A4_MXFP4 || out->rows != N || out->cols != passes * K) return W4A4_ERR_INVALID_ARG;
+    if (N == 0) return W4A4_OK;
+    if (!W) return W4A4_ERR_INVALID_ARG;
+    if (!aligned16(W) || ldw % 8) return W4A4_ERR_MISALIGNED;
+    int sms = 0;
+    rc = device_check(&sms);
+    if (rc != W4A4_OK) return rc;
+    cudaStream_t st = as_stream(stream);
+    rc = quantize_rows(W, N, K, ldw, nullptr, K, nullptr, out, sms, st);
+    if (rc != W4A4_OK) return rc;
+    uint8_t* codes = static_cast<uint8_t*>(out->codes);
+    uint8_t* scales = static_cast<uint8_t*>(out->scales);
+    const size_t row_b = (size_t)passes * K / 2, part_b = (size_t)K / 2;
+    const size_t atoms = (size_t)K / 32 / 4, tile_b = (size_t)passes * atoms * 512;
+    for (int p = 1; p < passes; ++p) {
+        cudaError_t e = cudaMemcpy2DAsync(codes + p * part_b, row_b, codes, row_b, part_b, N, cudaMemcpyDeviceToDevice, st);
+        if (e == cudaSuccess)
+            e = cudaMemcpy2DAsync(scales + p * atoms * 512, tile_b, scales, tile_b, atoms * 512, pad128(N) / 128,
+                                  cudaMemcpyDeviceToDevice, st);
+        if (e != cudaSuccess) return W4A4_ERR_CUDA;
+    }
+    return W4A4_OK;
+}
+
 int w4a4_gemm(const w4a4_qtensor* A, const w4a4_qtensor* B, uint16_t* Y, int ldy, void* stream) {
     int rc = check_qtensor(A);
     if (rc == W4A4_OK) rc = check_qtensor(B);
@@ -457,6 +507,43 @@ int w4a4_linear(const uint16_t* X, int M, int K, int ldx, const w4a4_qtensor* Wq
                        static_cast<uint8_t*>(xq.scales), xq.cols / 16 / 4, xq.s2, xq.scale_mode};
         if (launch_residual(r, st) != cudaSuccess) return W4A4_ERR_CUDA;
     }
+    float* partial = small_m ? reinterpret_cast<float*>(base + L.partial) : nullptr;
+    return run_gemm(&xq, Wq, Y, ldy, partial, sms, true, st, counters);
+}
+
+int w4a4_linear_msd(const uint16_t* X, int M, int K, int ldx, const w4a4_qtensor* Wq, int passes, uint16_t* Y,
+                    int ldy, void* ws, size_t ws_bytes, void* stream) {
+    int rc = check_qtensor(Wq);
+    if (rc != W4A4_OK) return rc;
+    if (M < 0 || K < 128 || K % 128 || K > kMaxK || ldx < K || passes < 1 || passes > kMaxPasses)
+        return W4A4_ERR_INVALID_ARG;
+    if (Wq->format != W4A4_MXFP4 || Wq->cols != passes * K || Wq->rows < 128 || Wq->rows % 128 || ldy < Wq->rows)
+        return W4A4_ERR_INVALID_ARG;
+    if (M == 0) return W4A4_OK;
+    if (!X || !Y) return W4A4_ERR_INVALID_ARG;
+    if (!aligned16(X) || ldx % 8 || !aligned16(Y) || ldy % 8) return W4A4_ERR_MISALIGNED;
+    const int N = Wq->rows;
+    const WsLayout L = ws_layout(M, N, K, W4A4_MXFP4, (passes - 1) * K);
+    if (!ws || ws_bytes < L.total) return W4A4_ERR_WORKSPACE;
+    if (reinterpret_cast<uintptr_t>(ws) & 255) return W4A4_ERR_MISALIGNED;
+    int sms = 0;
+    rc = device_check(&sms);
+    if (rc != W4A4_OK) return rc;
+    cudaStream_t st = as_stream(stream);
+    uint8_t* base = static_cast<uint8_t*>(ws);
+    w4a4_qtensor xq{};
+    xq.format = W4A4_MXFP4;
+    xq.rows = M;
+    xq.cols = passes * K;
+    xq.group = 32;
+    xq.codes = base + L.codes;
+    xq.scales = base + L.scales;
+    xq.s2 = nullptr;
+    const bool small_m = M <= 16;
+    int* counters = small_m ? reinterpret_cast<int*>(base + L.counters) : nullptr;
+    rc = quantize_rows(X, M, K, ldx, nullptr, K, nullptr, &xq, sms, st, counters, small_m ? (N + kBM - 1) / kBM : 0,
+                       passes);
+    if (rc != W4A4_OK) return rc;
     float* partial = small_m ? reinterpret_cast<float*>(base + L.partial) : nullptr;
     return run_gemm(&xq, Wq, Y, ldy, partial, sms, true, st, counters);
 }

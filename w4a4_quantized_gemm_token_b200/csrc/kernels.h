@@ -29,6 +29,8 @@ struct QuantArgs {
     int rows_pad;              // pad128(M): rows of the scale atoms (set by the launcher)
     int* zero_words;           // nullable: words the first CTA clears (a later kernel's counters)
     int zero_count;
+    int passes;                // MXFP4: 1, or more for the multi-pass decomposition (pass p
+                               // in columns [p*K, (p+1)*K) of codes and scales)
 };
 
 struct ResidualArgs {

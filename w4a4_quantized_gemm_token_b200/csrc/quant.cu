@@ -160,6 +160,26 @@ __device__ __forceinline__ size_t sf_offset(int r, int c, int col_atoms) {
     return ((size_t)(r >> 7) * col_atoms + (c >> 2)) * 512 + (r & 31) * 16 + ((r >> 5) & 3) * 4 + (c & 3);
 }
 
+// MXFP4 shared-exponent code of a block with amax a > 0: floor(log2 a) - 2,
+// biased by 127 and clamped to E8M0's range (subnormal amaxes included).
+__device__ __forceinline__ uint32_t mx_code(float a) {
+    const uint32_t u = __float_as_uint(a);
+    const int E = (int)(u >> 23);
+    const int e = (E != 0) ? E - 127 : (31 - __clz((int)(u & 0x7FFFFF))) - 149;
+    return (uint32_t)min(max(e + 125, 0), 254);
+}
+// 2^(code - 127), the unit of an E8M0 code (code 0 is the subnormal 2^-127).
+__device__ __forceinline__ float mx_unit(uint32_t code) {
+    return code ? __uint_as_float(code << 23) : __uint_as_float(0x00400000u);
+}
+// Value of an E2M1 code (bit 3 the sign): m/2 for exponent field 0, else
+// (1 + m/2) * 2^(e-1); built as float bits.
+__device__ __forceinline__ float e2m1_decode(uint32_t nib) {
+    const uint32_t e = (nib >> 1) & 3u, m = nib & 1u;
+    const uint32_t mag = e ? (((e + 126u) << 23) | (m << 22)) : (m ? 0x3F000000u : 0u);
+    return __uint_as_float(mag | ((nib & 8u) << 28));
+}
+
 __device__ __forceinline__ float warp_max(float v) {
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
@@ -184,7 +204,8 @@ struct RowConsts {
     int pad;
 };
 
-template <int FMT, bool GATHER>
+// MULTI (MXFP4 only): the multi-pass decomposition, a.passes passes.
+template <int FMT, bool GATHER, bool MULTI = false>
 __global__ void __launch_bounds__(256, 4) quant_rows_kernel(QuantArgs a, int rows_per_cta, int nbuf) {
     pdl_launch_dependents();
     pdl_wait();  // X and the words to clear may belong to the preceding launch
@@ -341,10 +362,7 @@ __global__ void __launch_bounds__(256, 4) quant_rows_kernel(QuantArgs a, int row
             bmax = fmaxf(bmax, __shfl_xor_sync(0xffffffffu, bmax, 1));  // 32-element block = 2 items
             uint32_t code = 0;
             if (live && bmax > 0.0f) {
-                const uint32_t u = __float_as_uint(bmax);
-                const int E = (int)(u >> 23);
-                const int e = (E != 0) ? E - 127 : (31 - __clz((int)(u & 0x7FFFFF))) - 149;
-                code = (uint32_t)min(max(e + 125, 0), 254);
+                code = mx_code(bmax);
                 const float inv = __uint_as_float((254u - code) << 23);  // 2^(127 - code)
                 float q0[8], q1[8];
 #pragma unroll
@@ -363,6 +381,52 @@ __global__ void __launch_bounds__(256, 4) quant_rows_kernel(QuantArgs a, int row
             if (valid && (c & 7) == 0)
                 *reinterpret_cast<uint32_t*>(a.sf + sf_offset(r, c >> 1, a.sf_col_atoms)) =
                     code | (b1 << 8) | (b2 << 16) | (b3 << 24);
+            if constexpr (MULTI) {
+                // Multi-pass decomposition ("APEX4: Efficient Pure W4A4..." page,
+                // para 1, MSD): pass p quantizes, by the same rule, the residual
+                // x - (values of passes 0..p-1), formed in FP32 (exact: a bf16 value).
+                float res[16];
+#pragma unroll
+                for (int e2 = 0; e2 < 8; ++e2) {
+                    res[e2] = (e2 & 1) ? bf16hi(w[e2 >> 1]) : bf16lo(w[e2 >> 1]);
+                    res[8 + e2] = (e2 & 1) ? bf16hi(w[4 + (e2 >> 1)]) : bf16lo(w[4 + (e2 >> 1)]);
+                }
+                uint32_t pc = code, p0 = w0, p1 = w1;
+                for (int p = 1; p < a.passes; ++p) {
+                    const float unit = mx_unit(pc);
+                    float rmax = 0.0f;
+#pragma unroll
+                    for (int e2 = 0; e2 < 16; ++e2) {
+                        const uint32_t nib = ((e2 < 8 ? p0 : p1) >> (4 * (e2 & 7))) & 15u;
+                        res[e2] = __fsub_rn(res[e2], __fmul_rn(e2m1_decode(nib), unit));
+                        rmax = fmaxf(rmax, fabsf(res[e2]));
+                    }
+                    rmax = fmaxf(rmax, __shfl_xor_sync(0xffffffffu, rmax, 1));
+                    pc = 0;
+                    p0 = p1 = 0;
+                    if (live && rmax > 0.0f) {
+                        pc = mx_code(rmax);
+                        const float inv = __uint_as_float((254u - pc) << 23);
+                        float q0[8], q1[8];
+#pragma unroll
+                        for (int e2 = 0; e2 < 8; ++e2) {
+                            q0[e2] = __fmul_rn(res[e2], inv);
+                            q1[e2] = __fmul_rn(res[8 + e2], inv);
+                        }
+                        p0 = e2m1x8(q0);
+                        p1 = e2m1x8(q1);
+                    }
+                    const uint32_t c1 = __shfl_down_sync(0xffffffffu, pc, 2);
+                    const uint32_t c2 = __shfl_down_sync(0xffffffffu, pc, 4);
+                    const uint32_t c3 = __shfl_down_sync(0xffffffffu, pc, 6);
+                    if (valid && (c & 7) == 0)
+                        *reinterpret_cast<uint32_t*>(a.sf + sf_offset(r, p * (a.K >> 5) + (c >> 1), a.sf_col_atoms)) =
+                            pc | (c1 << 8) | (c2 << 16) | (c3 << 24);
+                    if (live)
+                        *reinterpret_cast<uint2*>(a.codes + (size_t)r * a.ldc + (size_t)p * (a.K >> 1) + 8 * c) =
+                            make_uint2(p0, p1);
+                }
+            }
         } else {  // INT4, 128-element group = 8 items
             bmax = fmaxf(bmax, __shfl_xor_sync(0xffffffffu, bmax, 1));
             bmax = fmaxf(bmax, __shfl_xor_sync(0xffffffffu, bmax, 2));
@@ -713,7 +777,7 @@ static cudaError_t launch_nvfp4_token(const QuantArgs& a, int rows_pad, int num_
     return e != cudaSuccess ? e : cudaGetLastError();
 }
 
-template <int FMT, bool GATHER>
+template <int FMT, bool GATHER, bool MULTI = false>
 static cudaError_t launch_quant_fmt(const QuantArgs& a, int rows_pad, int num_sms, cudaStream_t st) {
     const int row_bytes = a.K_src * 2;
     // One row block per CTA (about 32 KB of rows, several CTAs resident per
@@ -725,7 +789,7 @@ static cudaError_t launch_quant_fmt(const QuantArgs& a, int rows_pad, int num_sm
     const size_t smem = nbuf * buf + 8 * nbuf + 4 * rpc + sizeof(RowConsts) * rpc +
                         (FMT == FMT_NVFP4 ? 4 * (size_t)rpc * (a.K / 16) : 0) + 16;
     if (smem > 200 * 1024) return cudaErrorInvalidValue;
-    auto kern = quant_rows_kernel<FMT, GATHER>;
+    auto kern = quant_rows_kernel<FMT, GATHER, MULTI>;
     static size_t attr = 0;
     if (smem > 48 * 1024 && smem > attr) {
         cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
@@ -747,6 +811,8 @@ cudaError_t launch_quant(int fmt, bool gather, const QuantArgs& a, int rows_pad,
         return launch_nvfp4_token(a, rows_pad, num_sms, st);
     if (fmt == FMT_NVFP4) return gather ? launch_quant_fmt<FMT_NVFP4, true>(a, rows_pad, num_sms, st)
                                         : launch_quant_fmt<FMT_NVFP4, false>(a, rows_pad, num_sms, st);
+    if (fmt == FMT_MXFP4 && a.passes > 1)
+        return gather ? cudaErrorInvalidValue : launch_quant_fmt<FMT_MXFP4, false, true>(a, rows_pad, num_sms, st);
     if (fmt == FMT_MXFP4) return gather ? launch_quant_fmt<FMT_MXFP4, true>(a, rows_pad, num_sms, st)
                                         : launch_quant_fmt<FMT_MXFP4, false>(a, rows_pad, num_sms, st);
     return gather ? launch_quant_fmt<FMT_INT4, true>(a, rows_pad, num_sms, st)

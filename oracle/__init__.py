@@ -69,6 +69,10 @@ def _declare(L):
                                        C.c_int, C.c_int, C.c_int, _u16p, _f64p, _f64p]
     L.orc_quant_mxfp4.argtypes = [_u16p, C.c_int, C.c_int, C.c_int, _u8p, _u8p]
     L.orc_quant_mxfp4_msd.argtypes = [_u16p, C.c_int, C.c_int, C.c_int, C.c_int, _u8p, _u8p]
+    L.orc_rotate_blocks.argtypes = [_u16p, C.c_int, C.c_int, C.c_int, C.c_int, C.c_int, _f32p]
+    L.orc_quant_nvfp4_f32.argtypes = [_f32p, C.c_int, C.c_int, C.c_int, _u8p, _u8p, _f32p]
+    L.orc_quant_mxfp4_f32.argtypes = [_f32p, C.c_int, C.c_int, _u8p, _u8p]
+    L.orc_quant_int4_f32.argtypes = [_f32p, C.c_int, C.c_int, _u8p, _f32p]
     L.orc_quant_int4.argtypes = [_u16p, C.c_int, C.c_int, C.c_int, _u8p, _f32p]
     L.orc_dequant_nvfp4.argtypes = [_u8p, _u8p, _f32p, C.c_int, C.c_int, C.c_int, _f64p]
     L.orc_dequant_mxfp4.argtypes = [_u8p, _u8p, C.c_int, C.c_int, _f64p]
@@ -186,6 +190,45 @@ def quant_mxfp4_msd(X, passes=2):
     scales = np.zeros((M, passes * K // 32), np.uint8)
     _check(lib().orc_quant_mxfp4_msd(_p(X, _u16p), M, K, K, passes, _p(codes, _u8p), _p(scales, _u8p)),
            "quant_mxfp4_msd")
+    return codes, scales
+
+
+def rotate_blocks(X, n, act_side):
+    """Block-local Walsh-Hadamard rotation (FP32 butterflies) of bf16 X, blocks
+    of n along K; times 1/n on the activation side.  Returns float32 [M, K]."""
+    X = _bf16(X)
+    M, K = X.shape
+    out = np.zeros((M, K), np.float32)
+    _check(lib().orc_rotate_blocks(_p(X, _u16p), M, K, K, n, 1 if act_side else 0, _p(out, _f32p)), "rotate_blocks")
+    return out
+
+
+def quant_nvfp4_f32(Xf, mode=1):
+    Xf = np.ascontiguousarray(Xf, np.float32)
+    M, K = Xf.shape
+    codes = np.zeros((M, K // 2), np.uint8)
+    scales = np.zeros((M, K // 16), np.uint8)
+    s2 = np.zeros(max(M, 1) if mode == 1 else 1, np.float32)
+    _check(lib().orc_quant_nvfp4_f32(_p(Xf, _f32p), M, K, mode, _p(codes, _u8p), _p(scales, _u8p), _p(s2, _f32p)),
+           "quant_nvfp4_f32")
+    return codes, scales, s2
+
+
+def quant_mxfp4_f32(Xf):
+    Xf = np.ascontiguousarray(Xf, np.float32)
+    M, K = Xf.shape
+    codes = np.zeros((M, K // 2), np.uint8)
+    scales = np.zeros((M, K // 32), np.uint8)
+    _check(lib().orc_quant_mxfp4_f32(_p(Xf, _f32p), M, K, _p(codes, _u8p), _p(scales, _u8p)), "quant_mxfp4_f32")
+    return codes, scales
+
+
+def quant_int4_f32(Xf):
+    Xf = np.ascontiguousarray(Xf, np.float32)
+    M, K = Xf.shape
+    codes = np.zeros((M, K // 2), np.uint8)
+    scales = np.zeros((M, K // 128), np.float32)
+    _check(lib().orc_quant_int4_f32(_p(Xf, _f32p), M, K, _p(codes, _u8p), _p(scales, _f32p)), "quant_int4_f32")
     return codes, scales
 
 

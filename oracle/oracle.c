@@ -309,6 +309,80 @@ void orc_dequant_mxfp4(const uint8_t* codes, const uint8_t* scales, int M, int K
 }
 
 /* ======================================================================== */
+/* Block-local Walsh-Hadamard rotation                                      */
+/* ======================================================================== */
+
+/* In-place fast Walsh-Hadamard transform of n = 2^k FP32 values (Sylvester
+ * order, H[i][j] = (-1)^popcount(i & j)): stages h = 1, 2, 4, ..., n/2, each
+ * replacing every pair (v[j], v[j+h]) with j & h == 0 by (v[j] + v[j+h],
+ * v[j] - v[j+h]), rounded to FP32. */
+static void fwht_f32(float* v, int n) {
+    for (int h = 1; h < n; h *= 2)
+        for (int i = 0; i < n; i += 2 * h)
+            for (int j = i; j < i + h; ++j) {
+                const float a = v[j], b = v[j + h];
+                v[j] = a + b;
+                v[j + h] = a - b;
+            }
+}
+
+/* Rotation of each n-element block along K of X (bf16) before quantization
+ * (the block-local form of the Hadamard rotation the "Depth Registers Unlock
+ * W4A4 on SwiGLU" (mlsanity) abstract names as QuaRot; block-local so that
+ * block isolation, which the "APEX4..." page, para 2 (ARCQuant) says full
+ * rotations compromise, is kept).  act_side = 1 multiplies the transform by
+ * 1/n (an exact power of two), act_side = 0 leaves it unscaled, so that
+ * (X H/n)(W H)^T = X W^T.  out: FP32 [M][K]. */
+int orc_rotate_blocks(const uint16_t* X, int M, int K, int ldx, int n, int act_side, float* out) {
+    if (M < 0 || n < 2 || (n & (n - 1)) || K % n || ldx < K) return -1;
+    const float inv = 1.0f / (float)n;
+    for (int m = 0; m < M; ++m)
+        for (int b = 0; b < K / n; ++b) {
+            float* v = out + (size_t)m * K + (size_t)b * n;
+            for (int i = 0; i < n; ++i) v[i] = orc_bf16_to_f32(X[(size_t)m * ldx + (size_t)b * n + i]);
+            fwht_f32(v, n);
+            if (act_side)
+                for (int i = 0; i < n; ++i) v[i] = v[i] * inv;
+        }
+    return 0;
+}
+
+/* The quantizers on FP32 input (rotated values are not bf16): the same block
+ * rules as orc_quant_nvfp4 / orc_quant_mxfp4 / orc_quant_int4. */
+int orc_quant_nvfp4_f32(const float* X, int M, int K, int mode, uint8_t* codes, uint8_t* scales, float* s2) {
+    if (M < 0 || K % 16 || (mode != 0 && mode != 1)) return -1;
+    float tensor_s2 = 1.0f;
+    if (mode == 0) {
+        float amax = 0.0f;
+        for (size_t i = 0; i < (size_t)M * K; ++i) amax = fmaxf(amax, fabsf(X[i]));
+        tensor_s2 = orc_nvfp4_s2_from_amax(amax);
+        s2[0] = tensor_s2;
+    }
+    for (int m = 0; m < M; ++m) {
+        const float* row = X + (size_t)m * K;
+        float rs2 = tensor_s2;
+        if (mode == 1) {
+            float amax = 0.0f;
+            for (int k = 0; k < K; ++k) amax = fmaxf(amax, fabsf(row[k]));
+            rs2 = orc_nvfp4_s2_from_amax(amax);
+            s2[m] = rs2;
+        }
+        for (int b = 0; b < K / 16; ++b)
+            nvfp4_block(row + 16 * b, rs2, codes + (size_t)m * (K / 2) + 8 * b, scales + (size_t)m * (K / 16) + b);
+    }
+    return 0;
+}
+
+int orc_quant_mxfp4_f32(const float* X, int M, int K, uint8_t* codes, uint8_t* scales) {
+    if (M < 0 || K % 32) return -1;
+    for (int m = 0; m < M; ++m)
+        for (int b = 0; b < K / 32; ++b)
+            mxfp4_block(X + (size_t)m * K + 32 * b, codes + (size_t)m * (K / 2) + 16 * b,
+                        scales + (size_t)m * (K / 32) + b);
+    return 0;
+}
+
+/* ======================================================================== */
 /* INT4, group 128, symmetric round-to-nearest                              */
 /* ======================================================================== */
 
@@ -330,6 +404,15 @@ static void int4_group(const float* x, uint8_t* codes64 /* 64 bytes */, float* s
     for (int j = 0; j < 64; ++j)
         codes64[j] = (uint8_t)((q[2 * j] & 15) | ((q[2 * j + 1] & 15) << 4));
     *scale = s;
+}
+
+int orc_quant_int4_f32(const float* X, int M, int K, uint8_t* codes, float* scales) {
+    if (M < 0 || K % 128) return -1;
+    for (int m = 0; m < M; ++m)
+        for (int g = 0; g < K / 128; ++g)
+            int4_group(X + (size_t)m * K + 128 * g, codes + (size_t)m * (K / 2) + 64 * g,
+                       scales + (size_t)m * (K / 128) + g);
+    return 0;
 }
 
 int orc_quant_int4(const uint16_t* X, int M, int K, int ldx, uint8_t* codes, float* scales) {

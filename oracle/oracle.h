@@ -76,6 +76,18 @@ int orc_quant_mxfp4(const uint16_t* X, int M, int K, int ldx,
  * not exact (never, under the MXFP4 rule above).                           */
 int orc_quant_mxfp4_msd(const uint16_t* X, int M, int K, int ldx, int passes,
                         uint8_t* codes, uint8_t* scales);
+/* Block-local Walsh-Hadamard rotation of X (bf16 [M][ldx]) into FP32
+ * out[M][K]: each n-element block along K (n = 16, 32 or 128: the block of
+ * the format) is transformed by the fast Walsh-Hadamard butterflies in FP32
+ * (stages h = 1, 2, ..., n/2; (a, b) -> (a + b, a - b)), then multiplied by
+ * 1/n when act_side (activations), left unscaled otherwise (weights), so
+ * that (X H/n)(W H)^T = X W^T.                                             */
+int orc_rotate_blocks(const uint16_t* X, int M, int K, int ldx, int n, int act_side, float* out);
+/* The quantizers on FP32 input X[M][K] (rotated values), same rules.        */
+int orc_quant_nvfp4_f32(const float* X, int M, int K, int mode,
+                        uint8_t* codes, uint8_t* scales, float* s2);
+int orc_quant_mxfp4_f32(const float* X, int M, int K, uint8_t* codes, uint8_t* scales);
+int orc_quant_int4_f32(const float* X, int M, int K, uint8_t* codes, float* scales);
 /* codes [M][K/2] two's-complement nibbles, scales [M][K/128] FP32          */
 int orc_quant_int4(const uint16_t* X, int M, int K, int ldx,
                    uint8_t* codes, float* scales);

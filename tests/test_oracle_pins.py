@@ -500,3 +500,64 @@ def test_msd_two_passes_cut_the_error(orc):
     e1 = x - _mx_values(c1, s1, 1024)
     e2 = x - _mx_values(c2[:, :512], s2[:, :32], 1024) - _mx_values(c2[:, 512:], s2[:, 32:], 1024)
     assert np.sqrt((e2 ** 2).mean()) < np.sqrt((e1 ** 2).mean()) / 4
+
+
+# ---- block-local Walsh-Hadamard rotation ------------------------------------
+def _sylvester(n):
+    i = np.arange(n)
+    pc = np.vectorize(lambda v: bin(int(v)).count("1"))(i[:, None] & i[None, :])
+    return np.where(pc % 2 == 0, 1.0, -1.0)
+
+
+@pytest.mark.parametrize("n", [16, 32, 128])
+def test_rotation_of_unit_vectors_is_sylvester_hadamard(orc, n):
+    """Rows of the identity come out as the rows of H, H[i][j] = (-1)^popcount(i&j)
+    (closed form); the activation side is H/n."""
+    I = bf16(np.eye(n))
+    np.testing.assert_array_equal(orc.rotate_blocks(I, n, act_side=False), _sylvester(n))
+    np.testing.assert_array_equal(orc.rotate_blocks(I, n, act_side=True), _sylvester(n) / n)
+
+
+@pytest.mark.parametrize("n", [16, 32, 128])
+def test_rotation_exact_on_small_integers_and_cancels_in_the_product(orc, n):
+    """Small integers keep every butterfly exact, so the transform equals the
+    integer product X H (block by block), and (X H/n)(W H)^T = X W^T exactly."""
+    K = 2 * n
+    r = np.random.default_rng(61)
+    X = r.integers(-8, 9, size=(5, K)).astype(np.float64)
+    W = r.integers(-8, 9, size=(7, K)).astype(np.float64)
+    Hb = np.kron(np.eye(K // n), _sylvester(n))
+    Xa = orc.rotate_blocks(bf16(X), n, act_side=True).astype(np.float64)
+    Wr = orc.rotate_blocks(bf16(W), n, act_side=False).astype(np.float64)
+    np.testing.assert_array_equal(Xa, X @ Hb / n)
+    np.testing.assert_array_equal(Wr, W @ Hb)
+    np.testing.assert_array_equal(Xa @ Wr.T, X @ W.T)
+
+
+@pytest.mark.parametrize("n", [16, 32, 128])
+def test_rotation_rounding_within_the_butterfly_bound(orc, n):
+    """On general bf16 data each of the log2(n) stages rounds once: the FP32
+    result is within log2(n) * 2^-24 * (|X| |H|) of the exact product."""
+    K = 4 * n
+    spread = np.exp2(np.random.default_rng(62).integers(-14, 15, size=(8, K)))   # wide exponent range
+    Xb = bf16(synth.normal((8, K), 1.0, 62, 1) * spread)
+    x = synth.bf16_bits_to_f32(Xb).astype(np.float64)
+    Hb = np.kron(np.eye(K // n), _sylvester(n))
+    got = orc.rotate_blocks(Xb, n, act_side=False).astype(np.float64)
+    bound = np.log2(n) * 2.0 ** -24 * (np.abs(x) @ np.abs(Hb))
+    assert np.all(np.abs(got - x @ Hb) <= bound)
+    assert np.any(got != x @ Hb)  # the data really exercises rounding
+
+
+def test_fp32_quantizers_reduce_to_the_bf16_ones(orc):
+    """On bf16-valued FP32 input the FP32-input quantizers equal the pinned ones."""
+    Xb = synth.activations("llama2_70b", 9, 512, seed=63)
+    xf = synth.bf16_bits_to_f32(Xb)
+    for mode in (0, 1):
+        a, b = orc.quant_nvfp4_f32(xf, mode), orc.quant_nvfp4(Xb, mode=mode)
+        for u, v in zip(a, b):
+            np.testing.assert_array_equal(u, v)
+    for u, v in zip(orc.quant_mxfp4_f32(xf), orc.quant_mxfp4(Xb)):
+        np.testing.assert_array_equal(u, v)
+    for u, v in zip(orc.quant_int4_f32(xf), orc.quant_int4(Xb)):
+        np.testing.assert_array_equal(u.view(np.uint8), v.view(np.uint8))

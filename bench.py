@@ -521,6 +521,36 @@ def extra_rows(args, dev, stream, P):
                 "TFLOPS_effective_K": round(2.0 * M * N * K / (ms * 1e-3) / 1e12, 1), "us": round(ms * 1e3, 2)}
         del W1, W2, X, q, Y
 
+    # block-local Hadamard rotation, NVFP4 per token, Llama qkv shape: the
+    # rotating quantizer alone (L2 flushed) and the linear, beside the plain ones
+    if want("hadamard"):
+        K, N, M = 8192, 10240, args.tokens
+        Wd = to_dev(synth.weights("llama2_70b", N, K, tensor_id=100), dev)
+        Wp, Wr = w4.quantize_weight(Wd, w4.NVFP4), w4.quantize_weight(Wd, w4.NVFP4, hadamard=True)
+        del Wd
+        X = to_dev(synth.activations("llama2_70b", M, K, seed=8), dev)
+        fl = l2_flush_buffer(dev)
+        byts = 2 * M * K + M * K / 2 + M * K / 16 + 4 * M
+        for name, rot in (("plain", False), ("hadamard", True)):
+            q = w4.QTensor(w4.NVFP4, M, K, w4.SCALE_TOKEN, dev, w4.FLAG_HADAMARD if rot else 0)
+            f = lambda: w4.quantize_act(X, w4.NVFP4, w4.SCALE_TOKEN, out=q)
+            for _ in range(max(3, args.warmup)):
+                f()
+            ms = time_loop(f, it, stream, fl)
+            out[f"quant_nvfp4_token_{name}_llama_qkv_in"] = {"GB/s": round(byts / ms / 1e6, 1),
+                                                              "frac_hbm": round(byts / ms / 1e6 / hbm, 3),
+                                                              "us": round(ms * 1e3, 2)}
+        del fl
+        Y = torch.empty(M, N, dtype=torch.bfloat16, device=dev)
+        for name, Wq in (("plain", Wp), ("hadamard", Wr)):
+            fn = lambda: w4.linear(X, Wq, w4.SCALE_TOKEN, Y=Y)
+            for _ in range(max(3, args.warmup)):
+                fn()
+            ms = time_loop(fn, it, stream)
+            out[f"linear_nvfp4_{name}_llama_qkv_m{M}"] = {"TFLOPS": round(2.0 * M * N * K / (ms * 1e-3) / 1e12, 1),
+                                                          "us": round(ms * 1e3, 2)}
+        del Wp, Wr, X, Y
+
     if not want("mxfp4"):
         torch.cuda.synchronize()
         assert w4.device_status() == w4.OK
@@ -553,7 +583,7 @@ def main():
     ap.add_argument("--cpu-rows", type=int, default=8, help="cpu_baseline sample: tokens")
     ap.add_argument("--cpu-cols", type=int, default=4096, help="cpu_baseline sample: output columns")
     ap.add_argument("--no-rows", action="store_true", help="skip the secondary rows")
-    ap.add_argument("--only", choices=["gemm", "quant", "decode", "int4", "aug", "mxfp4", "segments", "msd"], default=None,
+    ap.add_argument("--only", choices=["gemm", "quant", "decode", "int4", "aug", "mxfp4", "segments", "msd", "hadamard"], default=None,
                     help="run only one secondary row (for profiling) and print it")
     ap.add_argument("--no-cpu", action="store_true", help="skip the oracle CPU baseline")
     ap.add_argument("--shape", default=None, help="--only gemm: one Llama linear (qkv, o, w1, w3, w2)")

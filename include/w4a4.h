@@ -66,6 +66,10 @@ extern "C" {
 #define W4A4_MXFP4 1   /* group 32 */
 #define W4A4_INT4  2   /* group 128 */
 
+/* w4a4_qtensor.flags */
+#define W4A4_FLAG_HADAMARD 1  /* each quantization block (16 / 32 / 128 elements along K) was
+                                 rotated by a Walsh-Hadamard matrix before quantization */
+
 /* NVFP4 second-level scale granularity */
 #define W4A4_SCALE_TENSOR 0  /* one FP32 scale for the whole tensor */
 #define W4A4_SCALE_TOKEN  1  /* one FP32 scale per row (per token) */
@@ -86,6 +90,23 @@ extern "C" {
  *
  * An "augmented" activation tensor has cols = K + nS: its first K columns
  * come from w4a4_quantize_act, the last nS from w4a4_augment_residual.
+ *
+ * W4A4_FLAG_HADAMARD (block-local rotation: the "Depth Registers Unlock W4A4
+ * on SwiGLU" (mlsanity) abstract names QuaRot's Hadamard rotations; the
+ * "APEX4..." page, para 2 (ARCQuant) notes that full rotations compromise
+ * block isolation, so here each quantization block is rotated on its own).
+ * When set on the output of a quantizer, each n-element block along K (n = 16
+ * NVFP4, 32 MXFP4, 128 INT4) is first transformed by the fast Walsh-Hadamard
+ * butterflies in FP32 (stages h = 1, 2, ..., n/2, (a, b) -> (a + b, a - b),
+ * Sylvester order), then quantized by the format's rule (NVFP4 amaxes, per
+ * token or per tensor, are those of the rotated values).  Activations
+ * (w4a4_quantize_act, w4a4_linear) are also multiplied by 1/n; weights
+ * (w4a4_quantize_weight, w4a4_quantize_weight_segments) are not, so that the
+ * product of a rotated activation and a rotated weight is X W^T unchanged
+ * (H H^T = n I): the GEMM needs no change.  w4a4_gemm requires both operands
+ * to carry the same flag; w4a4_linear rotates the activations when Wq
+ * carries it.  Not combined with residual channels (nS > 0) nor with the
+ * multi-pass decomposition (those calls return W4A4_ERR_INVALID_ARG).
  */
 typedef struct w4a4_qtensor {
     int32_t format;      /* W4A4_NVFP4 / W4A4_MXFP4 / W4A4_INT4 */
@@ -93,7 +114,7 @@ typedef struct w4a4_qtensor {
     int32_t cols;
     int32_t group;       /* 16 / 32 / 128, must match format */
     int32_t scale_mode;  /* NVFP4: W4A4_SCALE_TENSOR or W4A4_SCALE_TOKEN; else ignored */
-    int32_t reserved;    /* must be 0 */
+    int32_t flags;       /* 0, or W4A4_FLAG_HADAMARD (see below); other bits must be 0 */
     void*   codes;       /* device */
     void*   scales;      /* device */
     float*  s2;          /* device, NVFP4 only (else may be NULL) */

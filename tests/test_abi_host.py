@@ -163,3 +163,24 @@ def test_msd_arguments(L):
                              None) == w4.ERR_INVALID_ARG
     assert L.w4a4_linear_msd(X, 4, 256, 256, C.byref(W), 2, C.c_void_p(16), 256, C.c_void_p(256), 16,
                              None) == w4.ERR_WORKSPACE
+
+
+def test_hadamard_flag_arguments(L):
+    """The rotation flag: unknown bits rejected; operands must agree; no
+    rotation with residual channels or the multi-pass decomposition."""
+    X = C.c_void_p(16)
+    bad = _qt(w4.NVFP4, 4, 256, w4.SCALE_TOKEN)
+    bad.flags = 2
+    assert L.w4a4_quantize_act(X, 4, 256, 256, 0, 16, 1, None, C.byref(bad), None) == w4.ERR_INVALID_ARG
+    a = _qt(w4.NVFP4, 4, 256, w4.SCALE_TOKEN)
+    a.flags = w4.FLAG_HADAMARD
+    b = _qt(w4.NVFP4, 256, 256, w4.SCALE_TENSOR)
+    assert L.w4a4_gemm(C.byref(a), C.byref(b), C.c_void_p(16), 256, None) == w4.ERR_INVALID_ARG
+    Wr = _qt(w4.NVFP4, 256, 384, w4.SCALE_TENSOR)
+    Wr.flags = w4.FLAG_HADAMARD
+    assert L.w4a4_quantize_weight(X, 256, 256, 256, 0, 16, C.c_void_p(16), 128, C.byref(Wr), None) == w4.ERR_INVALID_ARG
+    assert L.w4a4_linear(X, 4, 256, 256, C.byref(Wr), 1, C.c_void_p(16), 128, C.c_void_p(16), 256,
+                         C.c_void_p(256), 1 << 20, None) == w4.ERR_INVALID_ARG
+    m = _qt(w4.MXFP4, 4, 512)
+    m.flags = w4.FLAG_HADAMARD
+    assert L.w4a4_quantize_act_msd(X, 4, 256, 256, 2, C.byref(m), None) == w4.ERR_INVALID_ARG

@@ -19,6 +19,7 @@ LIB_PATH = os.path.join(HERE, "lib", "libw4a4.so")
 NVFP4, MXFP4, INT4 = 0, 1, 2
 GROUP = {NVFP4: 16, MXFP4: 32, INT4: 128}
 SCALE_TENSOR, SCALE_TOKEN = 0, 1
+FLAG_HADAMARD = 1  # blocks rotated by a Walsh-Hadamard matrix before quantization
 
 OK, ERR_INVALID_ARG, ERR_MISALIGNED, ERR_WORKSPACE, ERR_ARCH, ERR_CUDA, ERR_DEVICE_TIMEOUT = range(7)
 
@@ -38,7 +39,7 @@ class W4A4Error(RuntimeError):
 
 class QTensorStruct(C.Structure):
     _fields_ = [("format", C.c_int32), ("rows", C.c_int32), ("cols", C.c_int32), ("group", C.c_int32),
-                ("scale_mode", C.c_int32), ("reserved", C.c_int32), ("codes", C.c_void_p),
+                ("scale_mode", C.c_int32), ("flags", C.c_int32), ("codes", C.c_void_p),
                 ("scales", C.c_void_p), ("s2", C.c_void_p)]
 
 
@@ -111,14 +112,14 @@ def qtensor_bytes(fmt: int, rows: int, cols: int, scale_mode: int = SCALE_TENSOR
 class QTensor:
     """A quantized tensor whose buffers are torch uint8/float32 device tensors."""
 
-    def __init__(self, fmt: int, rows: int, cols: int, scale_mode: int = SCALE_TENSOR, device="cuda"):
+    def __init__(self, fmt: int, rows: int, cols: int, scale_mode: int = SCALE_TENSOR, device="cuda", flags: int = 0):
         import torch
         cb, sb, tb = qtensor_bytes(fmt, rows, cols, scale_mode)
-        self.format, self.rows, self.cols, self.scale_mode = fmt, rows, cols, scale_mode
+        self.format, self.rows, self.cols, self.scale_mode, self.flags = fmt, rows, cols, scale_mode, flags
         self.codes = torch.zeros(max(cb, 16), dtype=torch.uint8, device=device)
         self.scales = torch.zeros(max(sb, 16), dtype=torch.uint8, device=device)
         self.s2 = torch.zeros(max(tb // 4, 4), dtype=torch.float32, device=device) if tb else None
-        self.struct = QTensorStruct(fmt, rows, cols, GROUP[fmt], scale_mode if fmt == NVFP4 else 0, 0,
+        self.struct = QTensorStruct(fmt, rows, cols, GROUP[fmt], scale_mode if fmt == NVFP4 else 0, flags,
                                     self.codes.data_ptr(), self.scales.data_ptr(),
                                     self.s2.data_ptr() if self.s2 is not None else None)
 
@@ -128,28 +129,31 @@ class QTensor:
 
 
 def quantize_act(X, fmt: int, scale_mode: int = SCALE_TOKEN, static_s2=None, out: QTensor | None = None,
-                 cols: int | None = None) -> QTensor:
-    """X: bf16 [M, K] CUDA tensor (row stride may exceed K)."""
+                 cols: int | None = None, hadamard: bool = False) -> QTensor:
+    """X: bf16 [M, K] CUDA tensor (row stride may exceed K).  hadamard: rotate
+    each quantization block first (activation side, times 1/block)."""
     M, K = X.shape
     if out is None:
-        out = QTensor(fmt, M, cols or K, scale_mode if fmt == NVFP4 else SCALE_TENSOR, X.device)
+        out = QTensor(fmt, M, cols or K, scale_mode if fmt == NVFP4 else SCALE_TENSOR, X.device,
+                      FLAG_HADAMARD if hadamard else 0)
     _check(lib().w4a4_quantize_act(_ptr(X), M, K, X.stride(0), fmt, GROUP[fmt], scale_mode, _ptr(static_s2),
                                    out.ref, _stream()), "w4a4_quantize_act")
     return out
 
 
-def quantize_weight(W, fmt: int, S=None, out: QTensor | None = None) -> QTensor:
-    """W: bf16 [N, K]; S: optional int32 CUDA tensor of augmented channels."""
+def quantize_weight(W, fmt: int, S=None, out: QTensor | None = None, hadamard: bool = False) -> QTensor:
+    """W: bf16 [N, K]; S: optional int32 CUDA tensor of augmented channels;
+    hadamard: rotate each quantization block first (weight side, unscaled)."""
     N, K = W.shape
     nS = 0 if S is None else S.numel()
     if out is None:
-        out = QTensor(fmt, N, K + nS, SCALE_TENSOR, W.device)
+        out = QTensor(fmt, N, K + nS, SCALE_TENSOR, W.device, FLAG_HADAMARD if hadamard else 0)
     _check(lib().w4a4_quantize_weight(_ptr(W), N, K, W.stride(0), fmt, GROUP[fmt], _ptr(S), nS, out.ref,
                                       _stream()), "w4a4_quantize_weight")
     return out
 
 
-def quantize_weight_segments(W, seg, S=None, out: QTensor | None = None) -> QTensor:
+def quantize_weight_segments(W, seg, S=None, out: QTensor | None = None, hadamard: bool = False) -> QTensor:
     """NVFP4 weights of a fused module, one global scale per row segment.
 
     W: bf16 [N, K]; seg: host sequence of N-row boundaries [0, ..., N], each a
@@ -160,7 +164,7 @@ def quantize_weight_segments(W, seg, S=None, out: QTensor | None = None) -> QTen
     nS = 0 if S is None else S.numel()
     seg = [int(v) for v in seg]
     if out is None:
-        out = QTensor(NVFP4, N, K + nS, SCALE_TOKEN, W.device)
+        out = QTensor(NVFP4, N, K + nS, SCALE_TOKEN, W.device, FLAG_HADAMARD if hadamard else 0)
     arr = (C.c_int32 * len(seg))(*seg)
     _check(lib().w4a4_quantize_weight_segments(_ptr(W), N, K, W.stride(0), arr, len(seg) - 1, _ptr(S), nS,
                                                out.ref, _stream()), "w4a4_quantize_weight_segments")

@@ -112,7 +112,7 @@ int make_map_sf_rep(CUtensorMap* map, const void* base, int row_tiles, int col_a
 
 int check_qtensor(const w4a4_qtensor* q) {
     if (!q || !q->codes || !q->scales) return W4A4_ERR_INVALID_ARG;
-    if (q->format < 0 || q->format > 2 || q->group != group_of(q->format) || q->reserved != 0)
+    if (q->format < 0 || q->format > 2 || q->group != group_of(q->format) || (q->flags & ~W4A4_FLAG_HADAMARD))
         return W4A4_ERR_INVALID_ARG;
     if (q->rows < 0 || q->cols < 128 || q->cols % 128 || q->cols > kMaxPasses * kMaxK) return W4A4_ERR_INVALID_ARG;
     if (q->format == W4A4_NVFP4) {
@@ -131,9 +131,10 @@ int cuda_status(cudaError_t e) { return e == cudaSuccess ? W4A4_OK : W4A4_ERR_CU
 // Quantize rows [0, M) of X into the first K columns of q (q->cols >= K).
 int quantize_rows(const uint16_t* X, int M, int K, int ldx, const int32_t* S, int K_src, const float* static_s2,
                   w4a4_qtensor* q, int num_sms, cudaStream_t st, int* zero_words = nullptr, int zero_count = 0,
-                  int passes = 1) {
+                  int passes = 1, bool weight_side = false) {
     QuantArgs a{};
     a.passes = passes;
+    a.rot = (q->flags & W4A4_FLAG_HADAMARD) ? (weight_side ? 2 : 1) : 0;
     a.zero_words = zero_words;
     a.zero_count = zero_count;
     a.X = X;
@@ -155,7 +156,7 @@ int quantize_rows(const uint16_t* X, int M, int K, int ldx, const int32_t* S, in
     if (q->format == W4A4_NVFP4 && q->scale_mode == W4A4_SCALE_TENSOR && !static_s2) {
         // dynamic tensor scale: amax pass into s2[1], then the quantizer reads it
         cudaError_t e = cudaMemsetAsync(q->s2 + 1, 0, sizeof(float), st);
-        if (e == cudaSuccess) e = launch_amax(X, M, K_src, ldx, q->s2 + 1, num_sms, st);
+        if (e == cudaSuccess) e = launch_amax(X, M, K_src, ldx, q->s2 + 1, num_sms, st, a.rot);
         if (e != cudaSuccess) return W4A4_ERR_CUDA;
         a.tensor_amax = q->s2 + 1;
     }
@@ -345,13 +346,15 @@ int w4a4_quantize_weight(const uint16_t* W, int N, int K, int ldw, int format, i
     if (rc != W4A4_OK) return rc;
     if (out->format != format || out->rows != N || out->cols != K + nS) return W4A4_ERR_INVALID_ARG;
     if (format == W4A4_NVFP4 && out->scale_mode != W4A4_SCALE_TENSOR) return W4A4_ERR_INVALID_ARG;
+    if (nS && out->flags) return W4A4_ERR_INVALID_ARG;
     if (N == 0) return W4A4_OK;
     if (!W) return W4A4_ERR_INVALID_ARG;
     if (!aligned16(W) || ldw % 8) return W4A4_ERR_MISALIGNED;
     int sms = 0;
     rc = device_check(&sms);
     if (rc != W4A4_OK) return rc;
-    return quantize_rows(W, N, K + nS, ldw, nS ? S : nullptr, K, nullptr, out, sms, as_stream(stream));
+    return quantize_rows(W, N, K + nS, ldw, nS ? S : nullptr, K, nullptr, out, sms, as_stream(stream), nullptr, 0, 1,
+                         true);
 }
 
 int w4a4_quantize_weight_segments(const uint16_t* W, int N, int K, int ldw, const int32_t* seg, int nseg,
@@ -366,6 +369,7 @@ int w4a4_quantize_weight_segments(const uint16_t* W, int N, int K, int ldw, cons
     if (rc != W4A4_OK) return rc;
     if (out->format != W4A4_NVFP4 || out->scale_mode != W4A4_SCALE_TOKEN || out->rows != N || out->cols != K + nS)
         return W4A4_ERR_INVALID_ARG;
+    if (nS && out->flags) return W4A4_ERR_INVALID_ARG;
     rc = check_weight_s2(out);
     if (rc != W4A4_OK) return rc;
     if (!W) return W4A4_ERR_INVALID_ARG;
@@ -385,7 +389,8 @@ int w4a4_quantize_weight_segments(const uint16_t* W, int N, int K, int ldw, cons
         q.codes = static_cast<uint8_t*>(out->codes) + (size_t)r0 * (cols / 2);
         q.scales = static_cast<uint8_t*>(out->scales) + (size_t)(r0 / 128) * (cols / 16 / 4) * 512;
         q.s2 = out->s2 + r0;
-        rc = quantize_rows(W + (size_t)r0 * ldw, rows, cols, ldw, nS ? S : nullptr, K, nullptr, &q, sms, st);
+        rc = quantize_rows(W + (size_t)r0 * ldw, rows, cols, ldw, nS ? S : nullptr, K, nullptr, &q, sms, st, nullptr, 0,
+                           1, true);
         if (rc != W4A4_OK) return rc;
         if (launch_spread_first(q.s2, rows, st) != cudaSuccess) return W4A4_ERR_CUDA;
     }
@@ -397,7 +402,8 @@ int w4a4_quantize_act_msd(const uint16_t* X, int M, int K, int ldx, int passes, 
         return W4A4_ERR_INVALID_ARG;
     int rc = check_qtensor(out);
     if (rc != W4A4_OK) return rc;
-    if (out->format != W4A4_MXFP4 || out->rows != M || out->cols != passes * K) return W4A4_ERR_INVALID_ARG;
+    if (out->format != W4A4_MXFP4 || out->rows != M || out->cols != passes * K || out->flags)
+        return W4A4_ERR_INVALID_ARG;
     if (M == 0) return W4A4_OK;
     if (!X) return W4A4_ERR_INVALID_ARG;
     if (!aligned16(X) || ldx % 8) return W4A4_ERR_MISALIGNED;
@@ -415,7 +421,8 @@ int w4a4_quantize_weight_msd(const uint16_t* W, int N, int K, int ldw, int passe
         return W4A4_ERR_INVALID_ARG;
     int rc = check_qtensor(out);
     if (rc != W4A4_OK) return rc;
-    if (out->format != W4A4_MXFP4 || out->rows != N || out->cols != passes * K) return W4A4_ERR_INVALID_ARG;
+    if (out->format != W4A4_MXFP4 || out->rows != N || out->cols != passes * K || out->flags)
+        return W4A4_ERR_INVALID_ARG;
     if (N == 0) return W4A4_OK;
     if (!W) return W4A4_ERR_INVALID_ARG;
     if (!aligned16(W) || ldw % 8) return W4A4_ERR_MISALIGNED;
@@ -443,7 +450,8 @@ int w4a4_gemm(const w4a4_qtensor* A, const w4a4_qtensor* B, uint16_t* Y, int ldy
     int rc = check_qtensor(A);
     if (rc == W4A4_OK) rc = check_qtensor(B);
     if (rc != W4A4_OK) return rc;
-    if (A->format != B->format || A->cols != B->cols || B->rows < 128 || B->rows % 128 || ldy < B->rows)
+    if (A->format != B->format || A->cols != B->cols || B->rows < 128 || B->rows % 128 || ldy < B->rows ||
+        A->flags != B->flags)
         return W4A4_ERR_INVALID_ARG;
     rc = check_weight_s2(B);
     if (rc != W4A4_OK) return rc;
@@ -470,7 +478,7 @@ int w4a4_linear(const uint16_t* X, int M, int K, int ldx, const w4a4_qtensor* Wq
     if (M < 0 || K < 128 || K % 128 || K > kMaxK || ldx < K) return W4A4_ERR_INVALID_ARG;
     rc = check_S_args(S, nS, K);
     if (rc != W4A4_OK) return rc;
-    if (nS && fmt != W4A4_NVFP4) return W4A4_ERR_INVALID_ARG;
+    if (nS && (fmt != W4A4_NVFP4 || Wq->flags)) return W4A4_ERR_INVALID_ARG;
     if (Wq->cols != K + nS || Wq->rows < 128 || Wq->rows % 128 || ldy < Wq->rows) return W4A4_ERR_INVALID_ARG;
     if (fmt == W4A4_NVFP4 && scale_mode != W4A4_SCALE_TENSOR && scale_mode != W4A4_SCALE_TOKEN)
         return W4A4_ERR_INVALID_ARG;
@@ -494,6 +502,7 @@ int w4a4_linear(const uint16_t* X, int M, int K, int ldx, const w4a4_qtensor* Wq
     xq.cols = K + nS;
     xq.group = group_of(fmt);
     xq.scale_mode = fmt == W4A4_NVFP4 ? scale_mode : 0;
+    xq.flags = Wq->flags;  // rotated weights: rotate the activations the same way
     xq.codes = base + L.codes;
     xq.scales = base + L.scales;
     xq.s2 = reinterpret_cast<float*>(base + L.s2);
@@ -517,7 +526,8 @@ int w4a4_linear_msd(const uint16_t* X, int M, int K, int ldx, const w4a4_qtensor
     if (rc != W4A4_OK) return rc;
     if (M < 0 || K < 128 || K % 128 || K > kMaxK || ldx < K || passes < 1 || passes > kMaxPasses)
         return W4A4_ERR_INVALID_ARG;
-    if (Wq->format != W4A4_MXFP4 || Wq->cols != passes * K || Wq->rows < 128 || Wq->rows % 128 || ldy < Wq->rows)
+    if (Wq->format != W4A4_MXFP4 || Wq->cols != passes * K || Wq->rows < 128 || Wq->rows % 128 || ldy < Wq->rows ||
+        Wq->flags)
         return W4A4_ERR_INVALID_ARG;
     if (M == 0) return W4A4_OK;
     if (!X || !Y) return W4A4_ERR_INVALID_ARG;
@@ -554,7 +564,8 @@ int w4a4_augment_residual(const uint16_t* X, int M, int K, int ldx, const int32_
     int rc = check_S_args(S, nS, K);
     if (rc == W4A4_OK) rc = check_qtensor(Xaug);
     if (rc != W4A4_OK) return rc;
-    if (Xaug->format != W4A4_NVFP4 || Xaug->rows != M || Xaug->cols != K + nS) return W4A4_ERR_INVALID_ARG;
+    if (Xaug->format != W4A4_NVFP4 || Xaug->rows != M || Xaug->cols != K + nS || Xaug->flags)
+        return W4A4_ERR_INVALID_ARG;
     if (M == 0) return W4A4_OK;
     if (!X) return W4A4_ERR_INVALID_ARG;
     if (!aligned16(X) || ldx % 8) return W4A4_ERR_MISALIGNED;

@@ -31,6 +31,8 @@ struct QuantArgs {
     int zero_count;
     int passes;                // MXFP4: 1, or more for the multi-pass decomposition (pass p
                                // in columns [p*K, (p+1)*K) of codes and scales)
+    int rot;                   // block-local Walsh-Hadamard rotation: 0 none, 1 activation
+                               // side (times 1/block), 2 weight side (unscaled)
 };
 
 struct ResidualArgs {
@@ -67,7 +69,9 @@ struct GemmArgs {
 };
 
 cudaError_t launch_quant(int fmt, bool gather, const QuantArgs& a, int rows_pad, int num_sms, cudaStream_t st);
-cudaError_t launch_amax(const uint16_t* X, int M, int K, int ldx, float* out, int num_sms, cudaStream_t st);
+// rot: 0 plain amax; 1 / 2 amax of the rotated 16-element blocks (activation / weight side)
+cudaError_t launch_amax(const uint16_t* X, int M, int K, int ldx, float* out, int num_sms, cudaStream_t st,
+                        int rot = 0);
 cudaError_t launch_residual(const ResidualArgs& a, cudaStream_t st);
 // p[1 .. n) = p[0] (device floats)
 cudaError_t launch_spread_first(float* p, int n, cudaStream_t st);

@@ -139,6 +139,90 @@ __device__ __forceinline__ uint32_t int4x8_exact(uint4 v, float s) {
     return out;
 }
 
+// The same encoders on FP32 inputs (rotated values): negated dividends are the
+// inputs with the sign bit flipped.
+__device__ __forceinline__ uint32_t neg_f(float v) { return __float_as_uint(v) ^ 0x80000000u; }
+__device__ __forceinline__ uint32_t e2m1x8_fast_f(const float* v, uint64_t ny2, uint64_t d2) {
+    float q[8];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) div2_refined(neg_f(v[2 * e]), neg_f(v[2 * e + 1]), ny2, d2, q[2 * e], q[2 * e + 1]);
+    return e2m1x8(q);
+}
+__device__ __forceinline__ uint32_t e2m1x8_exact_f(const float* v, float d) {
+    float q[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) q[e] = __fdiv_rn(v[e], d);
+    return e2m1x8(q);
+}
+__device__ __forceinline__ uint32_t int4x8_fast_f(const float* v, uint64_t ny2, uint64_t d2) {
+    constexpr float kMagic = 12582912.0f;  // 1.5 * 2^23
+    uint32_t out = 0;
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+        float q0, q1;
+        div2_refined(neg_f(v[2 * e]), neg_f(v[2 * e + 1]), ny2, d2, q0, q1);
+        const uint32_t n0 = __float_as_uint(__fadd_rn(q0, kMagic)) & 15u;
+        const uint32_t n1 = __float_as_uint(__fadd_rn(q1, kMagic)) & 15u;
+        out |= (n0 | (n1 << 4)) << (8 * e);
+    }
+    return out;
+}
+__device__ __forceinline__ uint32_t int4x8_exact_f(const float* v, float s) {
+    uint32_t out = 0;
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+        const int n0 = min(max(__float2int_rn(__fdiv_rn(v[2 * e], s)), -8), 7);
+        const int n1 = min(max(__float2int_rn(__fdiv_rn(v[2 * e + 1], s)), -8), 7);
+        out |= (uint32_t)((n0 & 15) | ((n1 & 15) << 4)) << (8 * e);
+    }
+    return out;
+}
+
+// Block-local Walsh-Hadamard rotation of one item (16 consecutive elements of
+// an N-element block; the block's items sit on N/16 consecutive lanes, the
+// item's place in its block is c mod N/16).  Fast Walsh-Hadamard butterflies
+// in FP32, stages h = 1, 2, ..., N/2, (a, b) -> (a + b, a - b): stages below
+// 16 inside the thread, the others with the lane holding the partner items.
+// The activation side then multiplies by 1/N (exact), the weight side keeps
+// the transform unscaled, so (X H/N)(W H)^T = X W^T.  Every lane of the warp
+// must call it (the shuffles use the full mask).
+template <int N>
+__device__ __forceinline__ void rotate_item(const uint32_t* w, float* v, int c, bool act) {
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+        v[2 * e] = bf16lo(w[e]);
+        v[2 * e + 1] = bf16hi(w[e]);
+    }
+#pragma unroll
+    for (int h = 1; h < 16; h *= 2)
+#pragma unroll
+        for (int e = 0; e < 16; ++e)
+            if (!(e & h)) {
+                const float x = v[e], y = v[e + h];
+                v[e] = __fadd_rn(x, y);
+                v[e + h] = __fsub_rn(x, y);
+            }
+#pragma unroll
+    for (int st = 0; (16 << st) < N; ++st) {
+        const bool upper = (c >> st) & 1;
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {
+            const float p = __shfl_xor_sync(0xffffffffu, v[e], 1 << st);
+            v[e] = upper ? __fsub_rn(p, v[e]) : __fadd_rn(v[e], p);
+        }
+    }
+    if (act) {
+#pragma unroll
+        for (int e = 0; e < 16; ++e) v[e] = __fmul_rn(v[e], 1.0f / N);
+    }
+}
+__device__ __forceinline__ float absmax16(const float* v) {
+    float m = 0.0f;
+#pragma unroll
+    for (int e = 0; e < 16; ++e) m = fmaxf(m, fabsf(v[e]));
+    return m;
+}
+
 __device__ __forceinline__ uint8_t e4m3_rn_sat(float t) {
     return (uint8_t)__nv_cvt_float_to_fp8(t, __NV_SATFINITE, __NV_E4M3);
 }
@@ -204,9 +288,12 @@ struct RowConsts {
     int pad;
 };
 
-// MULTI (MXFP4 only): the multi-pass decomposition, a.passes passes.
-template <int FMT, bool GATHER, bool MULTI = false>
+// MULTI (MXFP4 only): the multi-pass decomposition, a.passes passes.  ROT:
+// every block rotated first (rotate_item; a.rot 1 = activation side, 2 =
+// weight side).
+template <int FMT, bool GATHER, bool MULTI = false, bool ROT = false>
 __global__ void __launch_bounds__(256, 4) quant_rows_kernel(QuantArgs a, int rows_per_cta, int nbuf) {
+    constexpr int NB = FMT == FMT_NVFP4 ? 16 : FMT == FMT_MXFP4 ? 32 : 128;  // block (rotation) size
     pdl_launch_dependents();
     pdl_wait();  // X and the words to clear may belong to the preceding launch
     if (blockIdx.x == 0)
@@ -266,7 +353,14 @@ __global__ void __launch_bounds__(256, 4) quant_rows_kernel(QuantArgs a, int row
             const uint4* p = reinterpret_cast<const uint4*>(rows + (size_t)i * row_bytes) + 2 * c;
             const uint4 v0 = p[0], v1 = p[1];
             const uint32_t w[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
-            float m = bmax16(w);
+            float m;
+            if constexpr (ROT) {  // NVFP4 blocks are single items: no lane exchange here
+                float v[16];
+                rotate_item<16>(w, v, c, a.rot == 1);
+                m = absmax16(v);
+            } else {
+                m = bmax16(w);
+            }
             bm[it] = m;  // reused by the quantization pass
             // items of one row are consecutive: reduce over the 8-lane group first
             m = fmaxf(m, __shfl_xor_sync(__activemask(), m, 1));
@@ -322,7 +416,11 @@ __global__ void __launch_bounds__(256, 4) quant_rows_kernel(QuantArgs a, int row
 #pragma unroll
             for (int e = 0; e < 8; ++e) w[e] = 0;
         }
-        float bmax = (token && live) ? bm[it] : bmax16(w);
+        float v[16];  // ROT: the rotated values of the item
+        if constexpr (ROT) rotate_item<NB>(w, v, c, a.rot == 1);
+        float bmax;
+        if constexpr (ROT) bmax = (token && live) ? bm[it] : absmax16(v);
+        else bmax = (token && live) ? bm[it] : bmax16(w);
 
         uint32_t w0 = 0, w1 = 0;  // 16 codes
         if constexpr (FMT == FMT_NVFP4) {
@@ -333,8 +431,13 @@ __global__ void __launch_bounds__(256, 4) quant_rows_kernel(QuantArgs a, int row
             const uint8_t sb = live ? e4m3_rn_sat(div_refined(u, k.s2, k.rinv)) : 0;
             const float d = sb ? __fmul_rn(e4m3_value(sb), k.s2) : 1.0f;
             const float y = __frcp_rn(d);
-            w0 = e2m1x8_fast(w, pack2(-y), pack2(d));
-            w1 = e2m1x8_fast(w + 4, pack2(-y), pack2(d));
+            if constexpr (ROT) {
+                w0 = e2m1x8_fast_f(v, pack2(-y), pack2(d));
+                w1 = e2m1x8_fast_f(v + 8, pack2(-y), pack2(d));
+            } else {
+                w0 = e2m1x8_fast(w, pack2(-y), pack2(d));
+                w1 = e2m1x8_fast(w + 4, pack2(-y), pack2(d));
+            }
             const bool slow = live && !(k.fast && bmax >= 0x1p-100f && d >= 0x1p-100f && d <= 0x1p100f &&
                                         __fmul_rn(bmax, y) <= 0x1p60f);
             uint8_t sbf = sb;
@@ -342,8 +445,13 @@ __global__ void __launch_bounds__(256, 4) quant_rows_kernel(QuantArgs a, int row
                 if (slow) {
                     sbf = e4m3_rn_sat(__fdiv_rn(__fdiv_rn(bmax, 6.0f), k.s2));
                     const float de = __fmul_rn(e4m3_value(sbf), k.s2);
-                    w0 = sbf ? e2m1x8_exact(make_uint4(w[0], w[1], w[2], w[3]), de) : 0u;
-                    w1 = sbf ? e2m1x8_exact(make_uint4(w[4], w[5], w[6], w[7]), de) : 0u;
+                    if constexpr (ROT) {
+                        w0 = sbf ? e2m1x8_exact_f(v, de) : 0u;
+                        w1 = sbf ? e2m1x8_exact_f(v + 8, de) : 0u;
+                    } else {
+                        w0 = sbf ? e2m1x8_exact(make_uint4(w[0], w[1], w[2], w[3]), de) : 0u;
+                        w1 = sbf ? e2m1x8_exact(make_uint4(w[4], w[5], w[6], w[7]), de) : 0u;
+                    }
                 }
             }
             if (sbf == 0) {
@@ -367,6 +475,13 @@ __global__ void __launch_bounds__(256, 4) quant_rows_kernel(QuantArgs a, int row
                 float q0[8], q1[8];
 #pragma unroll
                 for (int e2 = 0; e2 < 4; ++e2) {
+                    if constexpr (ROT) {
+                        q0[2 * e2] = __fmul_rn(v[2 * e2], inv);
+                        q0[2 * e2 + 1] = __fmul_rn(v[2 * e2 + 1], inv);
+                        q1[2 * e2] = __fmul_rn(v[8 + 2 * e2], inv);
+                        q1[2 * e2 + 1] = __fmul_rn(v[9 + 2 * e2], inv);
+                        continue;
+                    }
                     q0[2 * e2] = __fmul_rn(bf16lo(w[e2]), inv);
                     q0[2 * e2 + 1] = __fmul_rn(bf16hi(w[e2]), inv);
                     q1[2 * e2] = __fmul_rn(bf16lo(w[4 + e2]), inv);
@@ -434,14 +549,24 @@ __global__ void __launch_bounds__(256, 4) quant_rows_kernel(QuantArgs a, int row
             const bool fast = bmax >= 0x1p-100f && bmax <= 0x1p100f;
             float sc = live ? div_refined(bmax, 7.0f, 0x1.24924ap-3f) : 0.0f;  // RN(1/7)
             const float y = __frcp_rn(sc > 0.0f ? sc : 1.0f);
-            w0 = int4x8_fast(w, pack2(-y), pack2(sc));
-            w1 = int4x8_fast(w + 4, pack2(-y), pack2(sc));
+            if constexpr (ROT) {
+                w0 = int4x8_fast_f(v, pack2(-y), pack2(sc));
+                w1 = int4x8_fast_f(v + 8, pack2(-y), pack2(sc));
+            } else {
+                w0 = int4x8_fast(w, pack2(-y), pack2(sc));
+                w1 = int4x8_fast(w + 4, pack2(-y), pack2(sc));
+            }
             const bool slow = live && !fast;
             if (__any_sync(0xffffffffu, slow)) {
                 if (slow) {
                     sc = __fdiv_rn(bmax, 7.0f);
-                    w0 = sc != 0.0f ? int4x8_exact(make_uint4(w[0], w[1], w[2], w[3]), sc) : 0u;
-                    w1 = sc != 0.0f ? int4x8_exact(make_uint4(w[4], w[5], w[6], w[7]), sc) : 0u;
+                    if constexpr (ROT) {
+                        w0 = sc != 0.0f ? int4x8_exact_f(v, sc) : 0u;
+                        w1 = sc != 0.0f ? int4x8_exact_f(v + 8, sc) : 0u;
+                    } else {
+                        w0 = sc != 0.0f ? int4x8_exact(make_uint4(w[0], w[1], w[2], w[3]), sc) : 0u;
+                        w1 = sc != 0.0f ? int4x8_exact(make_uint4(w[4], w[5], w[6], w[7]), sc) : 0u;
+                    }
                 }
             }
             if (sc == 0.0f) {
@@ -493,6 +618,35 @@ __global__ void __launch_bounds__(256) amax_kernel(const uint16_t* X, int M, int
         float v = 0.0f;
         for (int w = 0; w < (int)(blockDim.x >> 5); ++w) v = fmaxf(v, red[w]);
         atomicMax(reinterpret_cast<unsigned int*>(out), __float_as_uint(v));  // v >= 0: bit order = value order
+    }
+}
+
+// The tensor amax of the rotated NVFP4 tensor (16-element blocks rotated by
+// rotate_item, act: times 1/16): grid-stride over 16-element chunks.
+__global__ void __launch_bounds__(256) amax_rot_kernel(const uint16_t* X, int M, int K, int ldx, int act, float* out) {
+    pdl_launch_dependents();
+    const int chunks = K / 16;
+    const long long total = (long long)M * chunks;
+    float m = 0.0f;
+    for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < total;
+         i += (long long)gridDim.x * blockDim.x) {
+        const long long r = i / chunks;
+        const int c = (int)(i - r * chunks);
+        const uint4* p = reinterpret_cast<const uint4*>(X + r * ldx) + 2 * c;
+        const uint4 v0 = __ldg(p), v1 = __ldg(p + 1);
+        const uint32_t w[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
+        float v[16];
+        rotate_item<16>(w, v, c, act != 0);  // one item per block: no lane exchange
+        m = fmaxf(m, absmax16(v));
+    }
+    m = warp_max(m);
+    __shared__ float red[8];
+    if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = m;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        float v = 0.0f;
+        for (int w = 0; w < (int)(blockDim.x >> 5); ++w) v = fmaxf(v, red[w]);
+        atomicMax(reinterpret_cast<unsigned int*>(out), __float_as_uint(v));
     }
 }
 
@@ -777,7 +931,7 @@ static cudaError_t launch_nvfp4_token(const QuantArgs& a, int rows_pad, int num_
     return e != cudaSuccess ? e : cudaGetLastError();
 }
 
-template <int FMT, bool GATHER, bool MULTI = false>
+template <int FMT, bool GATHER, bool MULTI = false, bool ROT = false>
 static cudaError_t launch_quant_fmt(const QuantArgs& a, int rows_pad, int num_sms, cudaStream_t st) {
     const int row_bytes = a.K_src * 2;
     // One row block per CTA (about 32 KB of rows, several CTAs resident per
@@ -789,7 +943,7 @@ static cudaError_t launch_quant_fmt(const QuantArgs& a, int rows_pad, int num_sm
     const size_t smem = nbuf * buf + 8 * nbuf + 4 * rpc + sizeof(RowConsts) * rpc +
                         (FMT == FMT_NVFP4 ? 4 * (size_t)rpc * (a.K / 16) : 0) + 16;
     if (smem > 200 * 1024) return cudaErrorInvalidValue;
-    auto kern = quant_rows_kernel<FMT, GATHER, MULTI>;
+    auto kern = quant_rows_kernel<FMT, GATHER, MULTI, ROT>;
     static size_t attr = 0;
     if (smem > 48 * 1024 && smem > attr) {
         cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
@@ -807,6 +961,12 @@ static cudaError_t launch_quant_fmt(const QuantArgs& a, int rows_pad, int num_sm
 }
 
 cudaError_t launch_quant(int fmt, bool gather, const QuantArgs& a, int rows_pad, int num_sms, cudaStream_t st) {
+    if (a.rot) {  // block-local rotation (no gather, one pass)
+        if (gather || a.passes > 1) return cudaErrorInvalidValue;
+        if (fmt == FMT_NVFP4) return launch_quant_fmt<FMT_NVFP4, false, false, true>(a, rows_pad, num_sms, st);
+        if (fmt == FMT_MXFP4) return launch_quant_fmt<FMT_MXFP4, false, false, true>(a, rows_pad, num_sms, st);
+        return launch_quant_fmt<FMT_INT4, false, false, true>(a, rows_pad, num_sms, st);
+    }
     if (fmt == FMT_NVFP4 && !gather && a.mode == 1 && !a.static_s2 && a.K == a.K_src && a.K <= 49152)
         return launch_nvfp4_token(a, rows_pad, num_sms, st);
     if (fmt == FMT_NVFP4) return gather ? launch_quant_fmt<FMT_NVFP4, true>(a, rows_pad, num_sms, st)
@@ -819,12 +979,13 @@ cudaError_t launch_quant(int fmt, bool gather, const QuantArgs& a, int rows_pad,
                   : launch_quant_fmt<FMT_INT4, false>(a, rows_pad, num_sms, st);
 }
 
-cudaError_t launch_amax(const uint16_t* X, int M, int K, int ldx, float* out, int num_sms, cudaStream_t st) {
+cudaError_t launch_amax(const uint16_t* X, int M, int K, int ldx, float* out, int num_sms, cudaStream_t st, int rot) {
     long long vecs = (long long)M * (K / 8);
     long long blocks = (vecs + 255) / 256;
     int grid = (int)(blocks < (long long)num_sms * 8 ? blocks : (long long)num_sms * 8);
     if (grid < 1) grid = 1;
-    amax_kernel<<<grid, 256, 0, st>>>(X, M, K, ldx, out);
+    if (rot) amax_rot_kernel<<<grid, 256, 0, st>>>(X, M, K, ldx, rot == 1, out);
+    else amax_kernel<<<grid, 256, 0, st>>>(X, M, K, ldx, out);
     return cudaGetLastError();
 }
 

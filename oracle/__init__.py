@@ -73,6 +73,9 @@ def _declare(L):
     L.orc_quant_nvfp4_f32.argtypes = [_f32p, C.c_int, C.c_int, C.c_int, _u8p, _u8p, _f32p]
     L.orc_quant_mxfp4_f32.argtypes = [_f32p, C.c_int, C.c_int, _u8p, _u8p]
     L.orc_quant_int4_f32.argtypes = [_f32p, C.c_int, C.c_int, _u8p, _f32p]
+    L.orc_quant_int4_g.argtypes = [_u16p, C.c_int, C.c_int, C.c_int, C.c_int, _u8p, _f32p]
+    L.orc_quant_int4_f32_g.argtypes = [_f32p, C.c_int, C.c_int, C.c_int, _u8p, _f32p]
+    L.orc_gemm_int4_g.argtypes = [_u8p, _f32p, _u8p, _f32p, C.c_int, C.c_int, C.c_int, C.c_int, _u16p, _f64p, _f64p]
     L.orc_quant_int4.argtypes = [_u16p, C.c_int, C.c_int, C.c_int, _u8p, _f32p]
     L.orc_dequant_nvfp4.argtypes = [_u8p, _u8p, _f32p, C.c_int, C.c_int, C.c_int, _f64p]
     L.orc_dequant_mxfp4.argtypes = [_u8p, _u8p, C.c_int, C.c_int, _f64p]
@@ -230,6 +233,36 @@ def quant_int4_f32(Xf):
     scales = np.zeros((M, K // 128), np.float32)
     _check(lib().orc_quant_int4_f32(_p(Xf, _f32p), M, K, _p(codes, _u8p), _p(scales, _f32p)), "quant_int4_f32")
     return codes, scales
+
+
+def quant_int4_g(X, G):
+    """INT4 with groups of G elements: (codes [M, K/2], scales [M, K/G] f32)."""
+    X = _bf16(X)
+    M, K = X.shape
+    codes = np.zeros((M, K // 2), np.uint8)
+    scales = np.zeros((M, K // G), np.float32)
+    _check(lib().orc_quant_int4_g(_p(X, _u16p), M, K, K, G, _p(codes, _u8p), _p(scales, _f32p)), "quant_int4_g")
+    return codes, scales
+
+
+def quant_int4_f32_g(Xf, G):
+    Xf = np.ascontiguousarray(Xf, np.float32)
+    M, K = Xf.shape
+    codes = np.zeros((M, K // 2), np.uint8)
+    scales = np.zeros((M, K // G), np.float32)
+    _check(lib().orc_quant_int4_f32_g(_p(Xf, _f32p), M, K, G, _p(codes, _u8p), _p(scales, _f32p)), "quant_int4_f32_g")
+    return codes, scales
+
+
+def gemm_int4_g(ca, sa, cw, sw, G, want_ref=True):
+    M, K = ca.shape[0], ca.shape[1] * 2
+    N = cw.shape[0]
+    Y, yref, absd = _gemm_out(M, N, want_ref)
+    c = np.ascontiguousarray
+    _check(lib().orc_gemm_int4_g(_p(c(ca), _u8p), _p(c(sa, np.float32), _f32p), _p(c(cw), _u8p),
+                                 _p(c(sw, np.float32), _f32p), M, N, K, G, _p(Y, _u16p), _p(yref, _f64p),
+                                 _p(absd, _f64p)), "gemm_int4_g")
+    return Y, yref, absd
 
 
 def quant_int4(X):

@@ -406,6 +406,50 @@ static void int4_group(const float* x, uint8_t* codes64 /* 64 bytes */, float* s
     *scale = s;
 }
 
+/* The INT4 rule over a group of G elements (G a multiple of 128): the same
+ * steps as int4_group with the group's own amax.  Coarser groups are the
+ * granularity knob of the "Depth Registers..." thelatestinai page, para 2
+ * (APEX4: rho-aware granularity adaptation, mixed-granularity mode). */
+static void int4_group_n(const float* x, int G, uint8_t* codes, float* scale) {
+    float amax = 0.0f;
+    for (int i = 0; i < G; ++i) amax = fmaxf(amax, fabsf(x[i]));
+    const float s = amax / 7.0f;
+    for (int j = 0; j < G / 2; ++j) {
+        int q[2];
+        for (int h = 0; h < 2; ++h) {
+            q[h] = 0;
+            if (s == 0.0f) continue;
+            float r = rintf(x[2 * j + h] / s);
+            if (r > 7.0f) r = 7.0f;
+            if (r < -8.0f) r = -8.0f;
+            q[h] = (int)r;
+        }
+        codes[j] = (uint8_t)((q[0] & 15) | ((q[1] & 15) << 4));
+    }
+    *scale = s;
+}
+
+int orc_quant_int4_g(const uint16_t* X, int M, int K, int ldx, int G, uint8_t* codes, float* scales) {
+    if (M < 0 || G < 128 || G % 128 || K % G || ldx < K) return -1;
+    float* x = (float*)malloc(sizeof(float) * (size_t)G);
+    for (int m = 0; m < M; ++m)
+        for (int g = 0; g < K / G; ++g) {
+            for (int i = 0; i < G; ++i) x[i] = orc_bf16_to_f32(X[(size_t)m * ldx + (size_t)G * g + i]);
+            int4_group_n(x, G, codes + (size_t)m * (K / 2) + (size_t)(G / 2) * g, scales + (size_t)m * (K / G) + g);
+        }
+    free(x);
+    return 0;
+}
+
+int orc_quant_int4_f32_g(const float* X, int M, int K, int G, uint8_t* codes, float* scales) {
+    if (M < 0 || G < 128 || G % 128 || K % G) return -1;
+    for (int m = 0; m < M; ++m)
+        for (int g = 0; g < K / G; ++g)
+            int4_group_n(X + (size_t)m * K + (size_t)G * g, G, codes + (size_t)m * (K / 2) + (size_t)(G / 2) * g,
+                         scales + (size_t)m * (K / G) + g);
+    return 0;
+}
+
 int orc_quant_int4_f32(const float* X, int M, int K, uint8_t* codes, float* scales) {
     if (M < 0 || K % 128) return -1;
     for (int m = 0; m < M; ++m)
@@ -540,6 +584,33 @@ int orc_gemm_int4(const uint8_t* ca, const float* sa, const uint8_t* cw, const f
                     ap += t < 0 ? -t : t;
                 }
                 double sc = (double)sa[(size_t)m * G + g] * (double)sw[(size_t)n * G + g];
+                acc += (double)p * sc;
+                aacc += (double)ap * fabs(sc);
+            }
+            if (Y) Y[(size_t)m * N + n] = orc_f64_to_bf16(acc);
+            if (yref) yref[(size_t)m * N + n] = acc;
+            if (absdot) absdot[(size_t)m * N + n] = aacc;
+        }
+    return 0;
+}
+
+/* INT4 product with groups of G elements: exact integer partial sum per
+ * group, scaled by sa[m,g] * sw[n,g] (fp64), summed. */
+int orc_gemm_int4_g(const uint8_t* ca, const float* sa, const uint8_t* cw, const float* sw,
+                    int M, int N, int K, int G, uint16_t* Y, double* yref, double* absdot) {
+    if (G < 128 || G % 128 || K % G) return -1;
+    const int NG = K / G;
+    for (int m = 0; m < M; ++m)
+        for (int n = 0; n < N; ++n) {
+            double acc = 0.0, aacc = 0.0;
+            for (int g = 0; g < NG; ++g) {
+                long long p = 0, ap = 0;
+                for (int k = G * g; k < G * g + G; ++k) {
+                    int t = int4_value(nib(ca, K / 2, m, k)) * int4_value(nib(cw, K / 2, n, k));
+                    p += t;
+                    ap += t < 0 ? -t : t;
+                }
+                double sc = (double)sa[(size_t)m * NG + g] * (double)sw[(size_t)n * NG + g];
                 acc += (double)p * sc;
                 aacc += (double)ap * fabs(sc);
             }

@@ -88,6 +88,14 @@ int orc_quant_nvfp4_f32(const float* X, int M, int K, int mode,
                         uint8_t* codes, uint8_t* scales, float* s2);
 int orc_quant_mxfp4_f32(const float* X, int M, int K, uint8_t* codes, uint8_t* scales);
 int orc_quant_int4_f32(const float* X, int M, int K, uint8_t* codes, float* scales);
+/* INT4 with groups of G elements (G a multiple of 128, K a multiple of G;
+ * "Depth Registers..." thelatestinai page, para 2: rho-aware granularity):
+ * the same rule per group; scales [M][K/G].                                */
+int orc_quant_int4_g(const uint16_t* X, int M, int K, int ldx, int G,
+                     uint8_t* codes, float* scales);
+int orc_quant_int4_f32_g(const float* X, int M, int K, int G, uint8_t* codes, float* scales);
+int orc_gemm_int4_g(const uint8_t* ca, const float* sa, const uint8_t* cw, const float* sw,
+                    int M, int N, int K, int G, uint16_t* Y, double* yref, double* absdot);
 /* codes [M][K/2] two's-complement nibbles, scales [M][K/128] FP32          */
 int orc_quant_int4(const uint16_t* X, int M, int K, int ldx,
                    uint8_t* codes, float* scales);

@@ -561,3 +561,51 @@ def test_fp32_quantizers_reduce_to_the_bf16_ones(orc):
         np.testing.assert_array_equal(u, v)
     for u, v in zip(orc.quant_int4_f32(xf), orc.quant_int4(Xb)):
         np.testing.assert_array_equal(u.view(np.uint8), v.view(np.uint8))
+
+
+# ---- INT4 with coarser groups ------------------------------------------------
+def test_int4_g128_is_the_base_rule(orc):
+    Xb = synth.activations("qwen25_7b_int4", 7, 512, seed=71)
+    for u, v in zip(orc.quant_int4_g(Xb, 128), orc.quant_int4(Xb)):
+        np.testing.assert_array_equal(u.view(np.uint8), v.view(np.uint8))
+
+
+@pytest.mark.parametrize("G", [256, 512, 1024])
+def test_int4_groups_follow_the_rule(orc, G):
+    """Each group of G: s = RN32(amax/7), q = clamp(rint(x/s), -8, 7) with IEEE
+    FP32 division (numpy float32), ties to even; zero group -> s = 0, codes 0."""
+    K = 2048
+    Xb = synth.activations("qwen25_7b_int4", 5, K, seed=72)
+    Xb[1, :G] = 0
+    c, s = orc.quant_int4_g(Xb, G)
+    x = synth.bf16_bits_to_f32(Xb)
+    q = unpack(c).astype(np.int64)
+    q = np.where(q >= 8, q - 16, q)
+    for m in range(5):
+        for g in range(K // G):
+            blk = x[m, G * g:G * g + G]
+            sc = np.float32(np.abs(blk).max()) / np.float32(7)
+            assert s[m, g] == sc
+            want = np.zeros(G, np.int64) if sc == 0 else np.clip(np.rint(blk / sc), -8, 7).astype(np.int64)
+            np.testing.assert_array_equal(q[m, G * g:G * g + G], want)
+    assert s[1, 0] == 0 and np.all(q[1, :G] == 0)
+
+
+@pytest.mark.parametrize("G", [128, 512])
+def test_int4_group_gemm_vs_fp64(orc, G):
+    """The grouped product equals the fp64 product of the dequantized operands
+    (codes times their group's scale, restated here)."""
+    M, N, K = 6, 9, 1024
+    Xa = synth.activations("qwen25_7b_int4", M, K, seed=73)
+    Xw = synth.weights("qwen25_7b_int4", N, K, seed=73)
+    ca, sa = orc.quant_int4_g(Xa, G)
+    cw, sw = orc.quant_int4_g(Xw, G)
+
+    def deq(c, s):
+        q = unpack(c).astype(np.float64)
+        q = np.where(q >= 8, q - 16, q)
+        return q * np.repeat(s.astype(np.float64), G, axis=1)
+    want = deq(ca, sa) @ deq(cw, sw).T
+    _, yref, absd = orc.gemm_int4_g(ca, sa, cw, sw, G)
+    np.testing.assert_allclose(yref, want, rtol=1e-12, atol=1e-12 * np.abs(want).max())
+    assert np.all(absd >= np.abs(yref) * (1 - 1e-12))

@@ -425,23 +425,25 @@ def extra_rows(args, dev, stream, P):
                                             "us": round(ms * 1e3, 2)}
     del Ws
 
-    # INT4-g128, Qwen2.5-7B shapes at M = 2048
-    tot_ms, tot_ops = 0.0, 0.0
-    for li, (name, K, N) in enumerate(synth.SHAPES["qwen25_7b_int4"] if want("int4") else []):
-        M = 2048
-        Wq = w4.quantize_weight(to_dev(synth.weights("qwen25_7b_int4", N, K, tensor_id=300 + li), dev), w4.INT4)
-        X = to_dev(synth.activations("qwen25_7b_int4", M, K), dev)
-        Y = torch.empty(M, N, dtype=torch.bfloat16, device=dev)
-        ws = torch.empty(w4.linear_workspace(M, N, K, w4.INT4), dtype=torch.uint8, device=dev)
-        f = lambda: w4.linear(X, Wq, 0, Y=Y, ws=ws)
-        f()
-        ms = time_loop(f, it, stream)
-        tot_ms += ms
-        tot_ops += 2.0 * M * N * K
+    # INT4, Qwen2.5-7B shapes at M = 2048: groups of 128, and of 512 (the
+    # rho-aware choice for this device's tensor / CUDA-core ratio)
     i8_peak = P["bf16"] * INT8_PER_BF16
-    if tot_ms > 0:
+    for G in ((128, w4.int4_group_for_rho(60.0)) if want("int4") else ()):
+        tot_ms, tot_ops = 0.0, 0.0
+        for li, (name, K, N) in enumerate(synth.SHAPES["qwen25_7b_int4"]):
+            M = 2048
+            Wq = w4.quantize_weight(to_dev(synth.weights("qwen25_7b_int4", N, K, tensor_id=300 + li), dev), w4.INT4,
+                                    group=G)
+            X = to_dev(synth.activations("qwen25_7b_int4", M, K), dev)
+            Y = torch.empty(M, N, dtype=torch.bfloat16, device=dev)
+            ws = torch.empty(w4.linear_workspace(M, N, K, w4.INT4), dtype=torch.uint8, device=dev)
+            f = lambda: w4.linear(X, Wq, 0, Y=Y, ws=ws)
+            f()
+            ms = time_loop(f, it, stream)
+            tot_ms += ms
+            tot_ops += 2.0 * M * N * K
         v = tot_ops / (tot_ms * 1e-3) / 1e12
-        out["int4_g128_qwen25_7b_m2048"] = {"TOPS": round(v, 1), "frac_int8_peak": round(v / i8_peak, 3)}
+        out[f"int4_g{G}_qwen25_7b_m2048"] = {"TOPS": round(v, 1), "frac_int8_peak": round(v / i8_peak, 3)}
 
     # dual-stage residual augmentation, Qwen2.5-3B shapes at M = 8192
     tot_ms, tot_f, tot_fk = 0.0, 0.0, 0.0

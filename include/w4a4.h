@@ -83,8 +83,8 @@ extern "C" {
  *         consecutive scales, the scale of (row r, block c) at byte
  *           ((r/128) * (cols/g/4) + c/4) * 512 + (r%32)*16 + ((r%128)/32)*4 + c%4
  *         (g = 16 or 32); rows are padded to a multiple of 128 with zero
- *         scales.  INT4: FP32, group-major [cols/128][pad128(rows)], the scale
- *         of (row r, group c) at index c * pad128(rows) + r.
+ *         scales.  INT4: FP32, group-major [cols/group][pad128(rows)], the
+ *         scale of (row r, group c) at index c * pad128(rows) + r.
  * s2      NVFP4 only: FP32 second-level scales; TENSOR: s2[0] is the scale and
  *         s2[1] is scratch for the tensor amax; TOKEN: s2[r] per row.
  *
@@ -112,7 +112,7 @@ typedef struct w4a4_qtensor {
     int32_t format;      /* W4A4_NVFP4 / W4A4_MXFP4 / W4A4_INT4 */
     int32_t rows;
     int32_t cols;
-    int32_t group;       /* 16 / 32 / 128, must match format */
+    int32_t group;       /* 16 (NVFP4) / 32 (MXFP4) / 128, 256 or 512 (INT4; cols % group == 0) */
     int32_t scale_mode;  /* NVFP4: W4A4_SCALE_TENSOR or W4A4_SCALE_TOKEN; else ignored */
     int32_t flags;       /* 0, or W4A4_FLAG_HADAMARD (see below); other bits must be 0 */
     void*   codes;       /* device */
@@ -122,7 +122,8 @@ typedef struct w4a4_qtensor {
 
 /* Bytes each buffer of a quantized tensor needs.  Host only, no device work.
  * Any of the out-pointers may be NULL.  Returns W4A4_OK or
- * W4A4_ERR_INVALID_ARG. */
+ * W4A4_ERR_INVALID_ARG.  INT4 scales are sized for group 128, which bounds
+ * the coarser groups too. */
 int w4a4_qtensor_bytes(int format, int rows, int cols, int scale_mode,
                        size_t* codes_bytes, size_t* scales_bytes, size_t* s2_bytes);
 
@@ -130,7 +131,12 @@ int w4a4_qtensor_bytes(int format, int rows, int cols, int scale_mode,
  * Quantize activations X[M,K] (bf16, row stride ldx) into `out`, per token
  * ("Daily Papers" para 4: per-token quantization; "Depth Registers..."
  * abstract: round to nearest).
- *   format/group: (NVFP4,16), (MXFP4,32) or (INT4,128).
+ *   format/group: (NVFP4,16), (MXFP4,32) or (INT4, 128 / 256 / 512; K a
+ *     multiple of the group).  INT4 groups coarser than 128 are the
+ *     granularity knob of the "Depth Registers..." thelatestinai page, para 2
+ *     (APEX4: rho-aware granularity adaptation): the GEMM rescales once per
+ *     group, so a group of 512 takes a quarter of g128's CUDA-core work; the
+ *     weights must use the same group (w4a4_int4_group_for_rho picks one).
  *   scale_mode (NVFP4): TOKEN -> s2[r] = amax(row r)/2688; TENSOR ->
  *     s2[0] = amax(X)/2688 from an extra reduction pass (two reads of X).
  *     A zero amax, or a quotient below the smallest normal float, gives 1.
@@ -227,6 +233,13 @@ int w4a4_quantize_weight_msd(const uint16_t* W, int N, int K, int ldw, int passe
  */
 int w4a4_gemm(const w4a4_qtensor* A, const w4a4_qtensor* B,
               uint16_t* Y, int ldy, void* stream);
+
+/* INT4 group size for a device whose tensor-core / CUDA-core throughput
+ * ratio is rho ("Depth Registers..." thelatestinai page, para 2: APEX4's
+ * rho; g128 pays at rho = 16, not at 64): 128 up to rho = 16, then doubled
+ * per doubling of rho, at most 512.  B200's int8-tensor to FP32-FMA ratio is
+ * about 60, which gives 512.  Host only. */
+int w4a4_int4_group_for_rho(double rho);
 
 /* Workspace bytes w4a4_linear needs for these sizes (0 on bad arguments). */
 size_t w4a4_linear_workspace(int M, int N, int K, int format, int nS);

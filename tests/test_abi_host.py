@@ -184,3 +184,21 @@ def test_hadamard_flag_arguments(L):
     m = _qt(w4.MXFP4, 4, 512)
     m.flags = w4.FLAG_HADAMARD
     assert L.w4a4_quantize_act_msd(X, 4, 256, 256, 2, C.byref(m), None) == w4.ERR_INVALID_ARG
+
+
+def test_int4_group_choice_and_checks(L):
+    """rho-aware INT4 group size: 128 up to rho = 16, doubled per doubling, at
+    most 512; groups other than 128/256/512, or not dividing K, are rejected."""
+    assert [w4.int4_group_for_rho(r) for r in (0, 8, 16, 17, 32, 33, 60, 64, 1000)] == \
+        [128, 128, 128, 256, 256, 512, 512, 512, 512]
+    X = C.c_void_p(16)
+    q = _qt(w4.INT4, 4, 1024)
+    q.group = 384
+    assert L.w4a4_quantize_act(X, 4, 1024, 1024, w4.INT4, 384, 0, None, C.byref(q), None) == w4.ERR_INVALID_ARG
+    q = _qt(w4.INT4, 4, 384)
+    q.group = 256
+    assert L.w4a4_quantize_act(X, 4, 384, 384, w4.INT4, 256, 0, None, C.byref(q), None) == w4.ERR_INVALID_ARG
+    a = _qt(w4.INT4, 4, 1024)
+    a.group = 512
+    b = _qt(w4.INT4, 256, 1024)
+    assert L.w4a4_gemm(C.byref(a), C.byref(b), C.c_void_p(16), 256, None) == w4.ERR_INVALID_ARG  # groups differ

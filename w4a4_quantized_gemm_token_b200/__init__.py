@@ -28,7 +28,7 @@ EXPORTS = ("w4a4_qtensor_bytes", "w4a4_quantize_act", "w4a4_quantize_weight", "w
            "w4a4_linear_workspace", "w4a4_linear", "w4a4_augment_residual", "w4a4_select_channels",
            "w4a4_device_status", "w4a4_debug_set", "w4a4_status_string", "w4a4_linear_noalloc",
            "w4a4_quantize_weight_segments", "w4a4_quantize_act_msd", "w4a4_quantize_weight_msd",
-           "w4a4_linear_msd")
+           "w4a4_linear_msd", "w4a4_int4_group_for_rho")
 
 
 class W4A4Error(RuntimeError):
@@ -61,6 +61,7 @@ def lib():
         L.w4a4_quantize_weight.argtypes = [vp, i, i, i, i, i, vp, i, qp, vp]
         L.w4a4_quantize_weight_segments.argtypes = [vp, i, i, i, C.POINTER(C.c_int32), i, vp, i, qp, vp]
         L.w4a4_gemm.argtypes = [qp, qp, vp, i, vp]
+        L.w4a4_int4_group_for_rho.argtypes = [C.c_double]
         L.w4a4_quantize_act_msd.argtypes = [vp, i, i, i, i, qp, vp]
         L.w4a4_quantize_weight_msd.argtypes = [vp, i, i, i, i, qp, vp]
         L.w4a4_linear_msd.argtypes = [vp, i, i, i, qp, i, vp, i, vp, sz, vp]
@@ -78,7 +79,7 @@ def lib():
         for name in ("w4a4_qtensor_bytes", "w4a4_quantize_act", "w4a4_quantize_weight", "w4a4_gemm",
                      "w4a4_linear", "w4a4_augment_residual", "w4a4_select_channels", "w4a4_device_status",
                      "w4a4_linear_noalloc", "w4a4_quantize_weight_segments", "w4a4_quantize_act_msd",
-                     "w4a4_quantize_weight_msd", "w4a4_linear_msd"):
+                     "w4a4_quantize_weight_msd", "w4a4_linear_msd", "w4a4_int4_group_for_rho"):
             getattr(L, name).restype = i
         _lib = L
     return _lib
@@ -112,14 +113,16 @@ def qtensor_bytes(fmt: int, rows: int, cols: int, scale_mode: int = SCALE_TENSOR
 class QTensor:
     """A quantized tensor whose buffers are torch uint8/float32 device tensors."""
 
-    def __init__(self, fmt: int, rows: int, cols: int, scale_mode: int = SCALE_TENSOR, device="cuda", flags: int = 0):
+    def __init__(self, fmt: int, rows: int, cols: int, scale_mode: int = SCALE_TENSOR, device="cuda", flags: int = 0,
+                 group: int | None = None):
         import torch
         cb, sb, tb = qtensor_bytes(fmt, rows, cols, scale_mode)
         self.format, self.rows, self.cols, self.scale_mode, self.flags = fmt, rows, cols, scale_mode, flags
+        self.group = group or GROUP[fmt]
         self.codes = torch.zeros(max(cb, 16), dtype=torch.uint8, device=device)
         self.scales = torch.zeros(max(sb, 16), dtype=torch.uint8, device=device)
         self.s2 = torch.zeros(max(tb // 4, 4), dtype=torch.float32, device=device) if tb else None
-        self.struct = QTensorStruct(fmt, rows, cols, GROUP[fmt], scale_mode if fmt == NVFP4 else 0, flags,
+        self.struct = QTensorStruct(fmt, rows, cols, self.group, scale_mode if fmt == NVFP4 else 0, flags,
                                     self.codes.data_ptr(), self.scales.data_ptr(),
                                     self.s2.data_ptr() if self.s2 is not None else None)
 
@@ -129,26 +132,27 @@ class QTensor:
 
 
 def quantize_act(X, fmt: int, scale_mode: int = SCALE_TOKEN, static_s2=None, out: QTensor | None = None,
-                 cols: int | None = None, hadamard: bool = False) -> QTensor:
+                 cols: int | None = None, hadamard: bool = False, group: int | None = None) -> QTensor:
     """X: bf16 [M, K] CUDA tensor (row stride may exceed K).  hadamard: rotate
     each quantization block first (activation side, times 1/block)."""
     M, K = X.shape
     if out is None:
         out = QTensor(fmt, M, cols or K, scale_mode if fmt == NVFP4 else SCALE_TENSOR, X.device,
-                      FLAG_HADAMARD if hadamard else 0)
-    _check(lib().w4a4_quantize_act(_ptr(X), M, K, X.stride(0), fmt, GROUP[fmt], scale_mode, _ptr(static_s2),
+                      FLAG_HADAMARD if hadamard else 0, group)
+    _check(lib().w4a4_quantize_act(_ptr(X), M, K, X.stride(0), fmt, out.group, scale_mode, _ptr(static_s2),
                                    out.ref, _stream()), "w4a4_quantize_act")
     return out
 
 
-def quantize_weight(W, fmt: int, S=None, out: QTensor | None = None, hadamard: bool = False) -> QTensor:
+def quantize_weight(W, fmt: int, S=None, out: QTensor | None = None, hadamard: bool = False,
+                    group: int | None = None) -> QTensor:
     """W: bf16 [N, K]; S: optional int32 CUDA tensor of augmented channels;
     hadamard: rotate each quantization block first (weight side, unscaled)."""
     N, K = W.shape
     nS = 0 if S is None else S.numel()
     if out is None:
-        out = QTensor(fmt, N, K + nS, SCALE_TENSOR, W.device, FLAG_HADAMARD if hadamard else 0)
-    _check(lib().w4a4_quantize_weight(_ptr(W), N, K, W.stride(0), fmt, GROUP[fmt], _ptr(S), nS, out.ref,
+        out = QTensor(fmt, N, K + nS, SCALE_TENSOR, W.device, FLAG_HADAMARD if hadamard else 0, group)
+    _check(lib().w4a4_quantize_weight(_ptr(W), N, K, W.stride(0), fmt, out.group, _ptr(S), nS, out.ref,
                                       _stream()), "w4a4_quantize_weight")
     return out
 
@@ -212,6 +216,11 @@ def gemm(A: QTensor, B: QTensor, Y=None):
         Y = torch.empty(A.rows, B.rows, dtype=torch.bfloat16, device=A.codes.device)
     _check(lib().w4a4_gemm(A.ref, B.ref, _ptr(Y), Y.stride(0), _stream()), "w4a4_gemm")
     return Y
+
+
+def int4_group_for_rho(rho: float) -> int:
+    """INT4 scale-group size for a tensor-core / CUDA-core throughput ratio rho."""
+    return int(lib().w4a4_int4_group_for_rho(float(rho)))
 
 
 def linear_workspace(M: int, N: int, K: int, fmt: int, nS: int = 0) -> int:

@@ -67,6 +67,11 @@ inline int pad128(int x) { return (x + 127) / 128 * 128; }
 inline size_t align256(size_t x) { return (x + 255) / 256 * 256; }
 
 int group_of(int fmt) { return fmt == W4A4_NVFP4 ? 16 : fmt == W4A4_MXFP4 ? 32 : fmt == W4A4_INT4 ? 128 : -1; }
+// Group sizes a format accepts: its own, and for INT4 also 256 and 512 (the
+// coarser scale groups of the rho-aware granularity).
+bool group_ok(int fmt, int group) {
+    return group == group_of(fmt) || (fmt == W4A4_INT4 && (group == 256 || group == 512));
+}
 
 // 2-D byte tensor map over codes[rows][row_bytes] with a box of box_x bytes x box_y rows.
 int make_map(CUtensorMap* map, const void* base, int rows, int row_bytes, int box_x, int box_y, bool swizzle128) {
@@ -112,9 +117,10 @@ int make_map_sf_rep(CUtensorMap* map, const void* base, int row_tiles, int col_a
 
 int check_qtensor(const w4a4_qtensor* q) {
     if (!q || !q->codes || !q->scales) return W4A4_ERR_INVALID_ARG;
-    if (q->format < 0 || q->format > 2 || q->group != group_of(q->format) || (q->flags & ~W4A4_FLAG_HADAMARD))
+    if (q->format < 0 || q->format > 2 || !group_ok(q->format, q->group) || (q->flags & ~W4A4_FLAG_HADAMARD))
         return W4A4_ERR_INVALID_ARG;
     if (q->rows < 0 || q->cols < 128 || q->cols % 128 || q->cols > kMaxPasses * kMaxK) return W4A4_ERR_INVALID_ARG;
+    if (q->format == W4A4_INT4 && q->cols % q->group) return W4A4_ERR_INVALID_ARG;
     if (q->format == W4A4_NVFP4) {
         if (!q->s2) return W4A4_ERR_INVALID_ARG;
         if (q->scale_mode != W4A4_SCALE_TENSOR && q->scale_mode != W4A4_SCALE_TOKEN) return W4A4_ERR_INVALID_ARG;
@@ -147,6 +153,7 @@ int quantize_rows(const uint16_t* X, int M, int K, int ldx, const int32_t* S, in
     a.ldc = q->cols / 2;
     a.sf = static_cast<uint8_t*>(q->scales);
     a.sf_col_atoms = q->cols / q->group / 4;
+    a.group = q->group;
     a.sfi = static_cast<float*>(q->scales);
     a.sfi_ld = pad128(q->rows);
     a.mode = q->scale_mode;
@@ -195,6 +202,7 @@ int setup_gemm(const w4a4_qtensor* A, const w4a4_qtensor* B, uint16_t* Y, int ld
     g.sfa = static_cast<const uint8_t*>(A->scales);
     g.sfb = static_cast<const uint8_t*>(B->scales);
     g.sf_col_atoms = A->format == W4A4_INT4 ? 0 : A->cols / A->group / 4;
+    g.int4_group = A->group;
     g.sfa_ld = pad128(A->rows);
     g.sfb_ld = pad128(B->rows);
     g.s2a = A->s2;
@@ -320,7 +328,7 @@ int w4a4_qtensor_bytes(int format, int rows, int cols, int scale_mode, size_t* c
 int w4a4_quantize_act(const uint16_t* X, int M, int K, int ldx, int format, int group, int scale_mode,
                       const float* static_s2, w4a4_qtensor* out, void* stream) {
     if (M < 0 || K < 128 || K % 128 || K > kMaxK || ldx < K) return W4A4_ERR_INVALID_ARG;
-    if (group_of(format) != group) return W4A4_ERR_INVALID_ARG;
+    if (!group_ok(format, group) || K % group) return W4A4_ERR_INVALID_ARG;
     int rc = check_qtensor(out);
     if (rc != W4A4_OK) return rc;
     if (out->format != format || out->group != group || out->rows != M || out->cols < K ||
@@ -339,12 +347,13 @@ int w4a4_quantize_act(const uint16_t* X, int M, int K, int ldx, int format, int 
 int w4a4_quantize_weight(const uint16_t* W, int N, int K, int ldw, int format, int group, const int32_t* S, int nS,
                          w4a4_qtensor* out, void* stream) {
     if (N < 0 || K < 128 || K % 128 || K > kMaxK || ldw < K) return W4A4_ERR_INVALID_ARG;
-    if (group_of(format) != group) return W4A4_ERR_INVALID_ARG;
+    if (!group_ok(format, group) || K % group) return W4A4_ERR_INVALID_ARG;
     int rc = check_S_args(S, nS, K);
     if (rc != W4A4_OK) return rc;
     rc = check_qtensor(out);
     if (rc != W4A4_OK) return rc;
-    if (out->format != format || out->rows != N || out->cols != K + nS) return W4A4_ERR_INVALID_ARG;
+    if (out->format != format || out->group != group || out->rows != N || out->cols != K + nS)
+        return W4A4_ERR_INVALID_ARG;
     if (format == W4A4_NVFP4 && out->scale_mode != W4A4_SCALE_TENSOR) return W4A4_ERR_INVALID_ARG;
     if (nS && out->flags) return W4A4_ERR_INVALID_ARG;
     if (N == 0) return W4A4_OK;
@@ -451,7 +460,7 @@ int w4a4_gemm(const w4a4_qtensor* A, const w4a4_qtensor* B, uint16_t* Y, int ldy
     if (rc == W4A4_OK) rc = check_qtensor(B);
     if (rc != W4A4_OK) return rc;
     if (A->format != B->format || A->cols != B->cols || B->rows < 128 || B->rows % 128 || ldy < B->rows ||
-        A->flags != B->flags)
+        A->flags != B->flags || A->group != B->group)
         return W4A4_ERR_INVALID_ARG;
     rc = check_weight_s2(B);
     if (rc != W4A4_OK) return rc;
@@ -462,6 +471,15 @@ int w4a4_gemm(const w4a4_qtensor* A, const w4a4_qtensor* B, uint16_t* Y, int ldy
     rc = device_check(&sms);
     if (rc != W4A4_OK) return rc;
     return run_gemm(A, B, Y, ldy, nullptr, sms, false, as_stream(stream));
+}
+
+int w4a4_int4_group_for_rho(double rho) {
+    // rescales per tensor-core step scale as 1/G: keep them in step with the
+    // MMAs as rho grows past the value (16) where g128 still pays
+    if (!(rho > 0.0)) return 128;
+    int g = 128;
+    while (g < 512 && rho > 16.0 * (g / 128)) g *= 2;
+    return g;
 }
 
 size_t w4a4_linear_workspace(int M, int N, int K, int format, int nS) {
@@ -500,7 +518,7 @@ int w4a4_linear(const uint16_t* X, int M, int K, int ldx, const w4a4_qtensor* Wq
     xq.format = fmt;
     xq.rows = M;
     xq.cols = K + nS;
-    xq.group = group_of(fmt);
+    xq.group = fmt == W4A4_INT4 ? Wq->group : group_of(fmt);  // INT4: the weights' scale groups
     xq.scale_mode = fmt == W4A4_NVFP4 ? scale_mode : 0;
     xq.flags = Wq->flags;  // rotated weights: rotate the activations the same way
     xq.codes = base + L.codes;

@@ -1,13 +1,16 @@
 // INT4-g128 W4A4 GEMM on the sm_100a 8-bit integer MMA (tcgen05.mma kind::i8).
 //
 // sm_100's tensor cores have no 4-bit integer kind, so the packed nibbles are
-// widened to int8 in shared memory (as 16 * q, see widen8_x16).  Per 128-element K group g the MMA
-// produces the exact int32 partial sum P_g[m,n] = sum_{k in g} qa qw into one
-// of two TMEM buffers; CUDA-core warps rescale it,
+// widened to int8 in shared memory (as 16 * q, see widen8_x16).  Per scale
+// group g (GS = 128, 256 or 512 elements of K) the MMAs produce the exact
+// int32 partial sum P_g[m,n] = sum_{k in g} qa qw into one of two TMEM
+// buffers (GS/128 shared-memory stages of 128 elements accumulate into it);
+// CUDA-core warps rescale it,
 //     acc[m,n] += float(P_g[m,n]) * (sa[m,g] * sw[n,g])    (FP32),
 // and at the end round acc to bf16.  This per-group rescale on the CUDA cores
 // is the cost the APEX4 paragraph ("Depth Registers..." thelatestinai page,
-// para 2) analyses through the tensor-core / CUDA-core throughput ratio.
+// para 2) analyses through the tensor-core / CUDA-core throughput ratio; the
+// coarser groups are its rho-aware granularity: GS/128 times fewer rescales.
 //
 // Persistent (one CTA per SM, 128 x 128 output tiles in turn), 14 warps; the
 // MMA and unpack warps run ahead into the next tile while the rescale warps
@@ -89,7 +92,9 @@ __global__ void __launch_bounds__(i4::THREADS, 1)
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int G = g.K / 128;
+    const int KT = g.K / 128;               // shared-memory stages (128 elements of K) per tile
+    const int R = g.int4_group / 128;       // stages per scale group
+    const int NG = g.K / g.int4_group;      // scale groups per tile
     const uint64_t limit = g.wait_limit_ns;
     // persistent: tiles t = blockIdx.x, +gridDim.x, ...; grouped raster over (m tile, n tile)
     const int num_m = (g.M + 127) / 128, num_n = (g.N + kBN_I4 - 1) / kBN_I4;
@@ -138,7 +143,7 @@ __global__ void __launch_bounds__(i4::THREADS, 1)
             for (int t = blockIdx.x; t < ntiles && !stop; t += gridDim.x) {
                 int m_tile, n_tile;
                 coords(t, m_tile, n_tile);
-                for (int k = 0; k < G; ++k, ++gi) {
+                for (int k = 0; k < KT; ++k, ++gi) {
                     const int s = gi % STAGES, n = gi / STAGES;
                     if (gi >= STAGES && !mbar_wait(&empty[s], (n - 1) & 1, limit, abort_flag)) {
                         stop = true;
@@ -157,20 +162,26 @@ __global__ void __launch_bounds__(i4::THREADS, 1)
     } else if (warp == 1) {
         if (lane == 0) {
             bool ok = true;
-            int gi = 0;
+            int gi = 0, sg = 0;  // stages and scale groups of every tile, in order
             for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x) {
-                for (int k = 0; k < G; ++k, ++gi) {
-                    const int s = gi % STAGES, n = gi / STAGES, buf = gi & 1;
+                for (int k = 0; k < KT; ++k, ++gi) {
+                    const int s = gi % STAGES, n = gi / STAGES, buf = sg & 1, sub = k % R;
                     if (!mbar_wait(&conv[s], n & 1, limit, abort_flag)) { ok = false; break; }
-                    if (gi >= 2 && !mbar_wait(&tfree[buf], ((gi >> 1) - 1) & 1, limit, abort_flag)) { ok = false; break; }
+                    if (sub == 0 && sg >= 2 && !mbar_wait(&tfree[buf], ((sg >> 1) - 1) & 1, limit, abort_flag)) {
+                        ok = false;
+                        break;
+                    }
                     tc_fence_after();
                     const uint32_t sA = smem_u32(smem + s * STAGE), sB = sA + UN_BYTES;
 #pragma unroll
                     for (int j = 0; j < 4; ++j)
                         mma_i8(tmem + buf * 128, desc_kmajor_sw128(sA + 32 * j), desc_kmajor_sw128(sB + 32 * j),
-                               idesc_i8(128, kBN_I4), j > 0 ? 1u : 0u);
+                               idesc_i8(128, kBN_I4), (sub > 0 || j > 0) ? 1u : 0u);
                     tc_commit(&empty[s]);
-                    tc_commit(&accf[buf]);
+                    if (sub == R - 1) {
+                        tc_commit(&accf[buf]);
+                        ++sg;
+                    }
                 }
             }
             if (!ok) {
@@ -181,7 +192,7 @@ __global__ void __launch_bounds__(i4::THREADS, 1)
     } else if (warp < 6) {
         // ------------------------------ unpack ------------------------------
         const int uw = warp - 2;  // 0..3
-        const int total = ((ntiles - (int)blockIdx.x + (int)gridDim.x - 1) / (int)gridDim.x) * G;
+        const int total = ((ntiles - (int)blockIdx.x + (int)gridDim.x - 1) / (int)gridDim.x) * KT;
         for (int gi = 0; gi < total; ++gi) {
             const int s = gi % STAGES, n = gi / STAGES;
             if (!mbar_wait(&full[s], n & 1, limit, abort_flag)) break;
@@ -241,12 +252,12 @@ __global__ void __launch_bounds__(i4::THREADS, 1)
             float acc[64];
 #pragma unroll
             for (int i = 0; i < 64; ++i) acc[i] = 0.0f;
-            for (int k = 0; k < G; ++k, ++gi) {
+            for (int k = 0; k < NG; ++k, ++gi) {  // gi: scale groups of every tile, in order
                 const int buf = gi & 1;
                 float* sbb = sb_smem + buf * 128;
                 if (rt < 128) sbb[rt] = sb_next;
                 const float sa = sa_next;
-                if (k + 1 < G) scales_of(t, k + 1, sa_next, sb_next);
+                if (k + 1 < NG) scales_of(t, k + 1, sa_next, sb_next);
                 else if (t + (int)gridDim.x < ntiles) scales_of(t + gridDim.x, 0, sa_next, sb_next);
                 named_bar(1, 256);
                 if (ok) ok = mbar_wait(&accf[buf], (gi >> 1) & 1, limit, abort_flag);

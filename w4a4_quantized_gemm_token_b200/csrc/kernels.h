@@ -31,6 +31,7 @@ struct QuantArgs {
     int zero_count;
     int passes;                // MXFP4: 1, or more for the multi-pass decomposition (pass p
                                // in columns [p*K, (p+1)*K) of codes and scales)
+    int group;                 // INT4: elements per scale group (128, 256 or 512)
     int rot;                   // block-local Walsh-Hadamard rotation: 0 none, 1 activation
                                // side (times 1/block), 2 weight side (unscaled)
 };
@@ -64,6 +65,7 @@ struct GemmArgs {
     int* tile_count;           // decode variant: per weight tile, segments written so far (start at 0)
     int splits;                // split-K factor (decode variant)
     int k_tiles_per_split;
+    int int4_group;            // INT4: elements per scale group (128, 256 or 512)
     int skip_k_tile;           // debug: never load this k-tile (-1 = off)
     unsigned long long wait_limit_ns;
 };

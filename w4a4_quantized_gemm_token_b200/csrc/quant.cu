@@ -542,10 +542,9 @@ __global__ void __launch_bounds__(256, 4) quant_rows_kernel(QuantArgs a, int row
                             make_uint2(p0, p1);
                 }
             }
-        } else {  // INT4, 128-element group = 8 items
-            bmax = fmaxf(bmax, __shfl_xor_sync(0xffffffffu, bmax, 1));
-            bmax = fmaxf(bmax, __shfl_xor_sync(0xffffffffu, bmax, 2));
-            bmax = fmaxf(bmax, __shfl_xor_sync(0xffffffffu, bmax, 4));
+        } else {  // INT4, a group of a.group elements = R8 items on consecutive lanes
+            const int R8 = a.group >> 4;  // 8, 16 or 32
+            for (int o = 1; o < R8; o <<= 1) bmax = fmaxf(bmax, __shfl_xor_sync(0xffffffffu, bmax, o));
             const bool fast = bmax >= 0x1p-100f && bmax <= 0x1p100f;
             float sc = live ? div_refined(bmax, 7.0f, 0x1.24924ap-3f) : 0.0f;  // RN(1/7)
             const float y = __frcp_rn(sc > 0.0f ? sc : 1.0f);
@@ -573,7 +572,7 @@ __global__ void __launch_bounds__(256, 4) quant_rows_kernel(QuantArgs a, int row
                 w0 = 0;
                 w1 = 0;
             }
-            if (valid && (c & 7) == 0) a.sfi[(size_t)(c >> 3) * a.sfi_ld + r] = sc;
+            if (valid && (c & (R8 - 1)) == 0) a.sfi[(size_t)(c / R8) * a.sfi_ld + r] = sc;
         }
         if (live) *reinterpret_cast<uint2*>(a.codes + (size_t)r * a.ldc + 8 * c) = make_uint2(w0, w1);
         i += di;

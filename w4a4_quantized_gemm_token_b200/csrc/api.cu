@@ -21,6 +21,10 @@ namespace {
 constexpr int kMaxDevices = 64;
 constexpr int kMaxK = 65536;
 constexpr int kMaxPasses = 4;  // multi-pass MXFP4 decomposition
+// Internal only (workspace tensors of w4a4_linear, never accepted from a
+// caller): INT4 codes stored as int8 16 * q, [rows][cols] bytes, the layout
+// the INT4 GEMM's MMA reads, so that its unpack warps widen only the weights.
+constexpr int kFlagInt8Codes = 1 << 30;
 
 struct DevInfo {
     bool init = false;
@@ -150,7 +154,8 @@ int quantize_rows(const uint16_t* X, int M, int K, int ldx, const int32_t* S, in
     a.ldx = ldx;
     a.S = S;
     a.codes = static_cast<uint8_t*>(q->codes);
-    a.ldc = q->cols / 2;
+    a.int8_codes = (q->flags & kFlagInt8Codes) ? 1 : 0;
+    a.ldc = a.int8_codes ? q->cols : q->cols / 2;
     a.sf = static_cast<uint8_t*>(q->scales);
     a.sf_col_atoms = q->cols / q->group / 4;
     a.group = q->group;
@@ -216,7 +221,10 @@ int setup_gemm(const w4a4_qtensor* A, const w4a4_qtensor* B, uint16_t* Y, int ld
     const int row_bytes = A->cols / 2;
     int rc;
     if (A->format == W4A4_INT4) {
-        rc = make_map(&s->ta, A->codes, A->rows, row_bytes, 64, 128, false);
+        if (A->flags & kFlagInt8Codes)
+            rc = make_map(&s->ta, A->codes, A->rows, A->cols, 128, 128, true);
+        else
+            rc = make_map(&s->ta, A->codes, A->rows, row_bytes, 64, 128, false);
         if (rc == W4A4_OK) rc = make_map(&s->tb, B->codes, B->rows, row_bytes, 64, kBN_I4, false);
     } else if (!decode && use_pair(A)) {
         // each CTA of a pair stages 128 rows of A and 128 rows of B
@@ -251,7 +259,7 @@ int run_gemm(const w4a4_qtensor* A, const w4a4_qtensor* B, uint16_t* Y, int ldy,
     if (rc != W4A4_OK) return rc;
     cudaError_t e;
     if (A->format == W4A4_INT4) {
-        e = launch_gemm_int4(s.ta, s.tb, s.g, num_sms, pdl, st);
+        e = launch_gemm_int4(s.ta, s.tb, s.g, num_sms, pdl, st, (A->flags & kFlagInt8Codes) != 0);
     } else if (decode) {
         s.g.partial = partial;
         s.g.tile_count = tile_count;
@@ -275,6 +283,7 @@ WsLayout ws_layout(int M, int N, int K, int fmt, int nS) {
     const int cols = K + nS;
     size_t cb = 0, sb = 0, s2b = 0;
     w4a4_qtensor_bytes(fmt, M, cols, W4A4_SCALE_TOKEN, &cb, &sb, &s2b);
+    if (fmt == W4A4_INT4) cb *= 2;  // the linear keeps INT4 activations widened to int8
     if (s2b < 8) s2b = 8;
     w.codes = 0;
     w.scales = align256(cb);
@@ -521,6 +530,7 @@ int w4a4_linear(const uint16_t* X, int M, int K, int ldx, const w4a4_qtensor* Wq
     xq.group = fmt == W4A4_INT4 ? Wq->group : group_of(fmt);  // INT4: the weights' scale groups
     xq.scale_mode = fmt == W4A4_NVFP4 ? scale_mode : 0;
     xq.flags = Wq->flags;  // rotated weights: rotate the activations the same way
+    if (fmt == W4A4_INT4) xq.flags |= kFlagInt8Codes;
     xq.codes = base + L.codes;
     xq.scales = base + L.scales;
     xq.s2 = reinterpret_cast<float*>(base + L.s2);

@@ -37,7 +37,7 @@ __host__ __device__ __forceinline__ int decode_kb(int K) { return K % kBK_FP4 ==
 template <int KB>
 struct Dec {
     static constexpr int BN = kBN_DEC;                 // tokens per MMA (16)
-    static constexpr int STAGES = 8 / KB;
+    static constexpr int STAGES = KB == 2 ? 5 : 10;      // ~225 KB of shared memory in flight
     static constexpr int A_BYTES = KB * kBM * 128;     // weight tiles [kb][128 rows][128 B]
     static constexpr int B_BYTES = KB * BN * 128;      // token tiles [kb][16 rows][128 B]
     static constexpr int ATOM = 512;

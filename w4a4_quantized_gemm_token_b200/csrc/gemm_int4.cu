@@ -15,7 +15,10 @@
 // Persistent (one CTA per SM, 128 x 128 output tiles in turn), 14 warps; the
 // MMA and unpack warps run ahead into the next tile while the rescale warps
 // finish and store the previous one:
-//   warp 0 lane 0   TMA producer: packed codes of A and B (64-byte rows).
+//   warp 0 lane 0   TMA producer: packed codes of A and B (64-byte rows); with
+//                   A8 the activations arrive already widened (int8 16 * q,
+//                   written so by the quantizer of the fused linear) straight
+//                   into the swizzled layout the MMA reads, and only B is unpacked.
 //   warp 1          TMEM owner; lane 0 issues 4 MMAs (K=32) per group.
 //   warps 2..5      unpack: nibbles -> int8, written in the 128-byte swizzled
 //                   K-major layout the MMA reads.
@@ -41,17 +44,6 @@ constexpr int THREADS = 14 * 32;
 constexpr int TMEM_COLS = 256;                      // two int32 buffers of 128 columns
 }  // namespace i4
 
-// The 8 nibbles of w (element i in nibble i) as 8 int8 bytes holding 16 * q:
-// each nibble moves to the high half of its byte, whose sign bit is then the
-// nibble's, so no sign extension is needed (5 integer operations per 8
-// elements).  The MMA then yields 256 * P exactly (|256 P| <= 256 * 128 * 64).
-__device__ __forceinline__ void widen8_x16(uint32_t w, uint32_t& o0, uint32_t& o1) {
-    const uint32_t lo = (w << 4) & 0xF0F0F0F0u;  // elements 0,2,4,6
-    const uint32_t hi = w & 0xF0F0F0F0u;         // elements 1,3,5,7
-    o0 = __byte_perm(lo, hi, 0x5140);             // e0 e1 e2 e3
-    o1 = __byte_perm(lo, hi, 0x7362);             // e4 e5 e6 e7
-}
-
 __device__ __forceinline__ uint64_t pack2(float v) {
     const uint32_t u = __float_as_uint(v);
     return ((uint64_t)u << 32) | u;
@@ -76,6 +68,7 @@ __device__ __forceinline__ void rescale2(float& a0, float& a1, uint32_t p0, uint
 
 __device__ __forceinline__ void named_bar(int id, int n) { asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory"); }
 
+template <bool A8>
 __global__ void __launch_bounds__(i4::THREADS, 1)
     gemm_int4_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB, GemmArgs g) {
     using namespace i4;
@@ -151,8 +144,13 @@ __global__ void __launch_bounds__(i4::THREADS, 1)
                     }
                     if (k == g.skip_k_tile) continue;
                     uint8_t* st = smem + s * STAGE;
-                    mbar_arrive_expect_tx(&full[s], 2 * PK_BYTES);
-                    tma_load_2d(st + 2 * UN_BYTES, &tmA, k * 64, m_tile * 128, &full[s]);
+                    if constexpr (A8) {
+                        mbar_arrive_expect_tx(&full[s], UN_BYTES + PK_BYTES);
+                        tma_load_2d(st, &tmA, k * 128, m_tile * 128, &full[s]);
+                    } else {
+                        mbar_arrive_expect_tx(&full[s], 2 * PK_BYTES);
+                        tma_load_2d(st + 2 * UN_BYTES, &tmA, k * 64, m_tile * 128, &full[s]);
+                    }
                     tma_load_2d(st + 2 * UN_BYTES + PK_BYTES, &tmB, k * 64, n_tile * kBN_I4, &full[s]);
                 }
             }
@@ -199,7 +197,7 @@ __global__ void __launch_bounds__(i4::THREADS, 1)
             uint8_t* st = smem + s * STAGE;
             // each warp pass: 8 rows x 64 packed bytes; lane -> row r0 + lane/4, segment lane%4
 #pragma unroll
-            for (int op = 0; op < 2; ++op) {  // A then B
+            for (int op = A8 ? 1 : 0; op < 2; ++op) {  // A (unless it arrived widened), then B
                 const uint8_t* pk = st + 2 * UN_BYTES + op * PK_BYTES;
                 uint8_t* un = st + op * UN_BYTES;
 #pragma unroll
@@ -307,12 +305,13 @@ __global__ void __launch_bounds__(i4::THREADS, 1)
 }
 
 cudaError_t launch_gemm_int4(const CUtensorMap& tmA, const CUtensorMap& tmB, const GemmArgs& g, int num_sms,
-                             bool pdl, cudaStream_t st) {
-    static bool attr_set = false;
-    if (!attr_set) {
-        cudaError_t e = cudaFuncSetAttribute(gemm_int4_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, i4::SMEM);
+                             bool pdl, cudaStream_t st, bool a8) {
+    auto kern = a8 ? gemm_int4_kernel<true> : gemm_int4_kernel<false>;
+    static bool attr_set[2] = {false, false};
+    if (!attr_set[a8]) {
+        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, i4::SMEM);
         if (e != cudaSuccess) return e;
-        attr_set = true;
+        attr_set[a8] = true;
     }
     const int tiles = ((g.M + 127) / 128) * ((g.N + kBN_I4 - 1) / kBN_I4);
     cudaLaunchConfig_t cfg = {};
@@ -325,7 +324,7 @@ cudaError_t launch_gemm_int4(const CUtensorMap& tmA, const CUtensorMap& tmB, con
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = pdl ? 1 : 0;
-    return cudaLaunchKernelEx(&cfg, gemm_int4_kernel, tmA, tmB, g);
+    return cudaLaunchKernelEx(&cfg, kern, tmA, tmB, g);
 }
 
 }  // namespace w4a4

@@ -32,6 +32,7 @@ struct QuantArgs {
     int passes;                // MXFP4: 1, or more for the multi-pass decomposition (pass p
                                // in columns [p*K, (p+1)*K) of codes and scales)
     int group;                 // INT4: elements per scale group (128, 256 or 512)
+    int int8_codes;            // INT4: write codes as int8 16 * q ([M][ldc] bytes, ldc >= K)
     int rot;                   // block-local Walsh-Hadamard rotation: 0 none, 1 activation
                                // side (times 1/block), 2 weight side (unscaled)
 };
@@ -104,8 +105,10 @@ int decode_max_owners(int N, int K, int num_sms);
 // read as 3-D boxes of two K-blocks) when K % 256 == 0, else 1 (2-D boxes).
 int decode_k_blocks(int K);
 // INT4-g128 GEMM on the 8-bit integer MMA with per-group FP32 rescaling.
+// a8: A's codes are int8 (16 * q, row-major [M][K] bytes; tmA a 128-byte
+// swizzled map with 128 x 128-byte boxes) instead of packed nibbles.
 cudaError_t launch_gemm_int4(const CUtensorMap& tmA, const CUtensorMap& tmB, const GemmArgs& g, int num_sms,
-                             bool pdl, cudaStream_t st);
+                             bool pdl, cudaStream_t st, bool a8 = false);
 
 // Tile shapes (shared with the host-side tensor-map set-up).
 constexpr int kBM = 128;          // rows of A per tile

@@ -352,6 +352,17 @@ __device__ __forceinline__ uint64_t smem_desc(uint32_t saddr, uint32_t lbo_bytes
 
 // K-major operand tile whose rows are 128 bytes, stored with the 128-byte
 // swizzle (8-row groups 1024 bytes apart).
+// The 8 nibbles of w (element i in nibble i) as 8 int8 bytes holding 16 * q:
+// each nibble moves to the high half of its byte, whose sign bit is then the
+// nibble's, so no sign extension is needed (5 integer operations per 8
+// elements).  An int8 MMA of two such operands yields 256 * P exactly (|256 P| <= 256 * 512 * 64).
+__device__ __forceinline__ void widen8_x16(uint32_t w, uint32_t& o0, uint32_t& o1) {
+    const uint32_t lo = (w << 4) & 0xF0F0F0F0u;  // elements 0,2,4,6
+    const uint32_t hi = w & 0xF0F0F0F0u;         // elements 1,3,5,7
+    o0 = __byte_perm(lo, hi, 0x5140);             // e0 e1 e2 e3
+    o1 = __byte_perm(lo, hi, 0x7362);             // e4 e5 e6 e7
+}
+
 __device__ __forceinline__ uint64_t desc_kmajor_sw128(uint32_t saddr) { return smem_desc(saddr, 16, 1024, 2); }
 
 // 32 rows x 16 bytes, contiguous (no swizzle): four 8-row core matrices 128 bytes apart.

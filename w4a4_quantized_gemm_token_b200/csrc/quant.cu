@@ -423,6 +423,7 @@ __global__ void __launch_bounds__(256, 4) quant_rows_kernel(QuantArgs a, int row
         else bmax = (token && live) ? bm[it] : bmax16(w);
 
         uint32_t w0 = 0, w1 = 0;  // 16 codes
+        bool stored = false;      // INT4 codes already written widened
         if constexpr (FMT == FMT_NVFP4) {
             const RowConsts k = rc[i < nrows ? i : 0];
             // block scale E4M3(RN(RN(bmax/6)/s2)) and quotients x/(scale*s2), by refined
@@ -573,8 +574,17 @@ __global__ void __launch_bounds__(256, 4) quant_rows_kernel(QuantArgs a, int row
                 w1 = 0;
             }
             if (valid && (c & (R8 - 1)) == 0) a.sfi[(size_t)(c / R8) * a.sfi_ld + r] = sc;
+            if (a.int8_codes) {  // already widened for the GEMM: 16 bytes of 16 * q
+                if (live) {
+                    uint32_t o[4];
+                    widen8_x16(w0, o[0], o[1]);
+                    widen8_x16(w1, o[2], o[3]);
+                    *reinterpret_cast<uint4*>(a.codes + (size_t)r * a.ldc + 16 * c) = make_uint4(o[0], o[1], o[2], o[3]);
+                }
+                stored = true;
+            }
         }
-        if (live) *reinterpret_cast<uint2*>(a.codes + (size_t)r * a.ldc + 8 * c) = make_uint2(w0, w1);
+        if (live && !stored) *reinterpret_cast<uint2*>(a.codes + (size_t)r * a.ldc + 8 * c) = make_uint2(w0, w1);
         i += di;
         c += dc;
         if (c >= nchunk) {

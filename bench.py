@@ -43,8 +43,8 @@ INT8_PER_BF16 = 2.0       # nominal dense INT8 / BF16 (4.5 / 2.25)
 # dominant kernel, averaged over the five GEMM launches of one step, from the ncu
 # launch list summarised in profiles/launch_list_llama70b_layer_m4096.md; valid
 # only for the kernel source it was measured on (else reported as null).
-PROFILED_TRAFFIC = {"sources": ("gemm_fp4_pair.cu", "ptx.cuh"), "sha256_16": "c576354968618da2",
-                    "bytes_per_launch": 295.0e6}
+PROFILED_TRAFFIC = {"sources": ("gemm_fp4_pair.cu", "ptx.cuh"), "sha256_16": "4f89a520741370e8",
+                    "bytes_per_launch": 295.4e6}
 
 
 def profiled_traffic():

@@ -494,6 +494,29 @@ def extra_rows(args, dev, stream, P):
             del X, Y, ws
         del variants, fl
 
+    # the fused per-token NVFP4 linear over the Llama layer at the other token
+    # counts of the workload (256: the one-CTA GEMM; 16384: the CTA pair)
+    for Ms in ((256, 16384) if want("tokens") else ()):
+        lay = []
+        for li, (name, K, N) in enumerate(LLAMA):
+            Wq = w4.quantize_weight(to_dev(synth.weights("llama2_70b", N, K, seed=0, tensor_id=100 + li), dev),
+                                    w4.NVFP4)
+            X = to_dev(synth.activations("llama2_70b", Ms, K, seed=0, tensor_id=200 + li), dev)
+            Y = torch.empty(Ms, N, dtype=torch.bfloat16, device=dev)
+            ws = torch.empty(w4.linear_workspace(Ms, N, K, w4.NVFP4), dtype=torch.uint8, device=dev)
+            lay.append((K, N, Wq, X, Y, ws))
+
+        def layer_step():
+            for (K, N, Wq, X, Y, ws) in lay:
+                w4.linear(X, Wq, w4.SCALE_TOKEN, Y=Y, ws=ws)
+        for _ in range(max(3, args.warmup)):
+            layer_step()
+        ms = time_loop(layer_step, max(3, min(args.steps, 10)), stream)
+        fl = sum(2.0 * Ms * N * K for (K, N, *_r) in lay)
+        out[f"linear_nvfp4_llama_layer_m{Ms}"] = {"TFLOPS": round(fl / (ms * 1e-3) / 1e12, 1),
+                                                  "ms": round(ms, 3)}
+        del lay
+
     # multi-pass MXFP4 (two passes) on the Llama qkv shape: the quantizer alone
     # (L2 flushed before each launch) and the linear, beside one-pass MXFP4
     if want("msd"):
@@ -585,7 +608,7 @@ def main():
     ap.add_argument("--cpu-rows", type=int, default=8, help="cpu_baseline sample: tokens")
     ap.add_argument("--cpu-cols", type=int, default=4096, help="cpu_baseline sample: output columns")
     ap.add_argument("--no-rows", action="store_true", help="skip the secondary rows")
-    ap.add_argument("--only", choices=["gemm", "quant", "decode", "int4", "aug", "mxfp4", "segments", "msd", "hadamard"], default=None,
+    ap.add_argument("--only", choices=["gemm", "quant", "decode", "int4", "aug", "mxfp4", "segments", "msd", "hadamard", "tokens"], default=None,
                     help="run only one secondary row (for profiling) and print it")
     ap.add_argument("--no-cpu", action="store_true", help="skip the oracle CPU baseline")
     ap.add_argument("--shape", default=None, help="--only gemm: one Llama linear (qkv, o, w1, w3, w2)")

@@ -779,7 +779,9 @@ __global__ void __launch_bounds__(1024) compact_kernel(const int* selected, int 
 // that takes IEEE division throughout (a CTA-uniform branch).  Rows
 // M .. rows_pad-1 write the zero scales of the 128-row atoms' padding.
 // ---------------------------------------------------------------------------
-template <int J>
+// ROT: every 16-element block rotated first (rotate_item; a block is one
+// item, so no lane exchange; a.rot 1 = activation side, 2 = weight side).
+template <int J, bool ROT>
 __global__ void __launch_bounds__(J <= 2 ? 1024 : 768) quant_nvfp4_token_kernel(QuantArgs a, int nb) {
     pdl_launch_dependents();
     pdl_wait();  // X and the words to clear may belong to the preceding launch
@@ -813,6 +815,7 @@ __global__ void __launch_bounds__(J <= 2 ? 1024 : 768) quant_nvfp4_token_kernel(
         if (!mbar_wait(&bars[b], (i / nb) & 1, 2000000000ull, abort_flag)) break;
         const uint4* xr = reinterpret_cast<const uint4*>(qring + (size_t)b * row_bytes);
         uint32_t w[J][8];
+        float vr[ROT ? J : 1][16];  // ROT: the rotated values of each item
 #pragma unroll
         for (int j = 0; j < J; ++j) {
             const int it = t + T * j;
@@ -827,7 +830,12 @@ __global__ void __launch_bounds__(J <= 2 ? 1024 : 768) quant_nvfp4_token_kernel(
         float bm[J], m = 0.0f;
 #pragma unroll
         for (int j = 0; j < J; ++j) {
-            bm[j] = bmax16(w[j]);
+            if constexpr (ROT) {
+                rotate_item<16>(w[j], vr[j], 0, a.rot == 1);
+                bm[j] = absmax16(vr[j]);
+            } else {
+                bm[j] = bmax16(w[j]);
+            }
             m = fmaxf(m, bm[j]);
         }
         m = warp_max(m);
@@ -848,13 +856,23 @@ __global__ void __launch_bounds__(J <= 2 ? 1024 : 768) quant_nvfp4_token_kernel(
                 sb = e4m3_rn_sat(div_refined(u, s2, rinv));
                 const float d = sb ? __fmul_rn(e4m3_value((uint8_t)sb), s2) : 1.0f;
                 const float y = __frcp_rn(d);
-                w0 = e2m1x8_fast(w[j], pack2(-y), pack2(d));
-                w1 = e2m1x8_fast(w[j] + 4, pack2(-y), pack2(d));
+                if constexpr (ROT) {
+                    w0 = e2m1x8_fast_f(vr[j], pack2(-y), pack2(d));
+                    w1 = e2m1x8_fast_f(vr[j] + 8, pack2(-y), pack2(d));
+                } else {
+                    w0 = e2m1x8_fast(w[j], pack2(-y), pack2(d));
+                    w1 = e2m1x8_fast(w[j] + 4, pack2(-y), pack2(d));
+                }
             } else {
                 sb = e4m3_rn_sat(__fdiv_rn(__fdiv_rn(bm[j], 6.0f), s2));
                 const float d = sb ? __fmul_rn(e4m3_value((uint8_t)sb), s2) : 1.0f;
-                w0 = e2m1x8_exact(make_uint4(w[j][0], w[j][1], w[j][2], w[j][3]), d);
-                w1 = e2m1x8_exact(make_uint4(w[j][4], w[j][5], w[j][6], w[j][7]), d);
+                if constexpr (ROT) {
+                    w0 = e2m1x8_exact_f(vr[j], d);
+                    w1 = e2m1x8_exact_f(vr[j] + 8, d);
+                } else {
+                    w0 = e2m1x8_exact(make_uint4(w[j][0], w[j][1], w[j][2], w[j][3]), d);
+                    w1 = e2m1x8_exact(make_uint4(w[j][4], w[j][5], w[j][6], w[j][7]), d);
+                }
             }
             if (sb == 0) {
                 w0 = 0;
@@ -898,6 +916,18 @@ static cudaError_t launch_dep(void (*kern)(Args...), dim3 grid, dim3 block, size
     return cudaLaunchKernelEx(&cfg, kern, args...);
 }
 
+template <int J, bool ROT>
+static cudaError_t launch_tok(const QuantArgs& b, int grid, int T, size_t smem, int nb, cudaStream_t st) {
+    static size_t attr = 0;
+    if (smem > 48 * 1024 && smem > attr) {
+        const cudaError_t e =
+            cudaFuncSetAttribute(quant_nvfp4_token_kernel<J, ROT>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e != cudaSuccess) return e;
+        attr = smem;
+    }
+    return launch_dep(quant_nvfp4_token_kernel<J, ROT>, dim3(grid), dim3(T), smem, st, b, nb);
+}
+
 static cudaError_t launch_nvfp4_token(const QuantArgs& a, int rows_pad, int num_sms, cudaStream_t st) {
     // J items (32 J bytes of the row) per thread: two, so that the resident
     // CTAs bring enough warps to hide the per-item latency (at most 1024
@@ -910,7 +940,7 @@ static cudaError_t launch_nvfp4_token(const QuantArgs& a, int rows_pad, int num_
     // ring of at least three row buffers each (two rows in flight while one is
     // computed), within about 200 KB of shared memory per SM
     const int row_bytes = a.K * 2;
-    const int regs = J == 1 ? 48 : J == 2 ? 56 : 72;
+    const int regs = (J == 1 ? 48 : J == 2 ? 56 : 72) + (a.rot ? 8 : 0);
     int per_sm = 65536 / (T * regs);
     const int by_smem = (200 * 1024) / (3 * row_bytes);
     per_sm = per_sm < by_smem ? per_sm : by_smem;
@@ -923,20 +953,10 @@ static cudaError_t launch_nvfp4_token(const QuantArgs& a, int rows_pad, int num_
     if (grid > rows_pad) grid = rows_pad;
     QuantArgs b = a;
     b.rows_pad = rows_pad;
-    cudaError_t e = cudaSuccess;
-    if (J == 1) {
-        static size_t attr = 0;
-        if (smem > 48 * 1024 && smem > attr) e = cudaFuncSetAttribute(quant_nvfp4_token_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem), attr = smem;
-        if (e == cudaSuccess) e = launch_dep(quant_nvfp4_token_kernel<1>, dim3(grid), dim3(T), smem, st, b, nb);
-    } else if (J == 2) {
-        static size_t attr = 0;
-        if (smem > 48 * 1024 && smem > attr) e = cudaFuncSetAttribute(quant_nvfp4_token_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem), attr = smem;
-        if (e == cudaSuccess) e = launch_dep(quant_nvfp4_token_kernel<2>, dim3(grid), dim3(T), smem, st, b, nb);
-    } else {
-        static size_t attr = 0;
-        if (smem > 48 * 1024 && smem > attr) e = cudaFuncSetAttribute(quant_nvfp4_token_kernel<4>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem), attr = smem;
-        if (e == cudaSuccess) e = launch_dep(quant_nvfp4_token_kernel<4>, dim3(grid), dim3(T), smem, st, b, nb);
-    }
+    cudaError_t e;
+    if (J == 1) e = a.rot ? launch_tok<1, true>(b, grid, T, smem, nb, st) : launch_tok<1, false>(b, grid, T, smem, nb, st);
+    else if (J == 2) e = a.rot ? launch_tok<2, true>(b, grid, T, smem, nb, st) : launch_tok<2, false>(b, grid, T, smem, nb, st);
+    else e = launch_tok<4, false>(b, grid, T, smem, nb, st);
     return e != cudaSuccess ? e : cudaGetLastError();
 }
 
@@ -972,6 +992,8 @@ static cudaError_t launch_quant_fmt(const QuantArgs& a, int rows_pad, int num_sm
 cudaError_t launch_quant(int fmt, bool gather, const QuantArgs& a, int rows_pad, int num_sms, cudaStream_t st) {
     if (a.rot) {  // block-local rotation (no gather, one pass)
         if (gather || a.passes > 1) return cudaErrorInvalidValue;
+        if (fmt == FMT_NVFP4 && a.mode == 1 && !a.static_s2 && a.K == a.K_src && a.K <= 32768 && !a.int8_codes)
+            return launch_nvfp4_token(a, rows_pad, num_sms, st);
         if (fmt == FMT_NVFP4) return launch_quant_fmt<FMT_NVFP4, false, false, true>(a, rows_pad, num_sms, st);
         if (fmt == FMT_MXFP4) return launch_quant_fmt<FMT_MXFP4, false, false, true>(a, rows_pad, num_sms, st);
         return launch_quant_fmt<FMT_INT4, false, false, true>(a, rows_pad, num_sms, st);

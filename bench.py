@@ -517,6 +517,29 @@ def extra_rows(args, dev, stream, P):
                                                   "ms": round(ms, 3)}
         del lay
 
+    # the 300M SwiGLU decoder layer at M = 4096, NVFP4 with a tensor scale on
+    # both sides (the activation scale from an amax pass on every call)
+    if want("swiglu"):
+        lay = []
+        for li, (name, K, N) in enumerate(synth.SHAPES["swiglu300m"]):
+            Wq = w4.quantize_weight(to_dev(synth.weights("swiglu300m", N, K, seed=0, tensor_id=100 + li), dev),
+                                    w4.NVFP4)
+            X = to_dev(synth.activations("swiglu300m", args.tokens, K, seed=0, tensor_id=200 + li), dev)
+            Y = torch.empty(args.tokens, N, dtype=torch.bfloat16, device=dev)
+            ws = torch.empty(w4.linear_workspace(args.tokens, N, K, w4.NVFP4), dtype=torch.uint8, device=dev)
+            lay.append((K, N, Wq, X, Y, ws))
+
+        def sw_step():
+            for (K, N, Wq, X, Y, ws) in lay:
+                w4.linear(X, Wq, w4.SCALE_TENSOR, Y=Y, ws=ws)
+        for _ in range(max(3, args.warmup)):
+            sw_step()
+        ms = time_loop(sw_step, max(5, min(args.steps, 20)), stream)
+        fl = sum(2.0 * args.tokens * N * K for (K, N, *_r) in lay)
+        out[f"linear_nvfp4_tensor_swiglu300m_m{args.tokens}"] = {"TFLOPS": round(fl / (ms * 1e-3) / 1e12, 1),
+                                                                 "ms": round(ms, 3)}
+        del lay
+
     # multi-pass MXFP4 (two passes) on the Llama qkv shape: the quantizer alone
     # (L2 flushed before each launch) and the linear, beside one-pass MXFP4
     if want("msd"):
@@ -608,7 +631,7 @@ def main():
     ap.add_argument("--cpu-rows", type=int, default=8, help="cpu_baseline sample: tokens")
     ap.add_argument("--cpu-cols", type=int, default=4096, help="cpu_baseline sample: output columns")
     ap.add_argument("--no-rows", action="store_true", help="skip the secondary rows")
-    ap.add_argument("--only", choices=["gemm", "quant", "decode", "int4", "aug", "mxfp4", "segments", "msd", "hadamard", "tokens"], default=None,
+    ap.add_argument("--only", choices=["gemm", "quant", "decode", "int4", "aug", "mxfp4", "segments", "msd", "hadamard", "tokens", "swiglu"], default=None,
                     help="run only one secondary row (for profiling) and print it")
     ap.add_argument("--no-cpu", action="store_true", help="skip the oracle CPU baseline")
     ap.add_argument("--shape", default=None, help="--only gemm: one Llama linear (qkv, o, w1, w3, w2)")

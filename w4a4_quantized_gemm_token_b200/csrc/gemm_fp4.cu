@@ -415,12 +415,9 @@ template <bool NV, int KB>
 static cudaError_t launch_dec_t(const CUtensorMap& tmW, const CUtensorMap& tmX, const GemmArgs& g0, int num_sms,
                                 cudaStream_t st) {
     auto kern = gemm_fp4_decode_kernel<NV, KB>;
-    static bool attr_set = false;
-    if (!attr_set) {
-        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Dec<KB>::SMEM);
-        if (e != cudaSuccess) return e;
-        attr_set = true;
-    }
+    static SmemAttrCache attr;
+    cudaError_t e = ensure_dynamic_smem(reinterpret_cast<const void*>(kern), Dec<KB>::SMEM, attr);
+    if (e != cudaSuccess) return e;
     GemmArgs g = g0;
     const int G = decode_grid(g.N, g.K, num_sms);
     g.splits = decode_max_owners(g.N, g.K, num_sms);  // slots per weight tile in the workspace

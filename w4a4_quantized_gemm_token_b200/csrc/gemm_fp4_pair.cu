@@ -345,17 +345,16 @@ cudaError_t launch_gemm_fp4_pair(bool nvfp4, const CUtensorMap& tmA, const CUten
     const int v = !nvfp4 ? 0 : g.s2b_per_row ? 2 : 1;
     auto kern = v == 0 ? gemm_fp4_pair_kernel<false, false>
                        : v == 1 ? gemm_fp4_pair_kernel<true, false> : gemm_fp4_pair_kernel<true, true>;
-    static bool attr_set[3] = {false, false, false};
-    if (!attr_set[v]) {
-        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             nvfp4 ? pp::Cfg<true>::SMEM : pp::Cfg<false>::SMEM);
-        if (e != cudaSuccess) return e;
-        attr_set[v] = true;
-    }
+    static SmemAttrCache smem_attr[3];
+    cudaError_t e0 = ensure_dynamic_smem(reinterpret_cast<const void*>(kern),
+                                         nvfp4 ? pp::Cfg<true>::SMEM : pp::Cfg<false>::SMEM, smem_attr[v]);
+    if (e0 != cudaSuccess) return e0;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kAttrDevices) return cudaErrorInvalidDevice;
     const int tiles = ((g.M + pp::BM - 1) / pp::BM) * ((g.N + pp::BN - 1) / pp::BN);
     // as many pairs as can be resident at once (a persistent grid must not queue)
-    static int resident[3] = {0, 0, 0};
-    if (!resident[v]) {
+    static std::atomic<int> resident[kAttrDevices][3];  // per device (zero-initialised)
+    if (!resident[dev][v].load(std::memory_order_acquire)) {
         cudaLaunchConfig_t q = {};
         q.gridDim = dim3(2 * (num_sms / 2));
         q.blockDim = dim3(pp::THREADS);
@@ -372,10 +371,11 @@ cudaError_t launch_gemm_fp4_pair(bool nvfp4, const CUtensorMap& tmA, const CUten
             cudaGetLastError();
             n = num_sms / 2;
         }
-        resident[v] = n;
+        resident[dev][v].store(n, std::memory_order_release);
     }
     int pairs = tiles < num_sms / 2 ? tiles : num_sms / 2;
-    if (pairs > resident[v]) pairs = resident[v];
+    const int res = resident[dev][v].load(std::memory_order_acquire);
+    if (pairs > res) pairs = res;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(2 * pairs);
     cfg.blockDim = dim3(pp::THREADS);

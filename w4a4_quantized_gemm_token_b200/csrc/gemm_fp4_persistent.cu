@@ -286,12 +286,9 @@ cudaError_t launch_gemm_fp4(bool nvfp4, const CUtensorMap& tmA, const CUtensorMa
     const int v = !nvfp4 ? 0 : g.s2b_per_row ? 2 : 1;
     auto kern = v == 0 ? gemm_fp4_persistent_kernel<false, false>
                        : v == 1 ? gemm_fp4_persistent_kernel<true, false> : gemm_fp4_persistent_kernel<true, true>;
-    static bool attr_set[3] = {false, false, false};
-    if (!attr_set[v]) {
-        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, pf::SMEM);
-        if (e != cudaSuccess) return e;
-        attr_set[v] = true;
-    }
+    static SmemAttrCache smem_attr[3];
+    const cudaError_t e0 = ensure_dynamic_smem(reinterpret_cast<const void*>(kern), pf::SMEM, smem_attr[v]);
+    if (e0 != cudaSuccess) return e0;
     const int tiles = ((g.M + kBM - 1) / kBM) * ((g.N + pf::BN - 1) / pf::BN);
     const int grid = tiles < num_sms ? tiles : num_sms;
     cudaLaunchConfig_t cfg = {};

@@ -307,12 +307,9 @@ __global__ void __launch_bounds__(i4::THREADS, 1)
 cudaError_t launch_gemm_int4(const CUtensorMap& tmA, const CUtensorMap& tmB, const GemmArgs& g, int num_sms,
                              bool pdl, cudaStream_t st, bool a8) {
     auto kern = a8 ? gemm_int4_kernel<true> : gemm_int4_kernel<false>;
-    static bool attr_set[2] = {false, false};
-    if (!attr_set[a8]) {
-        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, i4::SMEM);
-        if (e != cudaSuccess) return e;
-        attr_set[a8] = true;
-    }
+    static SmemAttrCache smem_attr[2];
+    const cudaError_t e0 = ensure_dynamic_smem(reinterpret_cast<const void*>(kern), i4::SMEM, smem_attr[a8]);
+    if (e0 != cudaSuccess) return e0;
     const int tiles = ((g.M + 127) / 128) * ((g.N + kBN_I4 - 1) / kBN_I4);
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(tiles < num_sms ? tiles : num_sms);  // persistent: one CTA per SM

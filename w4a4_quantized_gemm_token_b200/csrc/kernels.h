@@ -1,11 +1,33 @@
 // Internal interface between the C-ABI layer (api.cu) and the kernels.
 #pragma once
+#include <atomic>
 #include <cstddef>
 #include <cstdint>
 #include <cuda.h>
 #include <cuda_runtime.h>
 
 namespace w4a4 {
+
+// Per-device record that a kernel's dynamic shared-memory limit has been
+// raised (cudaFuncSetAttribute acts on the current device); safe to share
+// between host threads.
+constexpr int kAttrDevices = 64;
+struct SmemAttrCache {
+    std::atomic<size_t> bytes[kAttrDevices] = {};
+};
+inline cudaError_t ensure_dynamic_smem(const void* func, size_t bytes, SmemAttrCache& c) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= kAttrDevices) return cudaErrorInvalidDevice;
+    if (bytes <= 48 * 1024 || c.bytes[dev].load(std::memory_order_acquire) >= bytes) return cudaSuccess;
+    e = cudaFuncSetAttribute(func, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+    if (e != cudaSuccess) return e;
+    size_t cur = c.bytes[dev].load(std::memory_order_relaxed);
+    while (cur < bytes && !c.bytes[dev].compare_exchange_weak(cur, bytes, std::memory_order_release)) {
+    }
+    return cudaSuccess;
+}
 
 enum { FMT_NVFP4 = 0, FMT_MXFP4 = 1, FMT_INT4 = 2 };
 

@@ -918,13 +918,10 @@ static cudaError_t launch_dep(void (*kern)(Args...), dim3 grid, dim3 block, size
 
 template <int J, bool ROT>
 static cudaError_t launch_tok(const QuantArgs& b, int grid, int T, size_t smem, int nb, cudaStream_t st) {
-    static size_t attr = 0;
-    if (smem > 48 * 1024 && smem > attr) {
-        const cudaError_t e =
-            cudaFuncSetAttribute(quant_nvfp4_token_kernel<J, ROT>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        if (e != cudaSuccess) return e;
-        attr = smem;
-    }
+    static SmemAttrCache smem_attr;
+    const cudaError_t e =
+        ensure_dynamic_smem(reinterpret_cast<const void*>(quant_nvfp4_token_kernel<J, ROT>), smem, smem_attr);
+    if (e != cudaSuccess) return e;
     return launch_dep(quant_nvfp4_token_kernel<J, ROT>, dim3(grid), dim3(T), smem, st, b, nb);
 }
 
@@ -973,12 +970,9 @@ static cudaError_t launch_quant_fmt(const QuantArgs& a, int rows_pad, int num_sm
                         (FMT == FMT_NVFP4 ? 4 * (size_t)rpc * (a.K / 16) : 0) + 16;
     if (smem > 200 * 1024) return cudaErrorInvalidValue;
     auto kern = quant_rows_kernel<FMT, GATHER, MULTI, ROT>;
-    static size_t attr = 0;
-    if (smem > 48 * 1024 && smem > attr) {
-        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        if (e != cudaSuccess) return e;
-        attr = smem;
-    }
+    static SmemAttrCache smem_attr;
+    const cudaError_t e0 = ensure_dynamic_smem(reinterpret_cast<const void*>(kern), smem, smem_attr);
+    if (e0 != cudaSuccess) return e0;
     const int items = rpc * (a.K / 16);
     const int T = items < 256 ? (items + 31) / 32 * 32 : 256;
     const int nblocks = (rows_pad + rpc - 1) / rpc;

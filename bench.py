@@ -43,8 +43,8 @@ INT8_PER_BF16 = 2.0       # nominal dense INT8 / BF16 (4.5 / 2.25)
 # dominant kernel, averaged over the five GEMM launches of one step, from the ncu
 # launch list summarised in profiles/launch_list_llama70b_layer_m4096.md; valid
 # only for the kernel source it was measured on (else reported as null).
-PROFILED_TRAFFIC = {"sources": ("gemm_fp4_pair.cu", "ptx.cuh"), "sha256_16": "4f89a520741370e8",
-                    "bytes_per_launch": 295.4e6}
+PROFILED_TRAFFIC = {"sources": ("gemm_fp4_pair.cu", "ptx.cuh"), "sha256_16": "718b7937ac7f9a8f",
+                    "bytes_per_launch": 295.0e6}
 
 
 def profiled_traffic():
@@ -494,9 +494,10 @@ def extra_rows(args, dev, stream, P):
             del X, Y, ws
         del variants, fl
 
-    # the fused per-token NVFP4 linear over the Llama layer at the other token
-    # counts of the workload (256: the one-CTA GEMM; 16384: the CTA pair)
-    for Ms in ((256, 16384) if want("tokens") else ()):
+    # the fused per-token NVFP4 linear over the Llama layer at other token
+    # counts (all on the CTA pair: 256 and 1024 fill few waves of 256 x 256
+    # tiles and stream the weights from memory once; 16384 runs many waves)
+    for Ms in ((256, 1024, 16384) if want("tokens") else ()):
         lay = []
         for li, (name, K, N) in enumerate(LLAMA):
             Wq = w4.quantize_weight(to_dev(synth.weights("llama2_70b", N, K, seed=0, tensor_id=100 + li), dev),

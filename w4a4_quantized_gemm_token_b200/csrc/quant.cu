@@ -10,6 +10,7 @@
 // words gathered by shuffles into the MMA's 128x4 scale atoms.
 #include <cstdint>
 #include <cuda_bf16.h>
+#include <type_traits>
 #include <cuda_fp8.h>
 
 #include "kernels.h"
@@ -604,20 +605,37 @@ __global__ void __launch_bounds__(256, 4) quant_rows_kernel(QuantArgs a, int row
 
 // ---------------------------------------------------------------------------
 // Tensor amax: max |x| over X[M, K] into *out (as float bits; *out must start
-// at 0).  Grid-stride over 16-byte vectors of each row.
+// at 0).  Flat index i over the 16-byte vectors of the rows (row i / (K/8));
+// each thread has four vectors in flight per step (a grid stride apart, so a
+// warp's loads stay contiguous).  WIDE: 64-bit indices for tensors of 2^31 or
+// more vectors.
 // ---------------------------------------------------------------------------
+__device__ __forceinline__ float absmax8(uint4 q) {
+    return fmaxf(fmaxf(fmaxf(fabsf(bf16lo(q.x)), fabsf(bf16hi(q.x))), fmaxf(fabsf(bf16lo(q.y)), fabsf(bf16hi(q.y)))),
+                 fmaxf(fmaxf(fabsf(bf16lo(q.z)), fabsf(bf16hi(q.z))), fmaxf(fabsf(bf16lo(q.w)), fabsf(bf16hi(q.w)))));
+}
+
+template <bool WIDE>
 __global__ void __launch_bounds__(256) amax_kernel(const uint16_t* X, int M, int K, int ldx, float* out) {
     pdl_launch_dependents();
-    const int vec_per_row = K / 8;
-    const long long total = (long long)M * vec_per_row;
+    using I = typename std::conditional<WIDE, unsigned long long, unsigned>::type;
+    const I vpr = (I)(K / 8);
+    const I total = (I)M * vpr;
+    const I S = (I)gridDim.x * blockDim.x;
     float m = 0.0f;
-    for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < total;
-         i += (long long)gridDim.x * blockDim.x) {
-        const long long r = i / vec_per_row;
-        const int v = (int)(i - r * vec_per_row);
-        uint4 q = __ldg(reinterpret_cast<const uint4*>(X + r * ldx) + v);
-        m = fmaxf(m, fmaxf(fmaxf(fabsf(bf16lo(q.x)), fabsf(bf16hi(q.x))), fmaxf(fabsf(bf16lo(q.y)), fabsf(bf16hi(q.y)))));
-        m = fmaxf(m, fmaxf(fmaxf(fabsf(bf16lo(q.z)), fabsf(bf16hi(q.z))), fmaxf(fabsf(bf16lo(q.w)), fabsf(bf16hi(q.w)))));
+    for (I i0 = (I)blockIdx.x * blockDim.x + threadIdx.x; i0 < total; i0 += 4 * S) {
+        uint4 q[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            const I i = i0 + (I)u * S;
+            q[u] = make_uint4(0, 0, 0, 0);
+            if (i < total) {
+                const I r = i / vpr;
+                q[u] = __ldg(reinterpret_cast<const uint4*>(X + (size_t)r * ldx) + (i - r * vpr));
+            }
+        }
+#pragma unroll
+        for (int u = 0; u < 4; ++u) m = fmaxf(m, absmax8(q[u]));
     }
     m = warp_max(m);
     __shared__ float red[8];
@@ -763,7 +781,8 @@ __global__ void __launch_bounds__(1024) compact_kernel(const int* selected, int 
 // Host launchers
 // ---------------------------------------------------------------------------
 // ---------------------------------------------------------------------------
-// NVFP4 with a dynamic per-token scale (the activation hot path).  Persistent
+// NVFP4 with a dynamic per-token scale (the activation hot path), or with the
+// dynamic tensor scale of an amax pass (TENSOR mode).  Persistent
 // CTAs walk rows r = blockIdx.x, +gridDim.x, ...; thread 0 keeps the next
 // NB-1 rows in flight as bulk copies into a ring of shared-memory row
 // buffers, so each SM has its loads outstanding while it computes.  For the
@@ -781,7 +800,8 @@ __global__ void __launch_bounds__(1024) compact_kernel(const int* selected, int 
 // ---------------------------------------------------------------------------
 // ROT: every 16-element block rotated first (rotate_item; a block is one
 // item, so no lane exchange; a.rot 1 = activation side, 2 = weight side).
-template <int J, bool ROT>
+// TENSOR: one s2 for the whole tensor (see below) instead of one per row.
+template <int J, bool ROT, bool TENSOR>
 __global__ void __launch_bounds__(J <= 2 ? 1024 : 768) quant_nvfp4_token_kernel(QuantArgs a, int nb) {
     pdl_launch_dependents();
     pdl_wait();  // X and the words to clear may belong to the preceding launch
@@ -798,6 +818,11 @@ __global__ void __launch_bounds__(J <= 2 ? 1024 : 768) quant_nvfp4_token_kernel(
     const int G = gridDim.x;
     // rows of this CTA that are loaded: blockIdx.x + i*G < M
     const int nlive = a.M > (int)blockIdx.x ? (a.M - 1 - (int)blockIdx.x) / G + 1 : 0;
+    // TENSOR mode: one s2 from the amax pass that precedes this launch; every
+    // block amax is at most that amax, so the quotients keep the ranges the
+    // refined division needs, as with a row's own s2
+    const float ts2 = TENSOR ? nvfp4_s2(*a.tensor_amax) : 1.0f;
+    if (TENSOR && blockIdx.x == 0 && threadIdx.x == 0) a.s2_out[0] = ts2;
     auto issue = [&](int i) {
         const int b = i % nb, r = blockIdx.x + i * G;
         mbar_arrive_expect_tx(&bars[b], (uint32_t)row_bytes);
@@ -838,14 +863,18 @@ __global__ void __launch_bounds__(J <= 2 ? 1024 : 768) quant_nvfp4_token_kernel(
             }
             m = fmaxf(m, bm[j]);
         }
-        m = warp_max(m);
-        if (lane == 0) wmax[i & 1][warp] = m;
+        if constexpr (!TENSOR) {
+            m = warp_max(m);
+            if (lane == 0) wmax[i & 1][warp] = m;
+        }
         __syncthreads();  // (also: every thread has its row data in registers)
         if (t == 0 && i + nb < nlive) issue(i + nb);  // the buffer is free again
-        const float amax = warp_max(lane < nwarps ? wmax[i & 1][lane] : 0.0f);
-        const float s2 = nvfp4_s2(amax);
+        float s2 = ts2;
+        if constexpr (!TENSOR) {
+            s2 = nvfp4_s2(warp_max(lane < nwarps ? wmax[i & 1][lane] : 0.0f));
+            if (t == 0) a.s2_out[r] = s2;
+        }
         const bool fast = s2 >= 0x1p-100f;  // the same for the whole CTA
-        if (t == 0) a.s2_out[r] = s2;
         const float rinv = __frcp_rn(s2);
 #pragma unroll
         for (int j = 0; j < J; ++j) {
@@ -917,12 +946,24 @@ static cudaError_t launch_dep(void (*kern)(Args...), dim3 grid, dim3 block, size
 }
 
 template <int J, bool ROT>
-static cudaError_t launch_tok(const QuantArgs& b, int grid, int T, size_t smem, int nb, cudaStream_t st) {
+static const void* tok_kernel(bool tensor) {
+    return tensor ? reinterpret_cast<const void*>(quant_nvfp4_token_kernel<J, ROT, true>)
+                  : reinterpret_cast<const void*>(quant_nvfp4_token_kernel<J, ROT, false>);
+}
+
+template <int J, bool ROT, bool TENSOR>
+static cudaError_t launch_tok_mode(const QuantArgs& b, int grid, int T, size_t smem, int nb, cudaStream_t st) {
     static SmemAttrCache smem_attr;
-    const cudaError_t e =
-        ensure_dynamic_smem(reinterpret_cast<const void*>(quant_nvfp4_token_kernel<J, ROT>), smem, smem_attr);
+    auto kern = quant_nvfp4_token_kernel<J, ROT, TENSOR>;
+    const cudaError_t e = ensure_dynamic_smem(reinterpret_cast<const void*>(kern), smem, smem_attr);
     if (e != cudaSuccess) return e;
-    return launch_dep(quant_nvfp4_token_kernel<J, ROT>, dim3(grid), dim3(T), smem, st, b, nb);
+    return launch_dep(kern, dim3(grid), dim3(T), smem, st, b, nb);
+}
+
+template <int J, bool ROT>
+static cudaError_t launch_tok(const QuantArgs& b, int grid, int T, size_t smem, int nb, cudaStream_t st) {
+    return b.mode == 0 ? launch_tok_mode<J, ROT, true>(b, grid, T, smem, nb, st)
+                       : launch_tok_mode<J, ROT, false>(b, grid, T, smem, nb, st);
 }
 
 static cudaError_t launch_nvfp4_token(const QuantArgs& a, int rows_pad, int num_sms, cudaStream_t st) {
@@ -933,12 +974,26 @@ static cudaError_t launch_nvfp4_token(const QuantArgs& a, int rows_pad, int num_
     const int J = items < 64 ? 1 : items <= 2048 ? 2 : 4;
     int T = (items + J - 1) / J;
     T = (T + 31) / 32 * 32;
-    // resident CTAs per SM from registers (about 44 + 8 J per thread) and from a
-    // ring of at least three row buffers each (two rows in flight while one is
-    // computed), within about 200 KB of shared memory per SM
+    // resident CTAs per SM from the kernel's registers (allocated per warp in
+    // units of 256) and from a ring of at least three row buffers each (two
+    // rows in flight while one is computed), within about 200 KB of shared
+    // memory per SM
     const int row_bytes = a.K * 2;
-    const int regs = (J == 1 ? 48 : J == 2 ? 56 : 72) + (a.rot ? 8 : 0);
-    int per_sm = 65536 / (T * regs);
+    const bool tensor = a.mode == 0;
+    const void* kern = J == 1 ? (a.rot ? tok_kernel<1, true>(tensor) : tok_kernel<1, false>(tensor))
+                     : J == 2 ? (a.rot ? tok_kernel<2, true>(tensor) : tok_kernel<2, false>(tensor))
+                              : tok_kernel<4, false>(tensor);
+    static std::atomic<int> regs_seen[3][2][2];  // [J 1/2/4][rot][tensor]: registers per thread
+    std::atomic<int>& rs = regs_seen[J == 1 ? 0 : J == 2 ? 1 : 2][a.rot ? 1 : 0][tensor ? 1 : 0];
+    int regs = rs.load(std::memory_order_relaxed);
+    if (!regs) {
+        cudaFuncAttributes fa{};
+        if (cudaFuncGetAttributes(&fa, kern) != cudaSuccess || fa.numRegs <= 0) return cudaErrorInvalidValue;
+        regs = fa.numRegs;
+        rs.store(regs, std::memory_order_relaxed);
+    }
+    const int warp_regs = (regs * 32 + 255) / 256 * 256;
+    int per_sm = 65536 / ((T / 32) * warp_regs);
     const int by_smem = (200 * 1024) / (3 * row_bytes);
     per_sm = per_sm < by_smem ? per_sm : by_smem;
     per_sm = per_sm < 1 ? 1 : (per_sm > 16 ? 16 : per_sm);
@@ -986,13 +1041,15 @@ static cudaError_t launch_quant_fmt(const QuantArgs& a, int rows_pad, int num_sm
 cudaError_t launch_quant(int fmt, bool gather, const QuantArgs& a, int rows_pad, int num_sms, cudaStream_t st) {
     if (a.rot) {  // block-local rotation (no gather, one pass)
         if (gather || a.passes > 1) return cudaErrorInvalidValue;
-        if (fmt == FMT_NVFP4 && a.mode == 1 && !a.static_s2 && a.K == a.K_src && a.K <= 32768 && !a.int8_codes)
+        if (fmt == FMT_NVFP4 && (a.mode == 1 || a.tensor_amax) && !a.static_s2 && a.K == a.K_src && a.K <= 32768 &&
+            !a.int8_codes)
             return launch_nvfp4_token(a, rows_pad, num_sms, st);
         if (fmt == FMT_NVFP4) return launch_quant_fmt<FMT_NVFP4, false, false, true>(a, rows_pad, num_sms, st);
         if (fmt == FMT_MXFP4) return launch_quant_fmt<FMT_MXFP4, false, false, true>(a, rows_pad, num_sms, st);
         return launch_quant_fmt<FMT_INT4, false, false, true>(a, rows_pad, num_sms, st);
     }
-    if (fmt == FMT_NVFP4 && !gather && a.mode == 1 && !a.static_s2 && a.K == a.K_src && a.K <= 49152)
+    if (fmt == FMT_NVFP4 && !gather && (a.mode == 1 || a.tensor_amax) && !a.static_s2 && a.K == a.K_src &&
+        a.K <= 49152)
         return launch_nvfp4_token(a, rows_pad, num_sms, st);
     if (fmt == FMT_NVFP4) return gather ? launch_quant_fmt<FMT_NVFP4, true>(a, rows_pad, num_sms, st)
                                         : launch_quant_fmt<FMT_NVFP4, false>(a, rows_pad, num_sms, st);
@@ -1010,7 +1067,8 @@ cudaError_t launch_amax(const uint16_t* X, int M, int K, int ldx, float* out, in
     int grid = (int)(blocks < (long long)num_sms * 8 ? blocks : (long long)num_sms * 8);
     if (grid < 1) grid = 1;
     if (rot) amax_rot_kernel<<<grid, 256, 0, st>>>(X, M, K, ldx, rot == 1, out);
-    else amax_kernel<<<grid, 256, 0, st>>>(X, M, K, ldx, out);
+    else if ((long long)M * (K / 8) < (1LL << 31)) amax_kernel<false><<<grid, 256, 0, st>>>(X, M, K, ldx, out);
+    else amax_kernel<true><<<grid, 256, 0, st>>>(X, M, K, ldx, out);
     return cudaGetLastError();
 }
 

@@ -271,6 +271,14 @@ __device__ __forceinline__ float warp_max(float v) {
     return v;
 }
 
+// The same maximum for values that are >= 0 or NaN, in one warp reduction:
+// the bit patterns of non-negative floats order as their values.  A NaN lane
+// counts as 0 (fmaxf ignores NaN operands); only an all-NaN warp differs (0
+// instead of NaN), and a row amax of 0 or NaN gives the same s2 (1).
+__device__ __forceinline__ float warp_max_nonneg(float v) {
+    return __uint_as_float(__reduce_max_sync(0xffffffffu, __float_as_uint(fmaxf(v, 0.0f))));
+}
+
 // ---------------------------------------------------------------------------
 // Quantize rows.  A CTA owns `rows_per_cta` consecutive rows: one bulk copy
 // per row brings the bf16 row into shared memory (several CTAs per SM keep
@@ -864,14 +872,14 @@ __global__ void __launch_bounds__(J <= 2 ? 1024 : 768) quant_nvfp4_token_kernel(
             m = fmaxf(m, bm[j]);
         }
         if constexpr (!TENSOR) {
-            m = warp_max(m);
+            m = warp_max_nonneg(m);
             if (lane == 0) wmax[i & 1][warp] = m;
         }
         __syncthreads();  // (also: every thread has its row data in registers)
         if (t == 0 && i + nb < nlive) issue(i + nb);  // the buffer is free again
         float s2 = ts2;
         if constexpr (!TENSOR) {
-            s2 = nvfp4_s2(warp_max(lane < nwarps ? wmax[i & 1][lane] : 0.0f));
+            s2 = nvfp4_s2(warp_max_nonneg(lane < nwarps ? wmax[i & 1][lane] : 0.0f));
             if (t == 0) a.s2_out[r] = s2;
         }
         const bool fast = s2 >= 0x1p-100f;  // the same for the whole CTA

@@ -86,7 +86,8 @@ extern "C" {
  *         scales.  INT4: FP32, group-major [cols/group][pad128(rows)], the
  *         scale of (row r, group c) at index c * pad128(rows) + r.
  * s2      NVFP4 only: FP32 second-level scales; TENSOR: s2[0] is the scale and
- *         s2[1] is scratch for the tensor amax; TOKEN: s2[r] per row.
+ *         s2[1..3] are scratch (the tensor amax, the one-pass quantizer's CTA
+ *         count); TOKEN: s2[r] per row.
  *
  * An "augmented" activation tensor has cols = K + nS: its first K columns
  * come from w4a4_quantize_act, the last nS from w4a4_augment_residual.

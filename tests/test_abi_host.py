@@ -45,7 +45,7 @@ def test_qtensor_bytes(L):
     c, s, t = w4.qtensor_bytes(w4.NVFP4, 200, 1024, w4.SCALE_TOKEN)
     assert (c, s, t) == (200 * 512, 256 * 64, 800)
     c, s, t = w4.qtensor_bytes(w4.NVFP4, 200, 1024, w4.SCALE_TENSOR)
-    assert t == 8
+    assert t == 16  # the scale and three scratch words
     c, s, t = w4.qtensor_bytes(w4.MXFP4, 1, 256, 0)
     assert (c, s, t) == (128, 128 * 8, 0)
     c, s, t = w4.qtensor_bytes(w4.INT4, 130, 384, 0)

@@ -192,3 +192,21 @@ def test_qwen25_3b_augmented(orc, li):
     _, yref, absd = orc.gemm_nvfp4(ca, sa, s2a, 1, cw, sw, s2w)
     bad = H.gemm_violations(H.to_np_u16(Y)[rows], yref, absd)
     assert not bad.any(), f"{bad.sum()} bad"
+
+
+@pytest.mark.parametrize("M", [4096, 600])
+def test_llama2_70b_tensor_scale_both_quantizer_paths(orc, llama_weights, M):
+    """NVFP4 with a tensor activation scale at the o projection's K = 8192:
+    M = 4096 rows do not fit in shared memory across the SMs (amax pass, then
+    the row-ring quantizer); M = 600 do (one cooperative pass).  Sampled rows
+    bit-exact against the oracle with the tensor's amax, outputs within
+    tolerance."""
+    name, K, N = synth.SHAPES["llama2_70b"][1]
+    Wb = llama_weights[1]
+    Xa = synth.activations("llama2_70b", M, K, seed=5, tensor_id=300)
+    Wq = w4.quantize_weight(dev(Wb), w4.NVFP4)
+    Xq = w4.quantize_act(dev(Xa), w4.NVFP4, w4.SCALE_TENSOR)
+    Y = w4.linear(dev(Xa), Wq, w4.SCALE_TENSOR)
+    torch.cuda.synchronize()
+    assert w4.device_status() == w4.OK
+    _check_nvfp4_linear(orc, Xa, Wb, w4.SCALE_TENSOR, Xq, Wq, Y, ("llama2_70b", 1))

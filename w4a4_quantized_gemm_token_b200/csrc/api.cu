@@ -166,11 +166,19 @@ int quantize_rows(const uint16_t* X, int M, int K, int ldx, const int32_t* S, in
     a.s2_out = q->s2;
     a.tensor_amax = nullptr;
     if (q->format == W4A4_NVFP4 && q->scale_mode == W4A4_SCALE_TENSOR && !static_s2) {
-        // dynamic tensor scale: amax pass into s2[1], then the quantizer reads it
-        cudaError_t e = cudaMemsetAsync(q->s2 + 1, 0, sizeof(float), st);
-        if (e == cudaSuccess) e = launch_amax(X, M, K_src, ldx, q->s2 + 1, num_sms, st, a.rot);
+        // dynamic tensor scale: s2[1] collects the amax (s2[2] counts the CTAs
+        // of the one-pass kernel); one cooperative pass when all rows fit in
+        // shared memory, else an amax pass and the quantizer
+        cudaError_t e = cudaMemsetAsync(q->s2 + 1, 0, 2 * sizeof(float), st);
         if (e != cudaSuccess) return W4A4_ERR_CUDA;
         a.tensor_amax = q->s2 + 1;
+        if (!S && K == K_src && !a.rot && passes == 1 && !a.int8_codes && nvfp4_tensor_onepass_fits(M, K, num_sms)) {
+            e = launch_nvfp4_tensor_onepass(a, pad128(M), num_sms, reinterpret_cast<unsigned*>(q->s2 + 2), st);
+            if (e != cudaErrorCooperativeLaunchTooLarge) return cuda_status(e);
+            cudaGetLastError();  // fewer SMs available than reported: two passes
+        }
+        e = launch_amax(X, M, K_src, ldx, q->s2 + 1, num_sms, st, a.rot);
+        if (e != cudaSuccess) return W4A4_ERR_CUDA;
     }
     return cuda_status(launch_quant(q->format, S != nullptr, a, pad128(M), num_sms, st));
 }
@@ -327,7 +335,7 @@ int w4a4_qtensor_bytes(int format, int rows, int cols, int scale_mode, size_t* c
     size_t s = format == W4A4_INT4 ? (size_t)(cols / 128) * pad128(rows) * sizeof(float)
                                    : (size_t)pad128(rows) * (cols / g);
     size_t t = 0;
-    if (format == W4A4_NVFP4) t = scale_mode == W4A4_SCALE_TOKEN ? (size_t)(rows > 0 ? rows : 1) * 4 : 8;
+    if (format == W4A4_NVFP4) t = scale_mode == W4A4_SCALE_TOKEN ? (size_t)(rows > 0 ? rows : 1) * 4 : 16;
     if (codes_bytes) *codes_bytes = c;
     if (scales_bytes) *scales_bytes = s;
     if (s2_bytes) *s2_bytes = t;

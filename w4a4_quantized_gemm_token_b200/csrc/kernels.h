@@ -94,6 +94,12 @@ struct GemmArgs {
 };
 
 cudaError_t launch_quant(int fmt, bool gather, const QuantArgs& a, int rows_pad, int num_sms, cudaStream_t st);
+// NVFP4 TENSOR mode (dynamic scale, no gather, no rotation) in one
+// cooperative launch of num_sms CTAs that hold all rows in shared memory:
+// whether M x K fits, and the launch (a.tensor_amax and *arrive zero).
+bool nvfp4_tensor_onepass_fits(int M, int K, int num_sms);
+cudaError_t launch_nvfp4_tensor_onepass(const QuantArgs& a, int rows_pad, int num_sms, unsigned* arrive,
+                                        cudaStream_t st);
 // rot: 0 plain amax; 1 / 2 amax of the rotated 16-element blocks (activation / weight side)
 cudaError_t launch_amax(const uint16_t* X, int M, int K, int ldx, float* out, int num_sms, cudaStream_t st,
                         int rot = 0);

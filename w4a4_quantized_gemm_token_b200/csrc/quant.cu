@@ -935,6 +935,170 @@ __global__ void __launch_bounds__(J <= 2 ? 1024 : 768) quant_nvfp4_token_kernel(
             *reinterpret_cast<uint32_t*>(a.sf + sf_offset(r, 4 * c4, a.sf_col_atoms)) = 0u;
 }
 
+// NVFP4 TENSOR mode in one pass, for activations that fit in shared memory
+// across the grid: one CTA per SM, launched cooperatively so that every CTA
+// is resident.  Each CTA brings its rows r = blockIdx.x, +G, ... into shared
+// memory and folds their amax into the tensor amax (atomicMax on s2[1]). It
+// then counts itself in on s2[2] and waits, bounded, until every CTA has.
+// Last it quantizes its rows from shared memory with s2 = amax/2688.  The
+// codes, block scales and s2 are those of the amax pass followed by
+// quant_nvfp4_token_kernel<TENSOR>: the same block maxima, refined divisions
+// and E2M1 conversions.  s2[1] and s2[2] are zero at launch.
+__device__ __forceinline__ unsigned ld_acquire_u32(const unsigned* p) {
+    unsigned v;
+    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+
+__global__ void __launch_bounds__(1024) quant_nvfp4_tensor_onepass_kernel(QuantArgs a, unsigned* arrive) {
+    pdl_launch_dependents();
+    pdl_wait();  // X and the words to clear may belong to the preceding launch
+    const int t = threadIdx.x, T = blockDim.x, lane = t & 31, warp = t >> 5, nwarps = T >> 5;
+    if (blockIdx.x == 0)
+        for (int i = t; i < a.zero_count; i += T) a.zero_words[i] = 0;
+    extern __shared__ __align__(128) uint8_t rows[];
+    __shared__ uint64_t bar;
+    __shared__ float red[32];
+    __shared__ float s2_sh;
+    __shared__ int abort_sh;
+    volatile int* abort_flag = &abort_sh;
+    const int G = gridDim.x;
+    const int items = a.K / 16, row_bytes = a.K * 2;
+    const int nlive = a.M > (int)blockIdx.x ? (a.M - 1 - (int)blockIdx.x) / G + 1 : 0;
+    if (t == 0) {
+        mbar_init(&bar, 1);
+        *abort_flag = 0;
+        fence_mbar_init();
+        if (nlive > 0) {
+            mbar_arrive_expect_tx(&bar, (uint32_t)(nlive * row_bytes));
+            for (int i = 0; i < nlive; ++i)
+                bulk_load(rows + (size_t)i * row_bytes, a.X + (size_t)(blockIdx.x + i * G) * a.ldx, row_bytes, &bar);
+        }
+    }
+    __syncthreads();
+    if (nlive > 0) mbar_wait(&bar, 0, 2000000000ull, abort_flag);
+    // the CTA's amax (block maxima as in the token kernel; NaN ignored)
+    const int total = nlive * items;
+    float m = 0.0f;
+    if (!*abort_flag)
+        for (int f = t; f < total; f += T) {
+            const int i = f / items, it = f - i * items;
+            const uint4* p = reinterpret_cast<const uint4*>(rows + (size_t)i * row_bytes) + 2 * it;
+            const uint4 v0 = p[0], v1 = p[1];
+            const uint32_t w[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
+            m = fmaxf(m, bmax16(w));
+        }
+    m = warp_max_nonneg(m);
+    if (lane == 0) red[warp] = m;
+    __syncthreads();
+    if (t == 0) {
+        float v = 0.0f;
+        for (int k = 0; k < nwarps; ++k) v = fmaxf(v, red[k]);
+        unsigned* amax = reinterpret_cast<unsigned*>(const_cast<float*>(a.tensor_amax));
+        atomicMax(amax, __float_as_uint(v));  // v >= 0: bit order = value order
+        __threadfence();                      // the maximum is visible before the count
+        atomicAdd(arrive, 1u);
+        // every CTA is resident (cooperative launch): wait for all, bounded
+        const uint64_t t0 = globaltimer();
+        while (ld_acquire_u32(arrive) < (unsigned)G) {
+            if (globaltimer() - t0 > 2000000000ull) {
+                report_error(kErrTimeout);
+                *abort_flag = 1;
+                break;
+            }
+            __nanosleep(100);
+        }
+        s2_sh = nvfp4_s2(__uint_as_float(ld_acquire_u32(amax)));
+        if (blockIdx.x == 0 && !*abort_flag) a.s2_out[0] = s2_sh;
+    }
+    __syncthreads();
+    if (*abort_flag) {  // (the outputs are undefined; the error word says so)
+        if (t == 0 && nlive > 0) mbar_wait_drain(&bar, 0, 100000000ull);  // copies still in flight
+        return;
+    }
+    const float s2 = s2_sh;
+    const float rinv = __frcp_rn(s2);
+    const bool fast = s2 >= 0x1p-100f;  // the same for the whole grid
+    const int iters = (total + T - 1) / T;
+    for (int k = 0; k < iters; ++k) {
+        const int f = t + k * T;
+        const bool valid = f < total;  // uniform over groups of four lanes
+        const int i = valid ? f / items : 0, it = valid ? f - i * items : 0;
+        const int r = (int)blockIdx.x + i * G;
+        uint32_t w[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+        if (valid) {
+            const uint4* p = reinterpret_cast<const uint4*>(rows + (size_t)i * row_bytes) + 2 * it;
+            const uint4 v0 = p[0], v1 = p[1];
+            w[0] = v0.x; w[1] = v0.y; w[2] = v0.z; w[3] = v0.w;
+            w[4] = v1.x; w[5] = v1.y; w[6] = v1.z; w[7] = v1.w;
+        }
+        const float bm = bmax16(w);
+        uint32_t sb, w0, w1;
+        if (fast) {
+            const float u = div_refined(bm, 6.0f, 0x1.555556p-3f);  // RN(1/6)
+            sb = e4m3_rn_sat(div_refined(u, s2, rinv));
+            const float d = sb ? __fmul_rn(e4m3_value((uint8_t)sb), s2) : 1.0f;
+            const float y = __frcp_rn(d);
+            w0 = e2m1x8_fast(w, pack2(-y), pack2(d));
+            w1 = e2m1x8_fast(w + 4, pack2(-y), pack2(d));
+        } else {
+            sb = e4m3_rn_sat(__fdiv_rn(__fdiv_rn(bm, 6.0f), s2));
+            const float d = sb ? __fmul_rn(e4m3_value((uint8_t)sb), s2) : 1.0f;
+            w0 = e2m1x8_exact(make_uint4(w[0], w[1], w[2], w[3]), d);
+            w1 = e2m1x8_exact(make_uint4(w[4], w[5], w[6], w[7]), d);
+        }
+        if (sb == 0) {
+            w0 = 0;
+            w1 = 0;
+        }
+        // four consecutive items of one row sit on lanes l .. l+3
+        const uint32_t b1 = __shfl_down_sync(0xffffffffu, sb, 1);
+        const uint32_t b2 = __shfl_down_sync(0xffffffffu, sb, 2);
+        const uint32_t b3 = __shfl_down_sync(0xffffffffu, sb, 3);
+        if (valid) {
+            if ((it & 3) == 0)
+                *reinterpret_cast<uint32_t*>(a.sf + sf_offset(r, it, a.sf_col_atoms)) =
+                    sb | (b1 << 8) | (b2 << 16) | (b3 << 24);
+            *reinterpret_cast<uint2*>(a.codes + (size_t)r * a.ldc + 8 * it) = make_uint2(w0, w1);
+        }
+    }
+    // padding rows of the 128-row scale atoms: zero scales
+    for (int r = a.M + (int)blockIdx.x; r < a.rows_pad; r += G)
+        for (int c4 = t; c4 < items / 4; c4 += T)
+            *reinterpret_cast<uint32_t*>(a.sf + sf_offset(r, 4 * c4, a.sf_col_atoms)) = 0u;
+}
+
+// Shared memory the one-pass kernel may hold per CTA.
+constexpr size_t kOnepassSmem = 200 * 1024;
+
+bool nvfp4_tensor_onepass_fits(int M, int K, int num_sms) {
+    if (M <= 0 || num_sms <= 0) return false;
+    const size_t rows = (size_t)((M + num_sms - 1) / num_sms);
+    return rows * (size_t)K * 2 <= kOnepassSmem;
+}
+
+cudaError_t launch_nvfp4_tensor_onepass(const QuantArgs& a, int rows_pad, int num_sms, unsigned* arrive,
+                                        cudaStream_t st) {
+    static SmemAttrCache smem_attr;
+    const void* kern = reinterpret_cast<const void*>(quant_nvfp4_tensor_onepass_kernel);
+    cudaError_t e = ensure_dynamic_smem(kern, kOnepassSmem, smem_attr);
+    if (e != cudaSuccess) return e;
+    QuantArgs b = a;
+    b.rows_pad = rows_pad;
+    const size_t smem = (size_t)((a.M + num_sms - 1) / num_sms) * (size_t)a.K * 2;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(num_sms);
+    cfg.blockDim = dim3(1024);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeCooperative;
+    attr[0].val.cooperative = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, quant_nvfp4_tensor_onepass_kernel, b, arrive);
+}
+
 // Launch as a programmatic dependent of the preceding launch (the kernels wait
 // for it before touching memory it may write).
 template <typename... Args>

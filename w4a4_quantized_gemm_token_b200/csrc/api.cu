@@ -407,7 +407,9 @@ int w4a4_quantize_weight_segments(const uint16_t* W, int N, int K, int ldw, cons
     const int cols = K + nS;
     for (int i = 0; i < nseg; ++i) {
         // the segment as a tensor of its own: rows r0..r1 of codes, its 128-row
-        // scale atoms, and s2[r0] as its tensor scale (s2[r0 + 1] holds its amax)
+        // scale atoms, and s2[r0] as its tensor scale (s2[r0 + 1], s2[r0 + 2]
+        // are its scratch, inside the segment's rows and overwritten by the
+        // spread below)
         const int r0 = seg[i], rows = seg[i + 1] - seg[i];
         w4a4_qtensor q = *out;
         q.rows = rows;

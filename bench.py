@@ -495,9 +495,10 @@ def extra_rows(args, dev, stream, P):
         del variants, fl
 
     # the fused per-token NVFP4 linear over the Llama layer at other token
-    # counts (all on the CTA pair: 256 and 1024 fill few waves of 256 x 256
-    # tiles and stream the weights from memory once; 16384 runs many waves)
-    for Ms in ((256, 1024, 16384) if want("tokens") else ()):
+    # counts: 128 on the one-CTA kernel (128 x 256 tiles, N / 256 of them);
+    # 256 and 1024 on the CTA pair, few waves of 256 x 256 tiles streaming the
+    # weights from memory once; 16384 runs many waves
+    for Ms in ((128, 256, 1024, 16384) if want("tokens") else ()):
         lay = []
         for li, (name, K, N) in enumerate(LLAMA):
             Wq = w4.quantize_weight(to_dev(synth.weights("llama2_70b", N, K, seed=0, tensor_id=100 + li), dev),

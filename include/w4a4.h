@@ -269,8 +269,11 @@ int w4a4_linear(const uint16_t* X, int M, int K, int ldx,
  *  - Sizes whose w4a4_linear_workspace() exceeds W4A4_NOALLOC_SCRATCH_BYTES
  *    return W4A4_ERR_WORKSPACE and launch nothing (16 MiB covers, e.g., every
  *    Llama-2-70B-sized linear at M <= 16, the small-M decode case).
- *  - The first call on a device (with that device current) looks up the
- *    array's address; make it before any stream capture.
+ *  - The first call in a CUDA context (with its device current) looks up
+ *    the array's address in that context and caches it per context handle;
+ *    make that first call before any stream capture.  Calls made in another
+ *    context (a driver-API context of the caller's, or the primary context
+ *    re-created after cudaDeviceReset) look the address up again there.
  *  - No scratch byte needs to start at zero: the call writes all it reads.
  *  - One scratch per device: calls on one device whose kernels could overlap
  *    (unordered streams, several host threads) race on it and must be

@@ -202,3 +202,13 @@ def test_int4_group_choice_and_checks(L):
     a.group = 512
     b = _qt(w4.INT4, 256, 1024)
     assert L.w4a4_gemm(C.byref(a), C.byref(b), C.c_void_p(16), 256, None) == w4.ERR_INVALID_ARG  # groups differ
+
+
+def test_noalloc_scratch_size_matches_header():
+    """The binding's copy of the no-alloc scratch size is the header's."""
+    import re
+    hdr = open(os.path.join(ROOT, "include", "w4a4.h")).read()
+    m = re.search(r"#define\s+W4A4_NOALLOC_SCRATCH_BYTES\s+\((\d+)u\s*<<\s*(\d+)\)", hdr)
+    assert m, "W4A4_NOALLOC_SCRATCH_BYTES not found"
+    import w4a4_quantized_gemm_token_b200 as w4
+    assert w4.NOALLOC_SCRATCH_BYTES == int(m.group(1)) << int(m.group(2))

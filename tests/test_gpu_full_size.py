@@ -171,24 +171,42 @@ def test_qwen25_7b_int4_g128(orc, li):
 @pytest.mark.parametrize("li", range(3))
 def test_qwen25_3b_augmented(orc, li):
     """Dual-stage NVFP4 augmentation, Qwen2.5-3B shapes at M = 8192, the 256
-    channels chosen from the seed-1 calibration batch; sampled rows."""
+    channels chosen from the seed-1 calibration batch ("APEX4..." page, para 2:
+    ARCQuant).  Bit for bit on sampled rows: the augmented activation codes and
+    block scales over all K + 256 columns (first stage, then the residual
+    stage, as the fused linear runs them), the row scales, and the weight codes
+    and block scales of [W | W[:, S]]; the sampled output rows within the GEMM
+    tolerance."""
     name, K, N = synth.SHAPES["qwen25_3b_aug"][li]
     M, nS = 8192, 256
+    cols = K + nS
     S_np = orc.select_channels(synth.calibration("qwen25_3b_aug", K), nS)
     S = torch.from_numpy(S_np).cuda()
     np.testing.assert_array_equal(w4.select_channels(dev(synth.calibration("qwen25_3b_aug", K)), nS).cpu().numpy(),
                                   S_np)
     Xa = synth.activations("qwen25_3b_aug", M, K, seed=0, tensor_id=200 + li)
     Wb = synth.weights("qwen25_3b_aug", N, K, seed=0, tensor_id=100 + li)
+    Xd = dev(Xa)
     Wq = w4.quantize_weight(dev(Wb), w4.NVFP4, S=S)
-    Y = w4.linear(dev(Xa), Wq, w4.SCALE_TOKEN, S=S)
+    Xq = w4.quantize_act(Xd, w4.NVFP4, w4.SCALE_TOKEN, cols=cols)
+    w4.augment_residual(Xd, S, Xq)
+    Y = w4.linear(Xd, Wq, w4.SCALE_TOKEN, S=S)
     torch.cuda.synchronize()
     assert w4.device_status() == w4.OK
     rows = _rows(M)
     ca, sa, s2a = orc.quant_nvfp4(Xa[rows], mode=1)
     rc, rs = orc.augment_nvfp4(Xa[rows], S_np, ca, sa, s2a, 1)
     ca, sa = np.concatenate([ca, rc], 1), np.concatenate([sa, rs], 1)
-    cw, sw, s2w = orc.quant_nvfp4(np.concatenate([Wb, Wb[:, S_np]], 1), mode=0)
+    gc, gs = _nv_rows(Xq, rows, cols)
+    np.testing.assert_array_equal(gc, ca)
+    np.testing.assert_array_equal(gs, sa)
+    np.testing.assert_array_equal(Xq.s2.cpu().numpy()[rows], s2a)
+    cw, sw, s2w = orc.quant_nvfp4(np.ascontiguousarray(np.concatenate([Wb, Wb[:, S_np]], 1)), mode=0)
+    assert np.float32(Wq.s2.cpu().numpy()[0]) == np.float32(s2w[0])
+    wrows = _rows(N)
+    gc, gs = _nv_rows(Wq, wrows, cols)
+    np.testing.assert_array_equal(gc, cw[wrows])
+    np.testing.assert_array_equal(gs, sw[wrows])
     _, yref, absd = orc.gemm_nvfp4(ca, sa, s2a, 1, cw, sw, s2w)
     bad = H.gemm_violations(H.to_np_u16(Y)[rows], yref, absd)
     assert not bad.any(), f"{bad.sum()} bad"

@@ -287,3 +287,38 @@ def test_abi_errors_on_gpu():
     with pytest.raises(w4.W4A4Error) as e:
         w4.linear(X, Wq, w4.SCALE_TOKEN, ws=torch.empty(256, dtype=torch.uint8, device="cuda"))
     assert e.value.status == w4.ERR_WORKSPACE
+
+
+@pytest.mark.parametrize("fmt", [w4.NVFP4, w4.MXFP4, w4.INT4])
+@pytest.mark.parametrize("N,K,nS", [(200, 1024, 128), (130, 2048, 256), (1, 384, 384)])
+def test_weight_gather_bitexact(orc, fmt, N, K, nS):
+    """w4a4_quantize_weight with channels S: [W | W[:, S]] quantized as one
+    tensor of K + nS columns ("APEX4..." page, para 2: ARCQuant duplicates the
+    weight columns of the augmented channels), bit for bit at ragged N.  The
+    duplicated columns form blocks of their own, so their codes are compared
+    against the oracle's quantization of the concatenated matrix, not copied
+    from the first K columns."""
+    Xw = synth.weights("qwen25_3b_aug", N, K, seed=11)
+    S_np = np.sort(np.random.default_rng(7).choice(K, nS, replace=False)).astype(np.int32)
+    S = torch.from_numpy(S_np).cuda()
+    Wq = w4.quantize_weight(dev(Xw), fmt, S=S)
+    torch.cuda.synchronize()
+    assert w4.device_status() == w4.OK
+    cols = K + nS
+    Wcat = np.ascontiguousarray(np.concatenate([Xw, Xw[:, S_np]], 1))
+    codes = Wq.codes.cpu().numpy()[: N * cols // 2].reshape(N, cols // 2)
+    if fmt == w4.NVFP4:
+        oc, osc, os2 = orc.quant_nvfp4(Wcat, mode=0)
+        np.testing.assert_array_equal(codes, oc)
+        np.testing.assert_array_equal(H.unswizzle_scales(Wq.scales.cpu().numpy(), N, cols, 16), osc)
+        assert np.float32(Wq.s2.cpu().numpy()[0]) == np.float32(os2[0])
+        assert np.all(H.padding_scales(Wq.scales.cpu().numpy(), N, cols, 16) == 0)
+    elif fmt == w4.MXFP4:
+        oc, osc = orc.quant_mxfp4(Wcat)
+        np.testing.assert_array_equal(codes, oc)
+        np.testing.assert_array_equal(H.unswizzle_scales(Wq.scales.cpu().numpy(), N, cols, 32), osc)
+    else:
+        oc, osc = orc.quant_int4(Wcat)
+        np.testing.assert_array_equal(codes, oc)
+        sc = H.int4_scales(Wq.scales.cpu().numpy().view(np.float32), N, cols)
+        np.testing.assert_array_equal(sc.view(np.uint32), osc.view(np.uint32))

@@ -64,3 +64,27 @@ def test_noalloc_rejects_sizes_beyond_its_scratch():
     assert e.value.status == w4.ERR_WORKSPACE
     torch.cuda.synchronize()
     assert bool((Y == 3.0).all())          # nothing was launched
+
+
+@pytest.mark.parametrize("model,M,K,N,fmt,mode", [
+    ("llama2_70b", 1, 8192, 10240, w4.NVFP4, w4.SCALE_TOKEN),   # decode: split-K partials and tile counters
+    ("llama2_70b", 16, 2048, 1024, w4.MXFP4, 0),
+    ("llama2_70b", 300, 2048, 1024, w4.NVFP4, w4.SCALE_TOKEN),  # CTA-pair GEMM
+])
+def test_noalloc_back_to_back_calls_on_one_stream(model, M, K, N, fmt, mode):
+    """Three no-alloc calls with different inputs issued on one stream with
+    nothing between them (no synchronisation, no other launch), so each
+    call's quantizer may start while the previous call's GEMM still runs;
+    every output must equal the workspace path's, computed afterwards."""
+    Wq = w4.quantize_weight(dev(synth.weights(model, N, K, seed=22)), fmt)
+    Xs = [dev(synth.activations(model, M, K, seed=60 + c)) for c in range(3)]
+    Ys = [torch.full((M, N), float("nan"), dtype=torch.bfloat16, device="cuda") for _ in range(3)]
+    torch.cuda.synchronize()
+    for X, Y in zip(Xs, Ys):
+        w4.linear_noalloc(X, Wq, mode, Y=Y)
+    torch.cuda.synchronize()
+    assert w4.device_status() == w4.OK
+    for c, (X, Y) in enumerate(zip(Xs, Ys)):
+        ref = w4.linear(X, Wq, mode)
+        torch.cuda.synchronize()
+        assert torch.equal(Y.view(torch.int16), ref.view(torch.int16)), f"call {c}"

@@ -9,9 +9,12 @@
 // is loaded on that device.  Nothing here calls cudaMalloc, cudaFree or any
 // allocating library routine.
 //
-// Set-up: the first call on a device, with that device current, looks up the
-// array's device address (cudaGetSymbolAddress) and caches it for that
-// device; make that first call before any stream capture.
+// Set-up: the first call in a CUDA context (with its device current) looks up
+// the array's device address there (cudaGetSymbolAddress) and caches it for
+// that context; make that first call before any stream capture.  The array is
+// per module and context, so a caller that drives its own driver-API context
+// or re-creates the primary context (cudaDeviceReset) gets the address of the
+// copy in the context that is current at the call.
 //
 // Zero state: no byte of the scratch has to start at zero.  Every byte a
 // call reads is written earlier in the same call (quantized activation codes
@@ -22,6 +25,7 @@
 // calls whose kernels can run at the same time (different streams without an
 // ordering between them, or several host threads) overwrite each other's
 // scratch; such calls must be ordered (one stream, or events).
+#include <cuda.h>
 #include <cuda_runtime.h>
 
 #include <mutex>
@@ -32,29 +36,55 @@ namespace {
 
 static __device__ __align__(256) unsigned char g_linear_scratch[W4A4_NOALLOC_SCRATCH_BYTES];
 
-constexpr int kMaxDevices = 64;
-std::mutex g_scratch_mutex;
-void* g_scratch_ptr[kMaxDevices] = {};
+typedef CUresult (*CtxGetCurrentFn)(CUcontext*);
 
-// Device address of g_linear_scratch on the current device (looked up once).
-int scratch_for_current_device(void** out) {
+// A few cached (context, address) pairs; a context not among them is looked up
+// (and replaces the oldest entry).
+constexpr int kSlots = 64;
+struct Slot {
+    CUcontext ctx;
+    void* ptr;
+};
+std::mutex g_scratch_mutex;
+Slot g_slots[kSlots] = {};
+int g_next_slot = 0;
+CtxGetCurrentFn g_ctx_get_current = nullptr;
+
+// Device address of g_linear_scratch in the current context.
+int scratch_for_current_context(void** out) {
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return W4A4_ERR_CUDA;
-    if (dev < 0 || dev >= kMaxDevices) return W4A4_ERR_INVALID_ARG;
     std::lock_guard<std::mutex> lock(g_scratch_mutex);
-    if (!g_scratch_ptr[dev]) {
-        int major = 0;
-        if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess)
+    if (!g_ctx_get_current) {
+        void* fn = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &fn, cudaEnableDefault, &q) != cudaSuccess ||
+            q != cudaDriverEntryPointSuccess || !fn)
             return W4A4_ERR_CUDA;
-        if (major != 10) return W4A4_ERR_ARCH;
-        void* p = nullptr;
-        if (cudaGetSymbolAddress(&p, g_linear_scratch) != cudaSuccess || !p) {
-            cudaGetLastError();
-            return W4A4_ERR_CUDA;
-        }
-        g_scratch_ptr[dev] = p;
+        g_ctx_get_current = reinterpret_cast<CtxGetCurrentFn>(fn);
     }
-    *out = g_scratch_ptr[dev];
+    CUcontext ctx = nullptr;
+    if (g_ctx_get_current(&ctx) != CUDA_SUCCESS) return W4A4_ERR_CUDA;
+    if (ctx)
+        for (int i = 0; i < kSlots; ++i)
+            if (g_slots[i].ctx == ctx) {
+                *out = g_slots[i].ptr;
+                return W4A4_OK;
+            }
+    int major = 0;
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess) return W4A4_ERR_CUDA;
+    if (major != 10) return W4A4_ERR_ARCH;
+    // (with no context current yet, this runtime call makes the device's
+    // primary context current)
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_linear_scratch) != cudaSuccess || !p) {
+        cudaGetLastError();
+        return W4A4_ERR_CUDA;
+    }
+    if (!ctx && (g_ctx_get_current(&ctx) != CUDA_SUCCESS || !ctx)) return W4A4_ERR_CUDA;
+    g_slots[g_next_slot] = Slot{ctx, p};
+    g_next_slot = (g_next_slot + 1) % kSlots;
+    *out = p;
     return W4A4_OK;
 }
 
@@ -67,7 +97,7 @@ extern "C" int w4a4_linear_noalloc(const uint16_t* X, int M, int K, int ldx, con
     const size_t need = w4a4_linear_workspace(M, Wq->rows, K, Wq->format, nS);
     if (need > (size_t)W4A4_NOALLOC_SCRATCH_BYTES) return W4A4_ERR_WORKSPACE;
     void* scratch = nullptr;
-    const int rc = scratch_for_current_device(&scratch);
+    const int rc = scratch_for_current_context(&scratch);
     if (rc != W4A4_OK) return rc;
     return w4a4_linear(X, M, K, ldx, Wq, scale_mode, S, nS, Y, ldy, scratch, (size_t)W4A4_NOALLOC_SCRATCH_BYTES,
                        stream);

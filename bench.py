@@ -37,12 +37,22 @@ LLAMA = synth.SHAPES["llama2_70b"]
 PEAKS_FILE = os.path.join(ROOT, "MEASURED_PEAKS.json")
 FP4_PER_BF16 = 4.0        # nominal dense FP4 / BF16 tensor throughput (9 / 2.25 PFLOP/s)
 INT8_PER_BF16 = 2.0       # nominal dense INT8 / BF16 (4.5 / 2.25)
+NOMINAL_FP4_TFLOPS = 9000.0  # B200 dense FP4, nominal
+# FP4 MMA issue rate per SM: one 128x256x64 NVFP4 MMA (2 * 128 * 256 * 64 FLOP)
+# every 128 cycles, measured back to back on one SM
+MMA_FLOP_PER_CYCLE = 2 * 128 * 256 * 64 // 128
+
+
+def mma_issue_peak_tflops(dev, sm_mhz: float) -> float:
+    import torch
+    sms = torch.cuda.get_device_properties(dev).multi_processor_count
+    return sms * MMA_FLOP_PER_CYCLE * sm_mhz * 1e6 / 1e12
 
 
 # DRAM traffic (dram__bytes_read.sum + dram__bytes_write.sum) per launch of the
-# dominant kernel, averaged over the five GEMM launches of one step, from the ncu
-# launch list summarised in profiles/launch_list_llama70b_layer_m4096.md; valid
-# only for the kernel source it was measured on (else reported as null).
+# dominant kernel, averaged over the five GEMM launches of one step, from an ncu
+# capture of the pair GEMM on this workload; valid only for the kernel source it
+# was measured on (else reported as null).
 PROFILED_TRAFFIC = {"sources": ("gemm_fp4_pair.cu", "ptx.cuh"), "sha256_16": "718b7937ac7f9a8f",
                     "bytes_per_launch": 295.0e6}
 
@@ -60,9 +70,10 @@ def peaks():
     try:
         p = json.load(open(PEAKS_FILE))
         return {"hbm": float(p["hbm_gbs"]), "bf16": float(p["bf16_tflops"]),
-                "bf16_sustained": float(p.get("bf16_tflops_sustained", p["bf16_tflops"])), "src": "measured"}
+                "bf16_sustained": float(p.get("bf16_tflops_sustained", p["bf16_tflops"])), "src": "measured",
+                "sm_max_mhz": float(p.get("sm_max_mhz", 1965.0))}
     except Exception:
-        return {"hbm": 6650.0, "bf16": 1590.0, "bf16_sustained": 1400.0, "src": "fallback"}
+        return {"hbm": 6650.0, "bf16": 1590.0, "bf16_sustained": 1400.0, "src": "fallback", "sm_max_mhz": 1965.0}
 
 
 # ----------------------------------------------------------------------------------------------
@@ -118,29 +129,76 @@ class ClockSampler:
 _ORACLE_W = {}
 
 
-def oracle_sample(M_rows: int, n_cols: int):
-    """Time the C oracle (as it stands, one host thread) on the layer's five
-    linears for `M_rows` tokens and the first `n_cols` output columns of each:
-    per-token NVFP4 quantization of those rows plus the exact block-scaled GEMM.
+def _oracle_weights(li, n):
+    import oracle
+    key = (li, n)
+    if key not in _ORACLE_W:
+        name, K, N = LLAMA[li]
+        W = synth.weights("llama2_70b", N, K, seed=0, tensor_id=100 + li)[:n]
+        _ORACLE_W[key] = oracle.quant_nvfp4(W, mode=0)
+    return _ORACLE_W[key]
+
+
+def host_threads() -> int:
+    """Host cores this process may run on."""
+    try:
+        return len(os.sched_getaffinity(0))
+    except Exception:
+        return os.cpu_count() or 1
+
+
+def oracle_sample(M_rows: int, n_cols: int, threads: int = 1):
+    """Time the C oracle (as it stands) on the layer's five linears for
+    `M_rows` tokens and the first `n_cols` output columns of each: per-token
+    NVFP4 quantization of those rows plus the exact block-scaled GEMM.  With
+    threads > 1 the GEMM's output columns are split into `threads` contiguous
+    parts computed at once (the oracle's C calls release the interpreter lock).
     The weights' quantization is offline on both arms and is not timed.
     Returns (TFLOPS, seconds, flops)."""
     import oracle
+    from concurrent.futures import ThreadPoolExecutor
     oracle.build()
     t_total, flops = 0.0, 0.0
-    for li, (name, K, N) in enumerate(LLAMA):
-        n = min(N, n_cols)
-        key = (li, n)
-        if key not in _ORACLE_W:
-            W = synth.weights("llama2_70b", N, K, seed=0, tensor_id=100 + li)[:n]
-            _ORACLE_W[key] = oracle.quant_nvfp4(W, mode=0)
-        cw, sw, s2w = _ORACLE_W[key]
-        X = synth.activations("llama2_70b", M_rows, K, seed=0, tensor_id=200 + li)
-        t0 = time.perf_counter()
-        ca, sa, s2a = oracle.quant_nvfp4(X, mode=1)
-        oracle.gemm_nvfp4(ca, sa, s2a, 1, cw, sw, s2w, want_ref=False)
-        t_total += time.perf_counter() - t0
-        flops += 2.0 * M_rows * n * K
+    pool = ThreadPoolExecutor(threads) if threads > 1 else None
+    try:
+        for li, (name, K, N) in enumerate(LLAMA):
+            n = min(N, n_cols)
+            cw, sw, s2w = _oracle_weights(li, n)
+            X = synth.activations("llama2_70b", M_rows, K, seed=0, tensor_id=200 + li)
+            t0 = time.perf_counter()
+            ca, sa, s2a = oracle.quant_nvfp4(X, mode=1)
+            if pool is None:
+                oracle.gemm_nvfp4(ca, sa, s2a, 1, cw, sw, s2w, want_ref=False)
+            else:
+                cuts = [n * i // threads for i in range(threads + 1)]
+                parts = [(cuts[i], cuts[i + 1]) for i in range(threads) if cuts[i + 1] > cuts[i]]
+                list(pool.map(lambda r: oracle.gemm_nvfp4(ca, sa, s2a, 1, cw[r[0]:r[1]], sw[r[0]:r[1]], s2w,
+                                                          want_ref=False), parts))
+            t_total += time.perf_counter() - t0
+            flops += 2.0 * M_rows * n * K
+    finally:
+        if pool is not None:
+            pool.shutdown()
     return flops / t_total / 1e12, t_total, flops
+
+
+def mxfp4_small_parity(Y_gpu_bits):
+    """The MXFP4 16x256x256 workload (X ~ N(0,1), W ~ N(0,0.02), seed 0) by the
+    oracle, compared with the GPU's output: every element within 1 bf16 ulp +
+    1e-5 * sum|a w| of the exact product.  Returns (ok, oracle seconds)."""
+    import oracle
+    Xa = synth.activations("mxfp4_small", 16, 256, seed=0)
+    Xw = synth.weights("mxfp4_small", 256, 256, seed=0)
+    t0 = time.perf_counter()
+    ca, sa = oracle.quant_mxfp4(Xa)
+    cw, sw = oracle.quant_mxfp4(Xw)
+    _, yref, absd = oracle.gemm_mxfp4(ca, sa, cw, sw)
+    dt = time.perf_counter() - t0
+    y = (np.asarray(Y_gpu_bits, np.uint16).astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+    a = np.abs(yref)
+    ulp = np.exp2(np.maximum(np.floor(np.log2(np.where(a > 0, a, 1.0))), -126) - 7)
+    ok = bool((np.abs(y - yref) <= ulp + 1e-5 * absd).all())
+    return ok, dt
 
 
 def run_reference(args, rank, world):
@@ -148,11 +206,12 @@ def run_reference(args, rank, world):
         return
     K, W = args.steps, args.warmup
     rows, cols = args.ref_rows, args.ref_cols
+    threads = host_threads()
     for _ in range(W):
-        oracle_sample(1, cols)
+        oracle_sample(1, cols, threads)
     vals, secs = [], []
     for _ in range(K):
-        v, s, _ = oracle_sample(rows, cols)
+        v, s, _ = oracle_sample(rows, cols, threads)
         vals.append(v)
         secs.append(s)
     value = statistics.median(vals)
@@ -163,9 +222,9 @@ def run_reference(args, rank, world):
         "vs_baseline": None, "dtype": "nvfp4", "data": "synthetic",
         "config": {"workload": f"llama2_70b layer linears (qkv,o,w1,w3,w2), oracle on {rows} tokens x "
                                f"{cols} output columns per linear per step", "tokens": rows},
-        "cpu_baseline": {"value": value, "unit": "TFLOPS", "cores": 1, "kind": "oracle",
+        "cpu_baseline": {"value": value, "unit": "TFLOPS", "cores": threads, "kind": "oracle",
                          "sample": f"{rows} tokens x {cols} output columns of each of the 5 layer linears "
-                                   f"(full K), one host thread"},
+                                   f"(full K), GEMM columns split over {threads} host threads"},
         "e2e": {"value": value, "unit": "TFLOPS", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
@@ -236,7 +295,11 @@ def run_ours(args, rank, world):
     fp4_peak = P["bf16"] * FP4_PER_BF16
     M = args.tokens
     if args.only is not None:
-        print(json.dumps({"only": args.only, "rows": extra_rows(args, dev, stream, P)}), flush=True)
+        rows = extra_rows(args, dev, stream, P)
+        for v in rows.values():
+            if isinstance(v, dict):
+                v.pop("_y", None)
+        print(json.dumps({"only": args.only, "rows": rows}), flush=True)
         return
 
     # ---- workload: Llama-2-70B layer linears, NVFP4 weights quantized once ----
@@ -290,18 +353,52 @@ def run_ours(args, rank, world):
     h2d = sum(h.numel() * 2 for h in hX)
     d2h = sum(h.numel() * 2 for h in hY)
 
+    # Copies overlap the compute: a copy-in stream brings X of linear i + 1
+    # while linear i runs, a copy-out stream returns Y of linear i - 1 (PCIe is
+    # full duplex); events order each buffer's reuse across steps.
+    s_in, s_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+    nl = len(layers)
+    ev_in = [torch.cuda.Event() for _ in range(nl)]
+    ev_comp = [torch.cuda.Event() for _ in range(nl)]
+    ev_out = [torch.cuda.Event() for _ in range(nl)]
+    for i in range(nl):  # every buffer starts free
+        ev_comp[i].record(stream)
+        ev_out[i].record(stream)
+
     def e2e_step():
         for i, (_, K, N, Wq, X, Y, ws) in enumerate(layers):
-            X.copy_(hX[i], non_blocking=True)
+            s_in.wait_event(ev_comp[i])       # X_i no longer read by the previous step
+            with torch.cuda.stream(s_in):
+                X.copy_(hX[i], non_blocking=True)
+            ev_in[i].record(s_in)
+            stream.wait_event(ev_in[i])
+            stream.wait_event(ev_out[i])      # Y_i of the previous step has left
             w4.linear(X, Wq, w4.SCALE_TOKEN, Y=Y, ws=ws)
-            hY[i].copy_(Y, non_blocking=True)
+            ev_comp[i].record(stream)
+            s_out.wait_event(ev_comp[i])
+            with torch.cuda.stream(s_out):
+                hY[i].copy_(Y, non_blocking=True)
+            ev_out[i].record(s_out)
+
+    def e2e_timed(iters):
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        s_in.wait_event(e0)
+        for _ in range(iters):
+            e2e_step()
+        for i in range(nl):  # the last outputs are home
+            stream.wait_event(ev_out[i])
+        e1.record(stream)
+        e1.synchronize()
+        return e0.elapsed_time(e1) / iters
 
     e2e_iters = max(3, min(args.steps, 10))
     e2e_step()
     torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
-    e2e_ms = time_loop(e2e_step, e2e_iters, stream)
+    e2e_ms = e2e_timed(e2e_iters)
     e2e_ms = max_over_ranks(e2e_ms, dev, world)
     e2e_value = flops_step * world / (e2e_ms * 1e-3) / 1e12
 
@@ -318,10 +415,17 @@ def run_ours(args, rank, world):
         gemm_flops += f
         del Xq
     gemm_tflops = gemm_flops / (gemm_ms * 1e-3) / 1e12
+    sm_mhz = (clocks or {}).get("sm_mhz") or P["sm_max_mhz"]
+    issue_peak = mma_issue_peak_tflops(dev, sm_mhz)
     roofline = {"bound": "tensor", "achieved": round(gemm_tflops, 1), "peak": round(fp4_peak, 1),
                 "unit": "TFLOP/s", "frac": round(gemm_tflops / fp4_peak, 4), "traffic": profiled_traffic(),
                 "peak_src": f"{P['src']} bf16 burst x {FP4_PER_BF16:g} (nominal fp4/bf16)",
-                "kernel": "gemm_fp4_pair_kernel (NVFP4, 256x256 tile on a CTA pair)", "per_shape_tflops": per_shape}
+                "kernel": "gemm_fp4_pair_kernel (NVFP4, 256x256 tile on a CTA pair)", "per_shape_tflops": per_shape,
+                "frac_of_nominal_9pf": round(gemm_tflops / NOMINAL_FP4_TFLOPS, 4),
+                "frac_of_mma_issue_peak": round(gemm_tflops / issue_peak, 4),
+                "mma_issue_peak": round(issue_peak, 1),
+                "mma_issue_peak_src": f"SMs x {MMA_FLOP_PER_CYCLE} FLOP/cycle (back-to-back 128x256x64 NVFP4 MMA "
+                                      f"every 128 cycles) x median SM clock {sm_mhz:.0f} MHz"}
 
     rows = {} if args.no_rows else extra_rows(args, dev, stream, P)
 
@@ -336,6 +440,8 @@ def run_ours(args, rank, world):
                        "tokens_per_gpu": M, "l2": "inputs larger than L2 (0.47 GB of weights per step)",
                        "parallelism": f"replicas x{world}"},
             "frac_of_fp4_peak": round(value / world / fp4_peak, 4),
+            "frac_of_nominal_fp4_9pf": round(value / world / NOMINAL_FP4_TFLOPS, 4),
+            "frac_of_mma_issue_peak": round(value / world / issue_peak, 4),
             "roofline": roofline,
             "e2e": {"value": round(e2e_value, 3), "unit": "TFLOPS", "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h},
@@ -344,10 +450,22 @@ def run_ours(args, rank, world):
             "rows": rows,
         }
         if world == 1 and not args.no_cpu:
-            v, s, f = oracle_sample(args.cpu_rows, args.cpu_cols)
-            line["cpu_baseline"] = {"value": v, "unit": "TFLOPS", "cores": 1, "kind": "oracle",
-                                    "sample": f"{args.cpu_rows} tokens x {args.cpu_cols} output columns of each "
-                                              f"of the 5 layer linears (full K), one host thread, {s:.1f} s"}
+            threads = host_threads()
+            v1, s1, _ = oracle_sample(args.cpu_rows, args.cpu_cols, 1)
+            vn, sn, _ = oracle_sample(args.cpu_rows, args.cpu_cols, threads)
+            line["cpu_baseline"] = {
+                "value": vn, "unit": "TFLOPS", "cores": threads, "kind": "oracle",
+                "sample": f"{args.cpu_rows} tokens x {args.cpu_cols} output columns of each of the 5 layer "
+                          f"linears (full K); GEMM columns split over {threads} host threads, {sn:.1f} s",
+                "single_thread": {"value": v1, "cores": 1, "seconds": round(s1, 2)},
+                "host_cores": os.cpu_count()}
+            small = rows.get("mxfp4_small_16x256x256") if isinstance(rows, dict) else None
+            if small is not None and "_y" in small:
+                ok, dt = mxfp4_small_parity(small.pop("_y"))
+                small["parity_vs_oracle"] = ok
+                small["oracle_us"] = round(dt * 1e6, 1)
+        if isinstance(rows, dict) and isinstance(rows.get("mxfp4_small_16x256x256"), dict):
+            rows["mxfp4_small_16x256x256"].pop("_y", None)
         print(json.dumps(line), flush=True)
 
 
@@ -421,8 +539,30 @@ def extra_rows(args, dev, stream, P):
         dec()
         ms = time_loop(dec, it, stream)
         byts = sum(N * K * 0.5625 + 2 * Md * K + 2 * Md * N for (K, N, _) in Ws)
-        out[f"decode_m{Md}_llama_layer"] = {"GB/s": round(byts / ms / 1e6, 1), "frac_hbm": round(byts / ms / 1e6 / hbm, 3),
-                                            "us": round(ms * 1e3, 2)}
+        # the same layer as one CUDA graph (ten kernels, PDL edges kept): the
+        # difference to the eager stream is what host launches cost
+        t0 = time.perf_counter()
+        for _ in range(it):
+            dec()
+        host_us = (time.perf_counter() - t0) / (it * 2 * len(bufs)) * 1e6
+        torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        side = torch.cuda.Stream(dev)
+        side.wait_stream(stream)
+        with torch.cuda.stream(side):
+            dec()
+        stream.wait_stream(side)
+        torch.cuda.synchronize()
+        with torch.cuda.graph(g):
+            dec()
+        g.replay()
+        ms_g = time_loop(g.replay, it, stream)
+        out[f"decode_m{Md}_llama_layer"] = {
+            "GB/s": round(byts / ms / 1e6, 1), "frac_hbm": round(byts / ms / 1e6 / hbm, 3), "us": round(ms * 1e3, 2),
+            "graph_GB/s": round(byts / ms_g / 1e6, 1), "graph_frac_hbm": round(byts / ms_g / 1e6 / hbm, 3),
+            "graph_us": round(ms_g * 1e3, 2), "host_launch_us_per_kernel": round(host_us, 2),
+            "launch_overhead_us_per_layer": round((ms - ms_g) * 1e3, 2)}
+        del g
     del Ws
 
     # INT4, Qwen2.5-7B shapes at M = 2048: groups of 128, and of 512 (the
@@ -540,7 +680,40 @@ def extra_rows(args, dev, stream, P):
         fl = sum(2.0 * args.tokens * N * K for (K, N, *_r) in lay)
         out[f"linear_nvfp4_tensor_swiglu300m_m{args.tokens}"] = {"TFLOPS": round(fl / (ms * 1e-3) / 1e12, 1),
                                                                  "ms": round(ms, 3)}
-        del lay
+        # static activation scale (a calibrated constant per linear, here the
+        # tensor's own amax / 2688 taken once outside the timed region): the
+        # quantizer with the caller's s2, then the GEMM; and the quantizers
+        # alone, dynamic (amax inside the call) against static
+        qs, sts = [], []
+        for (K, N, Wq, X, Y, ws) in lay:
+            sts.append((X.float().abs().max() / 2688.0).reshape(1).contiguous())
+            qs.append(w4.QTensor(w4.NVFP4, args.tokens, K, w4.SCALE_TENSOR, dev))
+
+        def st_step():
+            for (K, N, Wq, X, Y, ws), q, st in zip(lay, qs, sts):
+                w4.quantize_act(X, w4.NVFP4, w4.SCALE_TENSOR, static_s2=st, out=q)
+                w4.gemm(q, Wq, Y)
+
+        def q_dyn():
+            for (K, N, Wq, X, Y, ws), q in zip(lay, qs):
+                w4.quantize_act(X, w4.NVFP4, w4.SCALE_TENSOR, out=q)
+
+        def q_st():
+            for (K, N, Wq, X, Y, ws), q, st in zip(lay, qs, sts):
+                w4.quantize_act(X, w4.NVFP4, w4.SCALE_TENSOR, static_s2=st, out=q)
+        for _ in range(max(3, args.warmup)):
+            st_step()
+        ms_s = time_loop(st_step, max(5, min(args.steps, 20)), stream)
+        out[f"linear_nvfp4_static_s2_swiglu300m_m{args.tokens}"] = {"TFLOPS": round(fl / (ms_s * 1e-3) / 1e12, 1),
+                                                                    "ms": round(ms_s, 3)}
+        q_dyn()
+        q_st()
+        ms_qd = time_loop(q_dyn, max(5, min(args.steps, 20)), stream)
+        ms_qs = time_loop(q_st, max(5, min(args.steps, 20)), stream)
+        out[f"quant_nvfp4_tensor_swiglu300m_layer_inputs_m{args.tokens}"] = {
+            "dynamic_us": round(ms_qd * 1e3, 2), "static_us": round(ms_qs * 1e3, 2),
+            "amax_cost_us": round((ms_qd - ms_qs) * 1e3, 2)}
+        del lay, qs, sts
 
     # multi-pass MXFP4 (two passes) on the Llama qkv shape: the quantizer alone
     # (L2 flushed before each launch) and the linear, beside one-pass MXFP4
@@ -601,6 +774,34 @@ def extra_rows(args, dev, stream, P):
                                                           "us": round(ms * 1e3, 2)}
         del Wp, Wr, X, Y
 
+    # the MXFP4 16 x 256 x 256 workload (X ~ N(0,1), W ~ N(0,0.02), seed 0):
+    # the fused linear's time, eager and as a CUDA graph; its output is kept
+    # for the oracle comparison of the CPU-baseline leg
+    if want("small"):
+        Xs = to_dev(synth.activations("mxfp4_small", 16, 256, seed=0), dev)
+        Wsm = w4.quantize_weight(to_dev(synth.weights("mxfp4_small", 256, 256, seed=0), dev), w4.MXFP4)
+        Ysm = torch.empty(16, 256, dtype=torch.bfloat16, device=dev)
+        wss = torch.empty(w4.linear_workspace(16, 256, 256, w4.MXFP4), dtype=torch.uint8, device=dev)
+        f = lambda: w4.linear(Xs, Wsm, 0, Y=Ysm, ws=wss)
+        for _ in range(10):
+            f()
+        ms = time_loop(f, 200, stream)
+        g = torch.cuda.CUDAGraph()
+        side = torch.cuda.Stream(dev)
+        side.wait_stream(stream)
+        with torch.cuda.stream(side):
+            f()
+        stream.wait_stream(side)
+        torch.cuda.synchronize()
+        with torch.cuda.graph(g):
+            f()
+        g.replay()
+        ms_g = time_loop(g.replay, 200, stream)
+        torch.cuda.synchronize()
+        out["mxfp4_small_16x256x256"] = {"us": round(ms * 1e3, 2), "graph_us": round(ms_g * 1e3, 2),
+                                         "_y": Ysm.view(torch.int16).cpu().numpy().view(np.uint16)}
+        del g
+
     if not want("mxfp4"):
         torch.cuda.synchronize()
         assert w4.device_status() == w4.OK
@@ -633,7 +834,8 @@ def main():
     ap.add_argument("--cpu-rows", type=int, default=8, help="cpu_baseline sample: tokens")
     ap.add_argument("--cpu-cols", type=int, default=4096, help="cpu_baseline sample: output columns")
     ap.add_argument("--no-rows", action="store_true", help="skip the secondary rows")
-    ap.add_argument("--only", choices=["gemm", "quant", "decode", "int4", "aug", "mxfp4", "segments", "msd", "hadamard", "tokens", "swiglu"], default=None,
+    ap.add_argument("--only", choices=["gemm", "quant", "decode", "int4", "aug", "mxfp4", "segments", "msd", "hadamard",
+                                       "tokens", "swiglu", "small"], default=None,
                     help="run only one secondary row (for profiling) and print it")
     ap.add_argument("--no-cpu", action="store_true", help="skip the oracle CPU baseline")
     ap.add_argument("--shape", default=None, help="--only gemm: one Llama linear (qkv, o, w1, w3, w2)")

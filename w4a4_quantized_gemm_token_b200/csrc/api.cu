@@ -139,9 +139,13 @@ cudaStream_t as_stream(void* s) { return reinterpret_cast<cudaStream_t>(s); }
 int cuda_status(cudaError_t e) { return e == cudaSuccess ? W4A4_OK : W4A4_ERR_CUDA; }
 
 // Quantize rows [0, M) of X into the first K columns of q (q->cols >= K).
+// pad_scales: also write the zero scales of the padding rows [M, pad128(M))
+// of the 128-row scale atoms (the public layout); the fused linear's
+// workspace skips them, since every GEMM masks rows past M.
 int quantize_rows(const uint16_t* X, int M, int K, int ldx, const int32_t* S, int K_src, const float* static_s2,
                   w4a4_qtensor* q, int num_sms, cudaStream_t st, int* zero_words = nullptr, int zero_count = 0,
-                  int passes = 1, bool weight_side = false) {
+                  int passes = 1, bool weight_side = false, bool pad_scales = true) {
+    const int rows_pad = pad_scales ? pad128(M) : M;
     QuantArgs a{};
     a.passes = passes;
     a.rot = (q->flags & W4A4_FLAG_HADAMARD) ? (weight_side ? 2 : 1) : 0;
@@ -173,14 +177,14 @@ int quantize_rows(const uint16_t* X, int M, int K, int ldx, const int32_t* S, in
         if (e != cudaSuccess) return W4A4_ERR_CUDA;
         a.tensor_amax = q->s2 + 1;
         if (!S && K == K_src && !a.rot && passes == 1 && !a.int8_codes && nvfp4_tensor_onepass_fits(M, K, num_sms)) {
-            e = launch_nvfp4_tensor_onepass(a, pad128(M), num_sms, reinterpret_cast<unsigned*>(q->s2 + 2), st);
+            e = launch_nvfp4_tensor_onepass(a, rows_pad, num_sms, reinterpret_cast<unsigned*>(q->s2 + 2), st);
             if (e != cudaErrorCooperativeLaunchTooLarge) return cuda_status(e);
             cudaGetLastError();  // fewer SMs available than reported: two passes
         }
         e = launch_amax(X, M, K_src, ldx, q->s2 + 1, num_sms, st, a.rot);
         if (e != cudaSuccess) return W4A4_ERR_CUDA;
     }
-    return cuda_status(launch_quant(q->format, S != nullptr, a, pad128(M), num_sms, st));
+    return cuda_status(launch_quant(q->format, S != nullptr, a, rows_pad, num_sms, st));
 }
 
 // NVFP4 weights with one s2 per row (per-segment scales): the GEMM epilogues
@@ -194,6 +198,23 @@ int check_S_args(const int32_t* S, int nS, int K) {
     if (nS < 0 || (nS > 0 && (!S || nS % 128 || nS > K))) return W4A4_ERR_INVALID_ARG;
     if (nS == 0 && S) return W4A4_ERR_INVALID_ARG;
     return W4A4_OK;
+}
+
+// The split-K small-M kernel (weights on the MMA's M side, every SM streaming
+// its share of the weights) or the tiled kernels (tokens on the M side, one
+// 128/256-row token tile against 256-row weight tiles), by the crossover
+// measured on the Llama-2-70B layer: the small-M kernel for M <= 16; for
+// 16 < M <= 64 unless N / 256 weight tiles already occupy every SM; for
+// 64 < M <= 128 only where the tiled kernel would run at most 32 long tiles
+// (K >= 16384) on as many SMs.  The small-M kernel pays an FP32 partial sum
+// per tile segment, which outweighs its parallelism beyond that.
+bool use_small_m(int fmt, int M, int N, int cols, int num_sms) {
+    if (fmt == W4A4_INT4 || decode_token_tile(M, cols) == 0) return false;
+    if (M <= 16) return true;
+    const int tiles = (N + kBN - 1) / kBN;
+    if (M <= 64) return tiles < num_sms / 2;
+    if (M <= 128) return tiles <= 32 && cols >= 16384;
+    return false;
 }
 
 struct GemmSetup {
@@ -247,10 +268,11 @@ int setup_gemm(const w4a4_qtensor* A, const w4a4_qtensor* B, uint16_t* Y, int ld
         rc = make_map(&s->ta, A->codes, A->rows, row_bytes, 128, kBM, true);
         if (rc == W4A4_OK) rc = make_map(&s->tb, B->codes, B->rows, row_bytes, 128, kBN, true);
     } else if (decode_k_blocks(A->cols) == 2) {
-        // weights take the MMA's M side (128 rows), tokens its N side (16 rows);
-        // both read as boxes of two consecutive 128-byte K-blocks per row
+        // weights take the MMA's M side (128 rows), tokens its N side (the token
+        // tile's rows); both read as boxes of two consecutive 128-byte K-blocks per row
         rc = make_map_kblocks(&s->ta, B->codes, B->rows, row_bytes, kBM, 2);
-        if (rc == W4A4_OK) rc = make_map_kblocks(&s->tb, A->codes, A->rows, row_bytes, kBN_DEC, 2);
+        if (rc == W4A4_OK)
+            rc = make_map_kblocks(&s->tb, A->codes, A->rows, row_bytes, decode_token_tile(A->rows, A->cols), 2);
     } else {
         // weights take the MMA's M side (box of 128 rows), tokens its N side (16 rows)
         rc = make_map(&s->ta, B->codes, B->rows, row_bytes, 128, kBM, true);
@@ -298,14 +320,17 @@ WsLayout ws_layout(int M, int N, int K, int fmt, int nS) {
     w.s2 = w.scales + align256(sb);
     w.partial = w.s2 + align256(s2b);
     size_t pb = 0;
-    if (fmt != W4A4_INT4 && M <= 16) {
-        // FP32 segment partials of the small-M variant: [tiles][owners][16][128];
-        // the owner count grows with the SM count, bounded here for up to 1024 SMs
+    // sized for the small-M variant whenever it can be chosen (on any SM count)
+    const bool small_m = use_small_m(fmt, M, N, cols, 1 << 20);
+    if (small_m) {
+        // FP32 segment partials of the small-M variant: [tiles][owners][token
+        // tile][128]; the owner count grows with the SM count, bounded here for
+        // up to 1024 SMs
         const int ntiles = (N + kBM - 1) / kBM;
-        pb = (size_t)ntiles * decode_max_owners(N, cols, 1024) * kBN_DEC * kBM * sizeof(float);
+        pb = (size_t)ntiles * decode_max_owners(N, cols, 1024) * decode_token_tile(M, cols) * kBM * sizeof(float);
     }
     w.counters = w.partial + align256(pb);
-    const size_t nb = (fmt != W4A4_INT4 && M <= 16) ? (size_t)((N + kBM - 1) / kBM) * sizeof(int) : 0;
+    const size_t nb = small_m ? (size_t)((N + kBM - 1) / kBM) * sizeof(int) : 0;
     w.total = w.counters + align256(nb);
     return w;
 }
@@ -544,10 +569,11 @@ int w4a4_linear(const uint16_t* X, int M, int K, int ldx, const w4a4_qtensor* Wq
     xq.codes = base + L.codes;
     xq.scales = base + L.scales;
     xq.s2 = reinterpret_cast<float*>(base + L.s2);
-    const bool small_m = fmt != W4A4_INT4 && M <= 16;
+    const bool small_m = use_small_m(fmt, M, N, xq.cols, sms);
     int* counters = small_m ? reinterpret_cast<int*>(base + L.counters) : nullptr;
     // the quantizer clears the decode GEMM's per-tile counters on its way
-    rc = quantize_rows(X, M, K, ldx, nullptr, K, nullptr, &xq, sms, st, counters, small_m ? (N + kBM - 1) / kBM : 0);
+    rc = quantize_rows(X, M, K, ldx, nullptr, K, nullptr, &xq, sms, st, counters, small_m ? (N + kBM - 1) / kBM : 0,
+                       1, false, false);
     if (rc != W4A4_OK) return rc;
     if (nS) {
         ResidualArgs r{X, M, K, ldx, pad128(M), S, nS, static_cast<uint8_t*>(xq.codes), xq.cols / 2,
@@ -587,10 +613,10 @@ int w4a4_linear_msd(const uint16_t* X, int M, int K, int ldx, const w4a4_qtensor
     xq.codes = base + L.codes;
     xq.scales = base + L.scales;
     xq.s2 = nullptr;
-    const bool small_m = M <= 16;
+    const bool small_m = use_small_m(W4A4_MXFP4, M, N, xq.cols, sms);
     int* counters = small_m ? reinterpret_cast<int*>(base + L.counters) : nullptr;
     rc = quantize_rows(X, M, K, ldx, nullptr, K, nullptr, &xq, sms, st, counters, small_m ? (N + kBM - 1) / kBM : 0,
-                       passes);
+                       passes, false, false);
     if (rc != W4A4_OK) return rc;
     float* partial = small_m ? reinterpret_cast<float*>(base + L.partial) : nullptr;
     return run_gemm(&xq, Wq, Y, ldy, partial, sms, true, st, counters);

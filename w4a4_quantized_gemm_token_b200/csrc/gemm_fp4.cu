@@ -1,8 +1,9 @@
 // Small-M ("decode") block-scaled FP4 GEMM: Y[M,N] = X[M,K] W[N,K]^T for
-// M <= 16, bound by streaming the 4-bit weights from HBM.
+// M <= 128, bound by streaming the 4-bit weights from HBM.
 //
 // The weights take the MMA's M side (128 rows per tile) and the tokens its N
-// side (16), so one tcgen05.mma kind::mxf4nvf4 covers 128 x 16 x 64.  A work
+// side (BN = 16, 32, 64 or 128: the smallest that holds M), so one
+// tcgen05.mma kind::mxf4nvf4 covers 128 x BN x 64.  A work
 // unit is a weight tile and KB consecutive K-stages of 256; the units are
 // split into equal contiguous ranges, one per SM (stream-K), so every SM
 // streams the same number of weight bytes whatever N and K are.  With KB = 2
@@ -10,8 +11,9 @@
 // contributes 256 contiguous bytes per copy instead of 128, which HBM serves
 // much faster, and the box still lands as standard 128-byte-swizzled tiles.
 // A CTA accumulates in TMEM while its range stays in one weight tile and
-// writes an FP32 partial sum per tile segment (double-buffered
-// accumulators); the CTA that writes a tile's last segment adds the tile's
+// writes an FP32 partial sum per tile segment (double-buffered accumulators
+// up to BN = 128, one of 256 columns for BN = 256); the CTA that writes a
+// tile's last segment adds the tile's
 // segments in a fixed order (deterministic), applies alpha and rounds to
 // bf16.  Launched as a
 // programmatic dependent, the kernel starts streaming weights while the
@@ -34,22 +36,30 @@ __device__ int g_error_word = 0;
 // 3-D box view needs K % 256 == 0), else one (2-D boxes).
 __host__ __device__ __forceinline__ int decode_kb(int K) { return K % kBK_FP4 == 0 ? 2 : 1; }
 
-template <int KB>
+template <int KB, int BN_>
 struct Dec {
-    static constexpr int BN = kBN_DEC;                 // tokens per MMA (16)
-    static constexpr int STAGES = KB == 2 ? 5 : 10;      // ~225 KB of shared memory in flight
+    static constexpr int BN = BN_;                     // tokens per MMA (the MMA's N)
+    static constexpr int TOK_TILES = BN > 128 ? 2 : 1; // 128-row tiles of the token scale atoms
+    static constexpr int ACC_BUFS = BN > 128 ? 1 : 2;  // accumulators of BN columns
     static constexpr int A_BYTES = KB * kBM * 128;     // weight tiles [kb][128 rows][128 B]
-    static constexpr int B_BYTES = KB * BN * 128;      // token tiles [kb][16 rows][128 B]
+    static constexpr int B_BYTES = KB * BN * 128;      // token tiles [kb][BN rows][128 B]
     static constexpr int ATOM = 512;
     static constexpr int SFA_C = KB * 4 * ATOM;        // weight scale atoms of a unit
-    static constexpr int SFB_C = KB * 4 * ATOM;        // token scale atoms of a unit
+    static constexpr int SFB_T = KB * 4 * ATOM;        // token scale atoms of a unit, per 128-row tile
+    static constexpr int SFB_C = TOK_TILES * SFB_T;
     static constexpr int STAGE = A_BYTES + B_BYTES + SFA_C + SFB_C;
+    static constexpr int SF_COLS = KB * 16 * (1 + TOK_TILES);  // per stage: weights, then tokens
+    static constexpr int SF_COL0 = ACC_BUFS * BN;              // after the accumulators
+    static constexpr int TMEM_COLS = 512;
+    static constexpr int SMEM_MAX = 232448 - 512 - 1024;
+    // as many stages as shared and tensor memory hold (at most 10)
+    static constexpr int S_SMEM = SMEM_MAX / STAGE, S_TMEM = (TMEM_COLS - SF_COL0) / SF_COLS;
+    static constexpr int STAGES = S_SMEM < S_TMEM ? (S_SMEM < 10 ? S_SMEM : 10) : (S_TMEM < 10 ? S_TMEM : 10);
     static constexpr int BAR_OFF = STAGES * STAGE;
     static constexpr int SMEM = BAR_OFF + 512 + 1024;
-    static constexpr int SF_COLS = KB * 32;            // per stage: weights KB*16 + tokens KB*16 columns
-    static constexpr int SF_COL0 = 2 * BN;             // after two accumulators of 16 columns
-    static constexpr int TMEM_COLS = 512;
     static constexpr int THREADS = 256;
+    static_assert(BN % 16 == 0 && BN <= 256, "MMA N");
+    static_assert(STAGES >= 2, "at least two stages");
     static_assert(STAGE % 1024 == 0, "stages keep the 1024-byte alignment of swizzled tiles");
     static_assert(SF_COL0 + STAGES * SF_COLS <= TMEM_COLS, "tensor memory holds 512 columns");
     static_assert(SMEM <= 232448, "shared memory per block");
@@ -79,13 +89,13 @@ __device__ __forceinline__ int unit_owner(long long u, long long U, int G) {
     return c;
 }
 
-template <bool NV, int KB>
-__global__ void __launch_bounds__(Dec<KB>::THREADS, 1)
+template <bool NV, int KB, int BN_>
+__global__ void __launch_bounds__(Dec<KB, BN_>::THREADS, 1)
     gemm_fp4_decode_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmX,
                            GemmArgs g) {
-    using D = Dec<KB>;
+    using D = Dec<KB, BN_>;
     constexpr int STAGES = D::STAGES, A_BYTES = D::A_BYTES, B_BYTES = D::B_BYTES, ATOM = D::ATOM;
-    constexpr int BN = D::BN;
+    constexpr int BN = D::BN, TT = D::TOK_TILES, NBUF = D::ACC_BUFS;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint64_t* full = reinterpret_cast<uint64_t*>(smem + D::BAR_OFF);
@@ -124,7 +134,7 @@ __global__ void __launch_bounds__(Dec<KB>::THREADS, 1)
             mbar_init(&empty[s], 1);
             mbar_init(&sfull[s], 1);
         }
-        for (int b = 0; b < 2; ++b) {
+        for (int b = 0; b < NBUF; ++b) {
             mbar_init(&accf[b], 1);
             mbar_init(&acce[b], 4);
         }
@@ -156,7 +166,7 @@ __global__ void __launch_bounds__(Dec<KB>::THREADS, 1)
                 unit_chunks(u, nk, atoms, k0);
                 uint8_t* st = smem + s * D::STAGE;
                 // full boxes (K-blocks past K are zero-filled) + the scale atoms in range
-                mbar_arrive_expect_tx(&full[s], (uint32_t)(A_BYTES + B_BYTES + 2 * atoms * ATOM));
+                mbar_arrive_expect_tx(&full[s], (uint32_t)(A_BYTES + B_BYTES + (1 + TT) * atoms * ATOM));
                 if (KB == 1)
                     tma_load_2d(st, &tmW, kt0 * 128, nt * kBM, &full[s]);
                 else
@@ -173,7 +183,11 @@ __global__ void __launch_bounds__(Dec<KB>::THREADS, 1)
                     tma_load_2d(st + A_BYTES, &tmX, kt0 * 128, 0, &full[s]);
                 else
                     tma_load_3d(st + A_BYTES, &tmX, 0, 0, kt0, &full[s]);
-                bulk_load(st + A_BYTES + B_BYTES + D::SFA_C, sfx + (size_t)k0 * ATOM, atoms * ATOM, &full[s]);
+                // the token scale atoms of each 128-row tile (rows past M are zero padding)
+#pragma unroll
+                for (int h = 0; h < TT; ++h)
+                    bulk_load(st + A_BYTES + B_BYTES + D::SFA_C + h * D::SFB_T,
+                              sfx + ((size_t)h * g.sf_col_atoms + k0) * ATOM, atoms * ATOM, &full[s]);
             };
             // stream the first weight units before the activations are known to be ready
             const int pre = min(STAGES, nunits);
@@ -203,8 +217,9 @@ __global__ void __launch_bounds__(Dec<KB>::THREADS, 1)
             while (u < u1 && ok) {
                 const int nt = (int)(u / KG);
                 const long long sbeg = u, send = min(u1, (long long)(nt + 1) * KG);
-                const int buf = seg & 1;
-                if (seg >= 2 && !mbar_wait(&acce[buf], ((seg >> 1) - 1) & 1, limit, abort_flag)) {
+                const int buf = NBUF == 2 ? (seg & 1) : 0;
+                const int use = NBUF == 2 ? (seg >> 1) : seg;  // earlier uses of this accumulator
+                if (use >= 1 && !mbar_wait(&acce[buf], (use - 1) & 1, limit, abort_flag)) {
                     ok = false;
                     break;
                 }
@@ -224,10 +239,12 @@ __global__ void __launch_bounds__(Dec<KB>::THREADS, 1)
                         const int kb = j >> 2, jj = j & 3;  // K-block of the unit, chunk within it
                         const int sfid = NV ? 0 : (j & 1) * 2;
                         const int aj = NV ? j : (j >> 1);
+                        // token scales: 4 columns per atom and 128-row tile (tile 1 of
+                        // BN = 256 at +4, where the MMA reads rows 128..255)
                         mma_fp4<NV>(tmem + buf * BN, desc_kmajor_sw128(sA + kb * (kBM * 128) + 32 * jj),
                                     desc_kmajor_sw128(sB + kb * (BN * 128) + 32 * jj),
                                     idesc_fp4(kBM, BN, !NV, sfid, sfid), (sfa_t + 4 * aj) | ((uint32_t)sfid << 30),
-                                    (sfb_t + 4 * aj) | ((uint32_t)sfid << 30), (u > sbeg || j > 0) ? 1u : 0u);
+                                    (sfb_t + 4 * TT * aj) | ((uint32_t)sfid << 30), (u > sbeg || j > 0) ? 1u : 0u);
                     }
                     tc_commit(&empty[s]);
                 }
@@ -257,7 +274,9 @@ __global__ void __launch_bounds__(Dec<KB>::THREADS, 1)
                 const uint32_t sfa_t = tmem + D::SF_COL0 + s * D::SF_COLS, sfb_t = sfa_t + 16 * KB;
                 for (int j = 0; j < atoms; ++j) {
                     tc_cp_32x128b_x4(sfa_t + 4 * j, desc_sf_32x16(ca + j * ATOM));
-                    tc_cp_32x128b_x4(sfb_t + 4 * j, desc_sf_32x16(cb + j * ATOM));
+#pragma unroll
+                    for (int h = 0; h < TT; ++h)
+                        tc_cp_32x128b_x4(sfb_t + 4 * TT * j + 4 * h, desc_sf_32x16(cb + h * D::SFB_T + j * ATOM));
                 }
                 tc_commit(sfull + s);
             }
@@ -268,7 +287,7 @@ __global__ void __launch_bounds__(Dec<KB>::THREADS, 1)
         }
     } else if (warp >= 4) {
         // ------------------------------ epilogue ------------------------------
-        // Segment partial sums -> workspace slot (tile, owner offset) [16 tokens][128
+        // Segment partial sums -> workspace slot (tile, owner offset) [BN tokens][128
         // rows] FP32.  The CTA whose segment completes a tile (a per-tile counter)
         // adds all the tile's slots in owner order -- the same order whichever CTA
         // arrives last -- applies alpha, writes Y and clears the counter.
@@ -283,22 +302,39 @@ __global__ void __launch_bounds__(Dec<KB>::THREADS, 1)
         while (u < u1) {
             const int nt = (int)(u / KG);
             const long long send = min(u1, (long long)(nt + 1) * KG);
-            const int buf = seg & 1;
+            const int buf = NBUF == 2 ? (seg & 1) : 0;
+            const int use = NBUF == 2 ? (seg >> 1) : seg;
             const int first = unit_owner((long long)nt * KG, U, G);
             const int last = unit_owner((long long)(nt + 1) * KG - 1, U, G);
             float* tile = g.partial + (size_t)nt * g.splits * (BN * kBM);
-            if (ok) ok = mbar_wait(&accf[buf], (seg >> 1) & 1, limit, abort_flag, 20000);
+            if (ok) ok = mbar_wait(&accf[buf], use & 1, limit, abort_flag, 20000);
             if (ok) {
                 tc_fence_after();
-                uint32_t r[16];
-                tmem_ld_32x32b_x16(tmem + ((uint32_t)(q * 32) << 16) + buf * BN, r);
-                tmem_ld_wait();
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&acce[buf]);
                 float* slot = tile + (size_t)(blockIdx.x - first) * (BN * kBM);
+                const uint32_t taddr = tmem + ((uint32_t)(q * 32) << 16) + buf * BN;
+                if constexpr (BN == 16) {
+                    uint32_t r[16];
+                    tmem_ld_32x32b_x16(taddr, r);
+                    tmem_ld_wait();
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&acce[buf]);
 #pragma unroll
-                for (int t = 0; t < BN; ++t) slot[t * kBM + row] = __uint_as_float(r[t]);
+                    for (int t = 0; t < BN; ++t) slot[t * kBM + row] = __uint_as_float(r[t]);
+                } else {
+                    // 32 tokens at a time: read, then store while the next chunk is read
+#pragma unroll 1
+                    for (int c = 0; c < BN / 32; ++c) {
+                        uint32_t r[32];
+                        tmem_ld_32x32b_x32(taddr + 32 * c, r);
+                        tmem_ld_wait();
+#pragma unroll
+                        for (int t = 0; t < 32; ++t) slot[(32 * c + t) * kBM + row] = __uint_as_float(r[t]);
+                    }
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&acce[buf]);
+                }
             }
             __threadfence();
             named_bar_sync(1, 128);  // the four epilogue warps wrote their rows
@@ -310,58 +346,62 @@ __global__ void __launch_bounds__(Dec<KB>::THREADS, 1)
             named_bar_sync(1, 128);
             if (last_flag) {
                 __threadfence();
-                // thread e of the 128 takes positions (token, 4 rows) p = e, e+128, ...:
-                // the float4 loads of all its positions and segments are issued
-                // before any addition, so the tile costs about one memory latency
+                // thread e of the 128 takes positions (token, 4 rows) p = e, e+128, ...,
+                // four at a time: the float4 loads of four positions and all their
+                // segments are issued before any addition
                 const int owners = last - first + 1, e = threadIdx.x - 128;
-                constexpr int PMAX = BN * kBM / 4 / 128, OMAX = 4;
-                float4 v[PMAX][OMAX];
+                constexpr int PMAX = BN * kBM / 4 / 128, PG = PMAX < 4 ? PMAX : 4, OMAX = 4;
+#pragma unroll 1
+                for (int p0 = 0; p0 < PMAX; p0 += PG) {
+                    float4 v[PG][OMAX];
 #pragma unroll
-                for (int pi = 0; pi < PMAX; ++pi) {
-                    const int p = e + 128 * pi, t = p >> 5, r4 = (p & 31) * 4;
-                    const float4* src = reinterpret_cast<const float4*>(tile + t * kBM + r4);
+                    for (int pi = 0; pi < PG; ++pi) {
+                        const int p = e + 128 * (p0 + pi), t = p >> 5, r4 = (p & 31) * 4;
+                        const float4* src = reinterpret_cast<const float4*>(tile + t * kBM + r4);
 #pragma unroll
-                    for (int c = 0; c < OMAX; ++c)
-                        if (t < g.M && c < owners) v[pi][c] = src[(size_t)c * (BN * kBM / 4)];
-                }
+                        for (int c = 0; c < OMAX; ++c)
+                            if (t < g.M && c < owners) v[pi][c] = src[(size_t)c * (BN * kBM / 4)];
+                    }
 #pragma unroll
-                for (int pi = 0; pi < PMAX; ++pi) {
-                    const int p = e + 128 * pi, t = p >> 5, r4 = (p & 31) * 4;
-                    if (t >= g.M) continue;
-                    const float4* src = reinterpret_cast<const float4*>(tile + t * kBM + r4);
-                    float4 acc = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
-                    // fixed order: owner offset 0, 1, ...
+                    for (int pi = 0; pi < PG; ++pi) {
+                        const int p = e + 128 * (p0 + pi), t = p >> 5, r4 = (p & 31) * 4;
+                        if (t >= g.M) continue;
+                        const float4* src = reinterpret_cast<const float4*>(tile + t * kBM + r4);
+                        float4 acc = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+                        // fixed order: owner offset 0, 1, ...
 #pragma unroll
-                    for (int c = 0; c < OMAX; ++c)
-                        if (c < owners) {
-                            acc.x += v[pi][c].x;
-                            acc.y += v[pi][c].y;
-                            acc.z += v[pi][c].z;
-                            acc.w += v[pi][c].w;
+                        for (int c = 0; c < OMAX; ++c)
+                            if (c < owners) {
+                                acc.x += v[pi][c].x;
+                                acc.y += v[pi][c].y;
+                                acc.z += v[pi][c].z;
+                                acc.w += v[pi][c].w;
+                            }
+                        for (int c = OMAX; c < owners; ++c) {
+                            const float4 w = src[(size_t)c * (BN * kBM / 4)];
+                            acc.x += w.x;
+                            acc.y += w.y;
+                            acc.z += w.z;
+                            acc.w += w.w;
                         }
-                    for (int c = OMAX; c < owners; ++c) {
-                        const float4 w = src[(size_t)c * (BN * kBM / 4)];
-                        acc.x += w.x;
-                        acc.y += w.y;
-                        acc.z += w.z;
-                        acc.w += w.w;
+                        const int n = nt * kBM + r4;
+                        // alpha per output column: s2 of token t times s2 of weight row n
+                        // (one weight scale, or one per row for per-segment weights)
+                        float4 al = make_float4(1.0f, 1.0f, 1.0f, 1.0f);
+                        if (NV) {
+                            const float sa = g.s2a[g.s2a_per_row ? t : 0];
+                            const float4 sb = g.s2b_per_row
+                                                  ? *reinterpret_cast<const float4*>(g.s2b + min(n, g.N - 4))
+                                                  : make_float4(g.s2b[0], g.s2b[0], g.s2b[0], g.s2b[0]);
+                            al = make_float4(__fmul_rn(sa, sb.x), __fmul_rn(sa, sb.y), __fmul_rn(sa, sb.z),
+                                             __fmul_rn(sa, sb.w));
+                        }
+                        __nv_bfloat162 h0 = __floats2bfloat162_rn(__fmul_rn(acc.x, al.x), __fmul_rn(acc.y, al.y));
+                        __nv_bfloat162 h1 = __floats2bfloat162_rn(__fmul_rn(acc.z, al.z), __fmul_rn(acc.w, al.w));
+                        if (n < g.N)
+                            *reinterpret_cast<uint2*>(g.Y + (size_t)t * g.ldy + n) =
+                                make_uint2(*reinterpret_cast<uint32_t*>(&h0), *reinterpret_cast<uint32_t*>(&h1));
                     }
-                    const int n = nt * kBM + r4;
-                    // alpha per output column: s2 of token t times s2 of weight row n
-                    // (one weight scale, or one per row for per-segment weights)
-                    float4 al = make_float4(1.0f, 1.0f, 1.0f, 1.0f);
-                    if (NV) {
-                        const float sa = g.s2a[g.s2a_per_row ? t : 0];
-                        const float4 sb = g.s2b_per_row ? *reinterpret_cast<const float4*>(g.s2b + min(n, g.N - 4))
-                                                        : make_float4(g.s2b[0], g.s2b[0], g.s2b[0], g.s2b[0]);
-                        al = make_float4(__fmul_rn(sa, sb.x), __fmul_rn(sa, sb.y), __fmul_rn(sa, sb.z),
-                                         __fmul_rn(sa, sb.w));
-                    }
-                    __nv_bfloat162 h0 = __floats2bfloat162_rn(__fmul_rn(acc.x, al.x), __fmul_rn(acc.y, al.y));
-                    __nv_bfloat162 h1 = __floats2bfloat162_rn(__fmul_rn(acc.z, al.z), __fmul_rn(acc.w, al.w));
-                    if (n < g.N)
-                        *reinterpret_cast<uint2*>(g.Y + (size_t)t * g.ldy + n) =
-                            make_uint2(*reinterpret_cast<uint32_t*>(&h0), *reinterpret_cast<uint32_t*>(&h1));
                 }
                 if (threadIdx.x == 128) g.tile_count[nt] = 0;  // ready for the next call
             }
@@ -411,29 +451,46 @@ int decode_max_owners(int N, int K, int num_sms) {
     return (int)((KG + per - 1) / per) + 1;
 }
 
-template <bool NV, int KB>
+template <bool NV, int KB, int BN>
 static cudaError_t launch_dec_t(const CUtensorMap& tmW, const CUtensorMap& tmX, const GemmArgs& g0, int num_sms,
                                 cudaStream_t st) {
-    auto kern = gemm_fp4_decode_kernel<NV, KB>;
+    using D = Dec<KB, BN>;
+    auto kern = gemm_fp4_decode_kernel<NV, KB, BN>;
     static SmemAttrCache attr;
-    cudaError_t e = ensure_dynamic_smem(reinterpret_cast<const void*>(kern), Dec<KB>::SMEM, attr);
+    cudaError_t e = ensure_dynamic_smem(reinterpret_cast<const void*>(kern), D::SMEM, attr);
     if (e != cudaSuccess) return e;
     GemmArgs g = g0;
     const int G = decode_grid(g.N, g.K, num_sms);
     g.splits = decode_max_owners(g.N, g.K, num_sms);  // slots per weight tile in the workspace
     CUtensorMap a = tmW, b = tmX;
     void* args[] = {&a, &b, &g};
-    return launch_pdl(reinterpret_cast<const void*>(kern), dim3(G), dim3(Dec<KB>::THREADS), Dec<KB>::SMEM, st,
-                      args);
+    return launch_pdl(reinterpret_cast<const void*>(kern), dim3(G), dim3(D::THREADS), D::SMEM, st, args);
 }
 
 int decode_k_blocks(int K) { return decode_kb(K); }
 
+int decode_token_tile(int M, int K) {
+    if (M <= 16) return kBN_DEC;
+    if (M > 128 || decode_kb(K) != 2) return 0;
+    return M <= 32 ? 32 : M <= 64 ? 64 : 128;
+}
+
+template <bool NV>
+static cudaError_t launch_dec_nv(const CUtensorMap& tmW, const CUtensorMap& tmX, const GemmArgs& g, int num_sms,
+                                 cudaStream_t st) {
+    switch (decode_token_tile(g.M, g.K)) {
+        case 16: return decode_kb(g.K) == 2 ? launch_dec_t<NV, 2, 16>(tmW, tmX, g, num_sms, st)
+                                            : launch_dec_t<NV, 1, 16>(tmW, tmX, g, num_sms, st);
+        case 32: return launch_dec_t<NV, 2, 32>(tmW, tmX, g, num_sms, st);
+        case 64: return launch_dec_t<NV, 2, 64>(tmW, tmX, g, num_sms, st);
+        case 128: return launch_dec_t<NV, 2, 128>(tmW, tmX, g, num_sms, st);
+        default: return cudaErrorInvalidValue;
+    }
+}
+
 cudaError_t launch_gemm_fp4_decode(bool nvfp4, const CUtensorMap& tmW, const CUtensorMap& tmX, const GemmArgs& g,
                                    int num_sms, cudaStream_t st) {
-    if (decode_kb(g.K) == 2)
-        return nvfp4 ? launch_dec_t<true, 2>(tmW, tmX, g, num_sms, st) : launch_dec_t<false, 2>(tmW, tmX, g, num_sms, st);
-    return nvfp4 ? launch_dec_t<true, 1>(tmW, tmX, g, num_sms, st) : launch_dec_t<false, 1>(tmW, tmX, g, num_sms, st);
+    return nvfp4 ? launch_dec_nv<true>(tmW, tmX, g, num_sms, st) : launch_dec_nv<false>(tmW, tmX, g, num_sms, st);
 }
 
 }  // namespace w4a4

@@ -17,14 +17,16 @@
 // an MXFP4 stage 6; each copy replicates its 32 x 16-byte source into the
 // four 32-lane sub-partitions, where the MMA reads row r's scales from
 // column base + r/32.
-// Warp roles (256 threads):
+// Warp roles (640 threads):
 //   warp 0 lane 0   TMA producer: A/B codes (128-byte swizzled K-major tiles of
 //                   256 elements) and compact scale atoms, 4-stage ring.
 //   warp 1          TMEM owner; lane 0 issues 4 MMAs (K = 64) per stage.
 //   warp 2 lane 0   scale-factor copies into a per-stage TMEM region.
-//   warps 4..7      epilogue: TMEM -> registers (lane quarter = warp % 4),
-//                   x alpha, bf16; the accumulator is released as soon as it
-//                   is in registers, the stores overlap the next tile.
+//   warps 4..19     epilogue: TMEM -> registers (lane quarter = warp % 4,
+//                   64-column slice (warp - 4) / 4), x alpha, bf16; the
+//                   accumulator is released as soon as it is in registers,
+//                   the stores (transposed in groups of four lanes, whole
+//                   128-byte lines of Y) overlap the next tile.
 // Every wait is bounded; on expiry the kernel records a timeout, drains what
 // it has in flight, frees TMEM and returns.
 #include <cstdint>
@@ -49,7 +51,8 @@ constexpr int SMEM = BAR_OFF + 256 + 1024;
 constexpr int SF_COLS = 48;                   // TMEM per stage: A up to 16 + B 32 columns
 constexpr int SF_COL0 = BN;                   // after the accumulator
 constexpr int TMEM_COLS = 512;
-constexpr int THREADS = 256;
+constexpr int EPI_WARPS = 16;                 // four per TMEM lane quarter, 64 columns each
+constexpr int THREADS = (4 + EPI_WARPS) * 32;
 static_assert(STAGE % 1024 == 0, "stages keep the 1024-byte alignment of swizzled tiles");
 static_assert(SF_COL0 + STAGES * SF_COLS <= TMEM_COLS, "tensor memory holds 512 columns");
 static_assert(SMEM <= 232448, "shared memory per block");
@@ -95,7 +98,7 @@ __global__ void __launch_bounds__(pf::THREADS, 1)
             mbar_init(&sfull[s], 1);
         }
         mbar_init(accf, 1);
-        mbar_init(acce, 4);
+        mbar_init(acce, pf::EPI_WARPS);
         mbar_init(drain, 1);
         mbar_init(drain2, 1);
         *abort_flag = 0;
@@ -220,32 +223,36 @@ __global__ void __launch_bounds__(pf::THREADS, 1)
         }
     } else if (warp >= 4) {
         // ------------------------------ epilogue ------------------------------
-        const int q = warp & 3;
+        const int q = warp & 3, slice = (warp - 4) >> 2;
+        const bool y32 = (reinterpret_cast<uintptr_t>(g.Y) & 31) == 0 && (g.ldy & 15) == 0;
+        const int j = lane & 3;  // place in the lane's group of four
         int ti = 0;
         for (int t = blockIdx.x; t < ntiles; t += gridDim.x, ++ti) {
             int at, bt;
             coords(t, at, bt);
-            // per-row B scales of the tile's columns, lane l holding column
-            // 32 * ch + l, fetched before the accumulator is ready (clamped
-            // inside N past its end, which is a multiple of 128)
-            float sbl[8];
+            const int n0 = bt * BN + slice * 64;
+            // per-row B scales of the slice's 64 columns, lane l holding column
+            // 32 * ch + l, fetched before the accumulator is ready (N is a
+            // multiple of 128: a slice is wholly inside N or wholly past it)
+            float sbl[2];
             if constexpr (PB) {
 #pragma unroll
-                for (int ch = 0; ch < 8; ++ch) sbl[ch] = g.s2b[min(bt * BN + 32 * ch, g.N - 32) + lane];
+                for (int ch = 0; ch < 2; ++ch) sbl[ch] = g.s2b[min(n0, g.N - 64) + 32 * ch + lane];
             }
             if (!mbar_wait(accf, ti & 1, limit, abort_flag, 100000)) break;
             tc_fence_after();
-            const int m = at * kBM + q * 32 + lane;
+            const int m0 = at * kBM + q * 32;
+            const int m = m0 + lane;
             float alpha = 1.0f, sa = 0.0f;
             if (NV && m < g.M) {
                 sa = g.s2a[g.s2a_per_row ? m : 0];
                 alpha = __fmul_rn(sa, g.s2b[0]);
             }
-            uint32_t pk[128];
+            uint32_t pk[32];
 #pragma unroll
-            for (int ch = 0; ch < 8; ++ch) {
+            for (int ch = 0; ch < 2; ++ch) {
                 uint32_t r[32];
-                tmem_ld_32x32b_x32(tmem + ((uint32_t)(q * 32) << 16) + 32 * ch, r);
+                tmem_ld_32x32b_x32(tmem + ((uint32_t)(q * 32) << 16) + slice * 64 + 32 * ch, r);
                 tmem_ld_wait();
 #pragma unroll
                 for (int e = 0; e < 16; ++e) {
@@ -262,13 +269,36 @@ __global__ void __launch_bounds__(pf::THREADS, 1)
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(acce);  // accumulator may be overwritten now
-            if (m < g.M) {
-                const int n0 = bt * BN;
-                const int nv = min(BN, g.N - n0) / 8;  // 16-byte vectors in range
-                uint4* dst = reinterpret_cast<uint4*>(g.Y + (size_t)m * g.ldy + n0);
+            if (n0 >= g.N) continue;
+            // 4 x 4 transpose of 32-byte units inside each group of four lanes:
+            // lane 4i + j then holds unit j of rows 4i .. 4i + 3
 #pragma unroll
-                for (int v = 0; v < 32; ++v)
-                    if (v < nv) dst[v] = make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
+            for (int sft = 2; sft >= 1; sft >>= 1) {
+#pragma unroll
+                for (int u0 = 0; u0 < 4; ++u0) {
+                    if (u0 & sft) continue;
+                    const int u1 = u0 | sft;
+#pragma unroll
+                    for (int w = 0; w < 8; ++w) {
+                        const uint32_t snd = (j & sft) ? pk[8 * u0 + w] : pk[8 * u1 + w];
+                        const uint32_t rcv = __shfl_xor_sync(0xffffffffu, snd, sft);
+                        if (j & sft) pk[8 * u0 + w] = rcv;
+                        else pk[8 * u1 + w] = rcv;
+                    }
+                }
+            }
+            const int rg = m0 + (lane & ~3);
+#pragma unroll
+            for (int r = 0; r < 4; ++r) {
+                if (rg + r >= g.M) break;
+                uint16_t* dst = g.Y + (size_t)(rg + r) * g.ldy + n0 + 16 * j;
+                if (y32) {
+                    st_global_v8(dst, pk + 8 * r);
+                } else {
+                    uint4* d4 = reinterpret_cast<uint4*>(dst);
+                    d4[0] = make_uint4(pk[8 * r], pk[8 * r + 1], pk[8 * r + 2], pk[8 * r + 3]);
+                    d4[1] = make_uint4(pk[8 * r + 4], pk[8 * r + 5], pk[8 * r + 6], pk[8 * r + 7]);
+                }
             }
         }
     }

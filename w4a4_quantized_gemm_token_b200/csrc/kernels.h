@@ -120,13 +120,19 @@ cudaError_t launch_gemm_fp4(bool nvfp4, const CUtensorMap& tmA, const CUtensorMa
 // four times (boxes of one stage's atoms for 1 (A) and 2 (B) row tiles).
 cudaError_t launch_gemm_fp4_pair(bool nvfp4, const CUtensorMap& tmA, const CUtensorMap& tmB, const CUtensorMap& tmSA,
                                  const CUtensorMap& tmSB, const GemmArgs& g, int num_sms, bool pdl, cudaStream_t st);
-// Small-M variant (M <= 16): weights take the MMA's M side (128 rows per tile),
-// the tokens its N side; the (tile, K-stage) units are split evenly over the
-// SMs, FP32 segment partials go to g.partial and the CTA that writes a tile's
-// last segment adds them into Y (g.tile_count[N/128] must be zero on entry and
-// is zero again on exit).  A programmatic dependent of the preceding launch.
+// Small-M variant (M <= 128): weights take the MMA's M side (128 rows per
+// tile), the tokens its N side (decode_token_tile(M, K) rows); the (tile,
+// K-stage) units are split evenly over the SMs, FP32 segment partials go to
+// g.partial ([tiles][owners][token tile][128]) and the CTA that writes a
+// tile's last segment adds them into Y (g.tile_count[N/128] must be zero on
+// entry and is zero again on exit).  A programmatic dependent of the
+// preceding launch.
 cudaError_t launch_gemm_fp4_decode(bool nvfp4, const CUtensorMap& tmW, const CUtensorMap& tmX, const GemmArgs& g,
                                    int num_sms, cudaStream_t st);
+// Token tile (the MMA's N) of the small-M variant for M tokens and K
+// columns: 16 for M <= 16; 32, 64 or 128 for 16 < M <= 128 when K is a
+// multiple of 256; 0 when the variant does not apply.
+int decode_token_tile(int M, int K);
 // Partial-sum slots per weight tile of the small-M variant on `num_sms` SMs.
 int decode_max_owners(int N, int K, int num_sms);
 // K-stages of 256 per work unit of the small-M variant: 2 (weights and tokens

@@ -55,6 +55,9 @@ __device__ __forceinline__ uint32_t e2m1x8(const float (&v)[8]) {
 // Correctly rounded quotient x/d from a correctly rounded reciprocal
 // y = RN(1/d): q = RN(x*y) is within an ulp of x/d, the residual x - q*d is
 // exact in one FMA, and one more FMA rounds q + residual*y to RN(x/d).  This
+// is Markstein's correction theorem for FMA-based division (P. Markstein,
+// IBM J. Res. Dev. 34(1), 1990; restated in Muller et al., Handbook of
+// Floating-Point Arithmetic, the section on Newton-Raphson division).  This
 // holds whenever the quotient is a normal float; the callers keep operands in
 // that range (or their results do not depend on it: quotients below the
 // normal range encode to zero anyway) and fall back to IEEE division outside.
@@ -1175,6 +1178,10 @@ static cudaError_t launch_nvfp4_token(const QuantArgs& a, int rows_pad, int num_
     if (smem > 220 * 1024) return cudaErrorInvalidValue;
     int grid = num_sms * per_sm;
     if (grid > rows_pad) grid = rows_pad;
+    // a few tokens (decode): as many CTAs as rows (they also write the zero
+    // scales of the padding rows), so that the few SMs they take are all the
+    // next launch has to wait for before it can start streaming its weights
+    if (a.M <= 16 && grid > (a.M > 4 ? a.M : 4)) grid = a.M > 4 ? a.M : 4;
     QuantArgs b = a;
     b.rows_pad = rows_pad;
     cudaError_t e;
@@ -1203,7 +1210,14 @@ static cudaError_t launch_quant_fmt(const QuantArgs& a, int rows_pad, int num_sm
     const int items = rpc * (a.K / 16);
     const int T = items < 256 ? (items + 31) / 32 * 32 : 256;
     const int nblocks = (rows_pad + rpc - 1) / rpc;
-    const int grid = nblocks;
+    int grid = nblocks;
+    // a few tokens (decode): few CTAs, which also write the padding rows' zero
+    // scales (the kernel walks row blocks blockIdx.x, +gridDim.x, ...)
+    if (a.M <= 16) {
+        const int live = (a.M + rpc - 1) / rpc;
+        const int want = live > 4 ? live : 4;
+        if (grid > want) grid = want;
+    }
     (void)num_sms;
     QuantArgs b = a;
     b.rows_pad = rows_pad;

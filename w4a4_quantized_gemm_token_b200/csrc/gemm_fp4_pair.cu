@@ -27,18 +27,15 @@
 // count their bytes on the even CTA's stage barrier (cta_group::2 form),
 // whose expected byte count covers both CTAs.  Out-of-range row tiles and K
 // tails are zero-filled by the copies.
-// Warp roles (640 threads per CTA):
+// Warp roles (384 threads per CTA):
 //   warp 0 lane 0   TMA producer (both CTAs), 4-stage (NVFP4) / 5-stage (MXFP4) ring;
 //                   each stage (56 KB NVFP4) is near the rate at which TMA fills
 //                   shared memory (~64 B per cycle per SM), the bound of this kernel
 //   warp 1          TMEM allocation (both CTAs, together); even CTA lane 0
 //                   issues the MMAs
 //   warp 2          even CTA lane 0 issues the scale-factor copies
-//   warps 4..19     epilogue (both CTAs): TMEM -> registers -> bf16 stores,
-//                   four warps per lane quarter so the accumulator (which the
-//                   next tile's MMAs wait for) drains fast; the stores leave
-//                   after the release, transposed within groups of four lanes
-//                   so that each writes whole 128-byte lines of Y
+//   warps 4..11     epilogue (both CTAs): TMEM -> registers -> bf16 stores,
+//                   two warps per lane quarter so the accumulator drains fast
 // Every wait is bounded; on expiry the kernel records a timeout, drains its
 // copies and MMAs, frees TMEM and returns.
 #include <cstdint>
@@ -60,8 +57,8 @@ constexpr int REP = 4;                        // each atom staged 4 times (the T
 constexpr int SF_COLS = 48;                   // TMEM per stage: A 16 + B 32 columns
 constexpr int SF_COL0 = BN;                   // after the accumulator
 constexpr int TMEM_COLS = 512;
-constexpr int EPI_WARPS = 16;                 // four per TMEM lane quarter, 64 columns each
-constexpr int THREADS = (4 + EPI_WARPS) * 32;
+constexpr int THREADS = 384;
+constexpr int EPI_WARPS = 8;                  // two per TMEM lane quarter, 128 columns each
 // Per format: NVFP4 stages 4 scale atoms per 128 rows and K-stage, MXFP4 2.
 template <bool NV>
 struct Cfg {
@@ -149,6 +146,9 @@ __global__ void __launch_bounds__(pp::THREADS, 1)
     cluster_sync();  // both CTAs' barriers and tensor memory exist from here on
     tc_fence_after();
     const uint32_t tmem = *tmem_holder;
+    // the next launch (the next linear's quantizer) may be placed on SMs as
+    // this grid's CTAs finish; it waits for this grid before touching memory
+    pdl_launch_dependents();
     const uint32_t full_leader = mapa_shared(smem_u32(full), 0);
     const uint32_t acce_leader = mapa_shared(smem_u32(acce), 0);
     // operands written by the preceding kernel (A, its scales, s2a) are visible
@@ -279,39 +279,36 @@ __global__ void __launch_bounds__(pp::THREADS, 1)
         }
     } else if (warp >= 4) {
         // ------------------------------ epilogue ------------------------------
-        // warp w reads TMEM lane quarter w % 4 (rows q*32..) and the 64-column
-        // slice (w - 4) / 4 of the accumulator (64 outputs of its row)
-        const int q = warp & 3, slice = (warp - 4) >> 2;
-        // rows of Y start on 32-byte boundaries: 32-byte stores
+        // warp w reads TMEM lane quarter w % 4 (rows q*32..) and column half
+        // (w - 4) / 4 (128 accumulator columns = 128 outputs of its row)
+        const int q = warp & 3, half = (warp - 4) >> 2;
+        // rows of Y start on 32-byte boundaries: whole-sector stores
         const bool y32 = (reinterpret_cast<uintptr_t>(g.Y) & 31) == 0 && (g.ldy & 15) == 0;
-        const int j = lane & 3;  // place in the lane's group of four
         int ti = 0;
         for (int t = pair; t < ntiles; t += npairs, ++ti) {
             int at, bt;
             coords(t, at, bt);
-            const int n0 = bt * BN + slice * 64;
-            // per-row B scales of these 64 columns, lane l holding column
+            // per-row B scales of these 128 columns, lane l holding column
             // 32 * ch + l, fetched before the accumulator is ready (N is a
-            // multiple of 128: a slice is wholly inside N or wholly past it)
-            float sbl[2];
+            // multiple of 128: a half tile is wholly inside N or wholly past it)
+            float sbl[4];
             if constexpr (PB) {
 #pragma unroll
-                for (int ch = 0; ch < 2; ++ch) sbl[ch] = g.s2b[min(n0, g.N - 64) + 32 * ch + lane];
+                for (int ch = 0; ch < 4; ++ch) sbl[ch] = g.s2b[min(bt * BN + half * 128, g.N - 128) + 32 * ch + lane];
             }
             if (!mbar_wait(accf, ti & 1, limit, abort_flag, 100000)) break;
             tc_fence_after();
-            const int m0 = at * BM + (int)rank * HALF + q * 32;  // row of lane 0
-            const int m = m0 + lane;
+            const int m = at * BM + (int)rank * HALF + q * 32 + lane;
             float alpha = 1.0f, sa = 0.0f;
             if (NV && m < g.M) {
                 sa = g.s2a[g.s2a_per_row ? m : 0];
                 alpha = __fmul_rn(sa, g.s2b[0]);
             }
-            uint32_t pk[32];  // bf16 pairs of the row's 64 columns
+            uint32_t pk[64];
 #pragma unroll
-            for (int ch = 0; ch < 2; ++ch) {
+            for (int ch = 0; ch < 4; ++ch) {
                 uint32_t r[32];
-                tmem_ld_32x32b_x32(tmem + ((uint32_t)(q * 32) << 16) + slice * 64 + 32 * ch, r);
+                tmem_ld_32x32b_x32(tmem + ((uint32_t)(q * 32) << 16) + half * 128 + 32 * ch, r);
                 tmem_ld_wait();
 #pragma unroll
                 for (int e = 0; e < 16; ++e) {
@@ -328,37 +325,22 @@ __global__ void __launch_bounds__(pp::THREADS, 1)
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive_cluster(acce_leader);  // this part of the accumulator is free
-            if (n0 >= g.N) continue;
-            // 4 x 4 transpose of 32-byte units (16 columns) inside each group of
-            // four lanes: lane 4i + j then holds unit j of rows 4i .. 4i + 3, so
-            // each store below writes four lanes x 32 bytes = one 128-byte line
-            // of a row (xor butterflies over lane bits 1 and 0)
+            if (m < g.M) {
+                const int n0 = bt * BN + half * 128;
+                const int nv = max(0, min(128, g.N - n0)) / 8;  // 16-byte vectors in range
+                uint16_t* row = g.Y + (size_t)m * g.ldy + n0;
+                if (y32 && nv == 16) {
+                    // whole sectors: 32 bytes per lane and store (each lane writes
+                    // its own row, so 16-byte stores would write half sectors and
+                    // hold up the next tile's loads for microseconds; measured
+                    // faster overall than transposing into whole lines first)
 #pragma unroll
-            for (int sft = 2; sft >= 1; sft >>= 1) {
-#pragma unroll
-                for (int u0 = 0; u0 < 4; ++u0) {
-                    if (u0 & sft) continue;
-                    const int u1 = u0 | sft;
-#pragma unroll
-                    for (int w = 0; w < 8; ++w) {
-                        const uint32_t snd = (j & sft) ? pk[8 * u0 + w] : pk[8 * u1 + w];
-                        const uint32_t rcv = __shfl_xor_sync(0xffffffffu, snd, sft);
-                        if (j & sft) pk[8 * u0 + w] = rcv;
-                        else pk[8 * u1 + w] = rcv;
-                    }
-                }
-            }
-            const int rg = m0 + (lane & ~3);  // first row of this lane's group
-#pragma unroll
-            for (int r = 0; r < 4; ++r) {
-                if (rg + r >= g.M) break;
-                uint16_t* dst = g.Y + (size_t)(rg + r) * g.ldy + n0 + 16 * j;
-                if (y32) {
-                    st_global_v8(dst, pk + 8 * r);
+                    for (int v = 0; v < 8; ++v) st_global_v8(row + 16 * v, pk + 8 * v);
                 } else {
-                    uint4* d4 = reinterpret_cast<uint4*>(dst);
-                    d4[0] = make_uint4(pk[8 * r], pk[8 * r + 1], pk[8 * r + 2], pk[8 * r + 3]);
-                    d4[1] = make_uint4(pk[8 * r + 4], pk[8 * r + 5], pk[8 * r + 6], pk[8 * r + 7]);
+                    uint4* dst = reinterpret_cast<uint4*>(row);
+#pragma unroll
+                    for (int v = 0; v < 16; ++v)
+                        if (v < nv) dst[v] = make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
                 }
             }
         }

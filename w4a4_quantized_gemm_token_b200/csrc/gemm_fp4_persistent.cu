@@ -116,6 +116,7 @@ __global__ void __launch_bounds__(pf::THREADS, 1)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_holder;
+    pdl_launch_dependents();  // the next launch may be placed as this grid's CTAs finish
     pdl_wait();  // operands written by the preceding kernel are visible from here on
 
     if (warp == 0) {

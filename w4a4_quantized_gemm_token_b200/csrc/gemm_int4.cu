@@ -37,8 +37,14 @@ constexpr int STAGES = 4;
 constexpr int PK_BYTES = 128 * 64;      // packed 128 rows x 128 nibbles
 constexpr int UN_BYTES = 128 * 128;     // unpacked 128 rows x 128 int8
 constexpr int STAGE = 2 * UN_BYTES + 2 * PK_BYTES;  // unpacked A, B, then packed A, B
-constexpr int SB_OFF = STAGES * STAGE;              // 2 x 128 floats of B scales
-constexpr int BAR_OFF = SB_OFF + 2 * 128 * 4;
+// Scale ring: the A and B scales of one scale group (128 + 128 floats, 512
+// contiguous bytes each in the group-major layout) are staged by the
+// producer when the group's first stage loads, SR groups ahead of the
+// rescale warps, so no global-memory latency sits on the rescale path.
+constexpr int SR = 8;
+constexpr int SC_BYTES = 2 * 128 * 4;
+constexpr int SC_OFF = STAGES * STAGE;
+constexpr int BAR_OFF = SC_OFF + SR * SC_BYTES;
 constexpr int SMEM = BAR_OFF + 512 + 1024;
 constexpr int THREADS = 14 * 32;
 constexpr int TMEM_COLS = 256;                      // two int32 buffers of 128 columns
@@ -74,14 +80,16 @@ __global__ void __launch_bounds__(i4::THREADS, 1)
     using namespace i4;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    float* sb_smem = reinterpret_cast<float*>(smem + SB_OFF);
+    const float* sc_smem = reinterpret_cast<const float*>(smem + SC_OFF);
     uint64_t* full = reinterpret_cast<uint64_t*>(smem + BAR_OFF);
     uint64_t* conv = full + STAGES;
     uint64_t* empty = conv + STAGES;
     uint64_t* accf = empty + STAGES;    // [2]
     uint64_t* tfree = accf + 2;         // [2]
     uint64_t* drain = tfree + 2;
-    uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(drain + 1);
+    uint64_t* scfull = drain + 1;       // [SR] scales of a group landed
+    uint64_t* scfree = scfull + SR;     // [SR] the rescale warps are done with a slot
+    uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(scfree + SR);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -111,6 +119,10 @@ __global__ void __launch_bounds__(i4::THREADS, 1)
             mbar_init(&tfree[b], 8);
         }
         mbar_init(drain, 1);
+        for (int i = 0; i < SR; ++i) {
+            mbar_init(&scfull[i], 1);
+            mbar_init(&scfree[i], 8);
+        }
         *abort_flag = 0;
         fence_mbar_init();
     }
@@ -131,8 +143,10 @@ __global__ void __launch_bounds__(i4::THREADS, 1)
     // gi counts the groups of every tile this CTA processes, in order
     if (warp == 0) {
         if (lane == 0) {
-            int gi = 0;
+            int gi = 0, gg = 0;  // stages and scale groups issued
             bool stop = false;
+            const float* sfa = reinterpret_cast<const float*>(g.sfa);
+            const float* sfb = reinterpret_cast<const float*>(g.sfb);
             for (int t = blockIdx.x; t < ntiles && !stop; t += gridDim.x) {
                 int m_tile, n_tile;
                 coords(t, m_tile, n_tile);
@@ -141,6 +155,18 @@ __global__ void __launch_bounds__(i4::THREADS, 1)
                     if (gi >= STAGES && !mbar_wait(&empty[s], (n - 1) & 1, limit, abort_flag)) {
                         stop = true;
                         break;
+                    }
+                    if (k % R == 0) {  // this group's scales, into its ring slot
+                        const int slot = gg % SR;
+                        if (gg >= SR && !mbar_wait(&scfree[slot], ((gg / SR) - 1) & 1, limit, abort_flag)) {
+                            stop = true;
+                            break;
+                        }
+                        uint8_t* dst = smem + SC_OFF + slot * SC_BYTES;
+                        mbar_arrive_expect_tx(&scfull[slot], SC_BYTES);
+                        bulk_load(dst, sfa + (size_t)(k / R) * g.sfa_ld + m_tile * 128, 512, &scfull[slot]);
+                        bulk_load(dst + 512, sfb + (size_t)(k / R) * g.sfb_ld + n_tile * kBN_I4, 512, &scfull[slot]);
+                        ++gg;
                     }
                     if (k == g.skip_k_tile) continue;
                     uint8_t* st = smem + s * STAGE;
@@ -154,8 +180,10 @@ __global__ void __launch_bounds__(i4::THREADS, 1)
                     tma_load_2d(st + 2 * UN_BYTES + PK_BYTES, &tmB, k * 64, n_tile * kBN_I4, &full[s]);
                 }
             }
-            if (*abort_flag)
+            if (*abort_flag) {
                 for (int j = max(0, gi - STAGES); j < gi; ++j) mbar_wait_drain(&full[j % STAGES], (j / STAGES) & 1, 100000000ull);
+                for (int j = max(0, gg - SR); j < gg; ++j) mbar_wait_drain(&scfull[j % SR], (j / SR) & 1, 100000000ull);
+            }
         }
     } else if (warp == 1) {
         if (lane == 0) {
@@ -223,23 +251,11 @@ __global__ void __launch_bounds__(i4::THREADS, 1)
     } else {
         // ------------------------------ rescale + epilogue ------------------------------
         const int q = warp & 3, half = (warp - 6) >> 2;
-        const int rt = (warp - 6) * 32 + lane;  // 0..255
         const int row = q * 32 + lane;
-        const float* sfa = reinterpret_cast<const float*>(g.sfa);
-        const float* sfb = reinterpret_cast<const float*>(g.sfb);
-        // the scales of group gi+1 (possibly the next tile's first) are fetched
-        // while group gi is rescaled; the MMA sums 16 qa * 16 qw = 256 P, and
-        // scaling sa by 2^-8 (exact) gives float(256 P) * RN(2^-8 sa * sw) = float(P) * RN(sa * sw)
-        auto scales_of = [&](int t, int k, float& sa, float& sb) {
-            int m_tile, n_tile;
-            coords(t, m_tile, n_tile);
-            sa = sfa[(size_t)k * g.sfa_ld + min(m_tile * 128 + row, g.sfa_ld - 1)] * 0.00390625f;
-            sb = rt < 128 ? sfb[(size_t)k * g.sfb_ld + n_tile * kBN_I4 + rt] : 0.0f;
-        };
-        float sa_next = 0.0f, sb_next = 0.0f;
-        if ((int)blockIdx.x < ntiles) scales_of(blockIdx.x, 0, sa_next, sb_next);
-        // After a failed wait the loop keeps running (without waiting or reading
-        // TMEM) so that every rescale thread passes the same named barriers.
+        // the MMA sums 16 qa * 16 qw = 256 P, and scaling sa by 2^-8 (exact)
+        // gives float(256 P) * RN(2^-8 sa * sw) = float(P) * RN(sa * sw)
+        // After a failed wait the loop keeps running without waiting or
+        // reading TMEM.
         bool ok = true;
         int gi = 0;
         for (int t = blockIdx.x; t < ntiles; t += gridDim.x) {
@@ -251,23 +267,19 @@ __global__ void __launch_bounds__(i4::THREADS, 1)
 #pragma unroll
             for (int i = 0; i < 64; ++i) acc[i] = 0.0f;
             for (int k = 0; k < NG; ++k, ++gi) {  // gi: scale groups of every tile, in order
-                const int buf = gi & 1;
-                float* sbb = sb_smem + buf * 128;
-                if (rt < 128) sbb[rt] = sb_next;
-                const float sa = sa_next;
-                if (k + 1 < NG) scales_of(t, k + 1, sa_next, sb_next);
-                else if (t + (int)gridDim.x < ntiles) scales_of(t + gridDim.x, 0, sa_next, sb_next);
-                named_bar(1, 256);
+                const int buf = gi & 1, slot = gi % SR;
+                if (ok) ok = mbar_wait(&scfull[slot], (gi / SR) & 1, limit, abort_flag);
                 if (ok) ok = mbar_wait(&accf[buf], (gi >> 1) & 1, limit, abort_flag);
                 if (!ok) continue;
                 tc_fence_after();
-                const uint64_t sa2 = pack2(sa);
+                const float* sc = sc_smem + slot * (SC_BYTES / 4);
+                const uint64_t sa2 = pack2(sc[row] * 0.00390625f);
 #pragma unroll
                 for (int ch = 0; ch < 2; ++ch) {
                     uint32_t r[32];
                     tmem_ld_32x32b_x32(tmem + ((uint32_t)(q * 32) << 16) + buf * 128 + 64 * half + 32 * ch, r);
                     tmem_ld_wait();
-                    const float4* sb4 = reinterpret_cast<const float4*>(sbb + 64 * half + 32 * ch);
+                    const float4* sb4 = reinterpret_cast<const float4*>(sc + 128 + 64 * half + 32 * ch);
 #pragma unroll
                     for (int i = 0; i < 8; ++i) {
                         const float4 b = sb4[i];
@@ -279,7 +291,10 @@ __global__ void __launch_bounds__(i4::THREADS, 1)
                 }
                 tc_fence_before();
                 __syncwarp();
-                if (lane == 0) mbar_arrive(&tfree[buf]);
+                if (lane == 0) {
+                    mbar_arrive(&tfree[buf]);
+                    mbar_arrive(&scfree[slot]);
+                }
             }
             if (ok && m < g.M && ncol0 < g.N) {
                 uint16_t* dst = g.Y + (size_t)m * g.ldy + ncol0;

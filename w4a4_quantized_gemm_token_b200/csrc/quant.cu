@@ -95,12 +95,29 @@ __device__ __forceinline__ uint32_t neg_lo(uint32_t w) { return (w << 16) ^ 0x80
 __device__ __forceinline__ uint32_t neg_hi(uint32_t w) { return (w & 0xFFFF0000u) ^ 0x80000000u; }
 
 // E2M1 codes of x/d for the 8 elements held in w[0..3], quotients correctly
-// rounded by the refined division (divisor and quotients in normal range).
+// rounded by the refined division (divisor and quotients in normal range),
+// on sm_100's packed FP32 operations.  ny2 holds ny = -RN(1/d) (both
+// halves), d2 holds d.  With the dividend x as it is: q = RN(x * ny) is
+// within an ulp of -x/d, R = q*d + x is exact, and q' = RN(R * ny + q) is
+// the correctly rounded -x/d (the same correction step as div_refined).
+// The codes of -x/d are those of x/d with the sign bit flipped (the E2M1
+// grid and its rounding are symmetric), so one XOR per 8 codes restores
+// them; a dividend of +0 or -0 gives the opposite zero, so the flip keeps
+// the sign of zero too.
 __device__ __forceinline__ uint32_t e2m1x8_fast(const uint32_t* w, uint64_t ny2, uint64_t d2) {
+    const float2 ny = make_float2(__uint_as_float((uint32_t)ny2), __uint_as_float((uint32_t)ny2));
+    const float2 d = make_float2(__uint_as_float((uint32_t)d2), __uint_as_float((uint32_t)d2));
     float q[8];
 #pragma unroll
-    for (int e = 0; e < 4; ++e) div2_refined(neg_lo(w[e]), neg_hi(w[e]), ny2, d2, q[2 * e], q[2 * e + 1]);
-    return e2m1x8(q);
+    for (int e = 0; e < 4; ++e) {
+        const float2 x = make_float2(bf16lo(w[e]), bf16hi(w[e]));
+        const float2 q0 = __fmul2_rn(x, ny);
+        const float2 r = __ffma2_rn(q0, d, x);
+        const float2 q1 = __ffma2_rn(r, ny, q0);
+        q[2 * e] = q1.x;
+        q[2 * e + 1] = q1.y;
+    }
+    return e2m1x8(q) ^ 0x88888888u;
 }
 // The same with IEEE division (any operands).
 __device__ __forceinline__ uint32_t e2m1x8_exact(uint4 v, float d) {
@@ -892,8 +909,12 @@ __global__ void __launch_bounds__(J <= 2 ? 1024 : 768) quant_nvfp4_token_kernel(
             const int it = t + T * j;
             uint32_t sb, w0, w1;
             if (fast) {
-                const float u = div_refined(bm[j], 6.0f, 0x1.555556p-3f);  // RN(1/6)
-                sb = e4m3_rn_sat(div_refined(u, s2, rinv));
+                // RN(RN(bm / 6) / s2) by the refined division; both operands are
+                // non-negative, so no sign fix-up is needed
+                const float u0 = __fmul_rn(bm[j], 0x1.555556p-3f);  // RN(1/6)
+                const float u = __fmaf_rn(__fmaf_rn(-u0, 6.0f, bm[j]), 0x1.555556p-3f, u0);
+                const float v0 = __fmul_rn(u, rinv);
+                sb = e4m3_rn_sat(__fmaf_rn(__fmaf_rn(-v0, s2, u), rinv, v0));
                 const float d = sb ? __fmul_rn(e4m3_value((uint8_t)sb), s2) : 1.0f;
                 const float y = __frcp_rn(d);
                 if constexpr (ROT) {

@@ -632,7 +632,7 @@ int orc_augment_nvfp4(const uint16_t* X, int M, int K, int ldx,
                       uint8_t* rcodes, uint8_t* rscales) {
     if (nS % 16 || K % 16 || ldx < K) return -1;
     for (int j = 0; j < nS; ++j)
-        if (S[j] < 0 || S[j] >= K || (j > 0 && S[j] <= S[j - 1])) return -1;
+        if (S[j] < 0 || S[j] >= K) return -1; /* any order: column K + j holds channel S[j] */
     float* r = (float*)malloc(sizeof(float) * (size_t)(nS > 0 ? nS : 1));
     for (int m = 0; m < M; ++m) {
         float rs2 = (mode == 1) ? s2[m] : s2[0];

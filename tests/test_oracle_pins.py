@@ -340,10 +340,13 @@ def test_gemm_fp64_brute_force(orc, K):
 
 
 # ---- residual augmentation ----------------------------------------------------
-def test_augment_invariants(orc):
+@pytest.mark.parametrize("order", ["asc", "perm"])
+def test_augment_invariants(orc, order):
     M, K, nS = 16, 512, 32
     X = bf16(synth.normal((M, K), 1.0, 30, 1) * np.where(np.arange(K) % 37 == 0, 30.0, 1.0))
     S = orc.select_channels(X, nS)
+    if order == "perm":  # column K + j holds channel S[j], whatever the order
+        S = S[np.random.default_rng(3).permutation(nS)]
     c, s, s2 = orc.quant_nvfp4(X, mode=1)
     rc, rs = orc.augment_nvfp4(X, S, c, s, s2, 1)
     x = synth.bf16_bits_to_f32(X).astype(np.float64)

@@ -53,8 +53,8 @@ def mma_issue_peak_tflops(dev, sm_mhz: float) -> float:
 # dominant kernel, averaged over the five GEMM launches of one step, from an ncu
 # capture of the pair GEMM on this workload; valid only for the kernel source it
 # was measured on (else reported as null).
-PROFILED_TRAFFIC = {"sources": ("gemm_fp4_pair.cu", "ptx.cuh"), "sha256_16": "718b7937ac7f9a8f",
-                    "bytes_per_launch": 295.0e6}
+PROFILED_TRAFFIC = {"sources": ("gemm_fp4_pair.cu", "ptx.cuh"), "sha256_16": "1c98d42c0906a8c3",
+                    "bytes_per_launch": 303.7e6}
 
 
 def profiled_traffic():

@@ -162,8 +162,8 @@ int w4a4_quantize_act(const uint16_t* X, int M, int K, int ldx,
  * Quantize weights W[N,K] (bf16, row stride ldw) once, offline.  Same block
  * rules as w4a4_quantize_act; NVFP4 weights here use one tensor scale
  * (out->scale_mode must be TENSOR; w4a4_quantize_weight_segments gives one
- * scale per row segment).  With S (device int32[nS], strictly
- * ascending channel indices in [0,K), nS a multiple of 128) the quantized
+ * scale per row segment).  With S (device int32[nS], channel indices in
+ * [0,K) in any order, nS a multiple of 128) the quantized
  * tensor is [W | W[:,S]] with cols = K + nS: the weight side of the
  * dual-stage residual augmentation ("APEX4..." page, para 2, ARCQuant).
  */
@@ -302,7 +302,11 @@ int w4a4_linear_msd(const uint16_t* X, int M, int K, int ldx,
  * x^ is the first-stage dequantized value (code * block scale * s2, rounded
  * to FP32) read from Xaug's first K columns, and R is quantized to NVFP4
  * with the row's own s2 into columns K .. K+nS-1 of Xaug.
- * S: device int32[nS], strictly ascending, in [0,K); nS a multiple of 128.
+ * S: device int32[nS], in [0,K), in any order (w4a4_select_channels writes
+ * them ascending; the order is the order of the residual columns, and the
+ * weights must be quantized with the same S); nS a multiple of 128.  An
+ * index outside [0,K) is replaced by channel 0 and makes
+ * w4a4_device_status return W4A4_ERR_INVALID_ARG.
  * Xaug: NVFP4, rows = M, cols = K + nS, first K columns already quantized.
  */
 int w4a4_augment_residual(const uint16_t* X, int M, int K, int ldx,

@@ -210,6 +210,11 @@ def test_qwen25_3b_augmented(orc, li):
     _, yref, absd = orc.gemm_nvfp4(ca, sa, s2a, 1, cw, sw, s2w)
     bad = H.gemm_violations(H.to_np_u16(Y)[rows], yref, absd)
     assert not bad.any(), f"{bad.sum()} bad"
+    # the linear's quantizer computes the residual stage in the same launch:
+    # its product equals the two-call path's byte for byte
+    Y2 = w4.gemm(Xq, Wq)
+    torch.cuda.synchronize()
+    assert torch.equal(Y.view(torch.int16), Y2.view(torch.int16))
 
 
 @pytest.mark.parametrize("M", [4096, 600])

@@ -219,7 +219,44 @@ def test_augment_parity(orc, mode):
     Y1 = w4.gemm(Xq, Wq)
     Y2 = w4.linear(dev(Xa), Wq, mode, S=S)
     torch.cuda.synchronize()
+    assert w4.device_status() == w4.OK
     _, yref, absd = _linear_ref(orc, w4.NVFP4, Xa, Xw, mode, S=S_np)
+    for Y in (Y1, Y2):
+        bad = H.gemm_violations(H.to_np_u16(Y), yref, absd)
+        assert not bad.any(), f"{bad.sum()} bad"
+    # the linear (whose per-token quantizer computes the residual stage in the
+    # same launch) multiplies the same operands as the two-call path: the
+    # same GEMM kernel gives the same bytes
+    assert torch.equal(Y1.view(torch.int16), Y2.view(torch.int16))
+
+
+@pytest.mark.parametrize("M,K,nS,order", [(1, 1024, 128, "asc"), (37, 2048, 256, "asc"), (300, 2816, 384, "asc"),
+                                           (5, 11008, 256, "asc"), (200, 2048, 256, "desc"),
+                                           (130, 4096, 128, "perm")])
+def test_fused_residual_stage_matches_two_calls(orc, M, K, nS, order):
+    """The fused linear's residual channels equal the separate second stage
+    (w4a4_augment_residual after w4a4_quantize_act) bit for bit: the two
+    paths' products agree byte for byte at every token count, on the
+    decode, one-CTA and CTA-pair GEMMs, whatever the order of the channels."""
+    N = 256
+    Xa = synth.activations("qwen25_3b_aug", M, K, seed=17)
+    Xw = synth.weights("qwen25_3b_aug", N, K, seed=17)
+    S = w4.select_channels(dev(synth.calibration("qwen25_3b_aug", K, rows=512)), nS)
+    if order == "desc":
+        S = S.flip(0).contiguous()
+    elif order == "perm":
+        S = S[torch.from_numpy(np.random.default_rng(5).permutation(nS)).to(S.device)].contiguous()
+    Wq = w4.quantize_weight(dev(Xw), w4.NVFP4, S=S)
+    Xd = dev(Xa)
+    Xq = w4.quantize_act(Xd, w4.NVFP4, w4.SCALE_TOKEN, cols=K + nS)
+    w4.augment_residual(Xd, S, Xq)
+    Y1 = w4.gemm(Xq, Wq)
+    Y2 = w4.linear(Xd, Wq, w4.SCALE_TOKEN, S=S)
+    torch.cuda.synchronize()
+    assert w4.device_status() == w4.OK
+    if M > 16:  # same GEMM kernel on both paths (the decode variant has its own reduction order)
+        assert torch.equal(Y1.view(torch.int16), Y2.view(torch.int16))
+    _, yref, absd = _linear_ref(orc, w4.NVFP4, Xa, Xw, w4.SCALE_TOKEN, S=S.cpu().numpy())
     for Y in (Y1, Y2):
         bad = H.gemm_violations(H.to_np_u16(Y), yref, absd)
         assert not bad.any(), f"{bad.sum()} bad"

@@ -142,10 +142,15 @@ int cuda_status(cudaError_t e) { return e == cudaSuccess ? W4A4_OK : W4A4_ERR_CU
 // pad_scales: also write the zero scales of the padding rows [M, pad128(M))
 // of the 128-row scale atoms (the public layout); the fused linear's
 // workspace skips them, since every GEMM masks rows past M.
+// res_S / res_n (NVFP4 activations with residual channels): when the
+// per-token quantizer runs, it also writes the second stage into columns
+// K .. K + res_n and *res_done is set; otherwise the caller runs it.
 int quantize_rows(const uint16_t* X, int M, int K, int ldx, const int32_t* S, int K_src, const float* static_s2,
                   w4a4_qtensor* q, int num_sms, cudaStream_t st, int* zero_words = nullptr, int zero_count = 0,
-                  int passes = 1, bool weight_side = false, bool pad_scales = true) {
+                  int passes = 1, bool weight_side = false, bool pad_scales = true, const int32_t* res_S = nullptr,
+                  int res_n = 0, bool* res_done = nullptr) {
     const int rows_pad = pad_scales ? pad128(M) : M;
+    if (res_done) *res_done = false;
     QuantArgs a{};
     a.passes = passes;
     a.rot = (q->flags & W4A4_FLAG_HADAMARD) ? (weight_side ? 2 : 1) : 0;
@@ -183,6 +188,14 @@ int quantize_rows(const uint16_t* X, int M, int K, int ldx, const int32_t* S, in
         }
         e = launch_amax(X, M, K_src, ldx, q->s2 + 1, num_sms, st, a.rot);
         if (e != cudaSuccess) return W4A4_ERR_CUDA;
+    }
+    // the per-token kernel (the path launch_quant takes for these arguments)
+    // can fuse the residual-channel stage
+    if (res_n && q->format == W4A4_NVFP4 && !S && !static_s2 && !a.rot && passes == 1 && !a.int8_codes &&
+        K == K_src && K <= 49152 && nvfp4_token_fuses_residual(K, res_n)) {
+        a.res_S = res_S;
+        a.res_n = res_n;
+        if (res_done) *res_done = true;
     }
     return cuda_status(launch_quant(q->format, S != nullptr, a, rows_pad, num_sms, st));
 }
@@ -572,10 +585,11 @@ int w4a4_linear(const uint16_t* X, int M, int K, int ldx, const w4a4_qtensor* Wq
     const bool small_m = use_small_m(fmt, M, N, xq.cols, sms);
     int* counters = small_m ? reinterpret_cast<int*>(base + L.counters) : nullptr;
     // the quantizer clears the decode GEMM's per-tile counters on its way
+    bool res_done = false;
     rc = quantize_rows(X, M, K, ldx, nullptr, K, nullptr, &xq, sms, st, counters, small_m ? (N + kBM - 1) / kBM : 0,
-                       1, false, false);
+                       1, false, false, nS ? S : nullptr, nS, &res_done);
     if (rc != W4A4_OK) return rc;
-    if (nS) {
+    if (nS && !res_done) {
         ResidualArgs r{X, M, K, ldx, pad128(M), S, nS, static_cast<uint8_t*>(xq.codes), xq.cols / 2,
                        static_cast<uint8_t*>(xq.scales), xq.cols / 16 / 4, xq.s2, xq.scale_mode};
         if (launch_residual(r, st) != cudaSuccess) return W4A4_ERR_CUDA;

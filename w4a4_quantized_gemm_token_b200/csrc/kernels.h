@@ -57,7 +57,13 @@ struct QuantArgs {
     int int8_codes;            // INT4: write codes as int8 16 * q ([M][ldc] bytes, ldc >= K)
     int rot;                   // block-local Walsh-Hadamard rotation: 0 none, 1 activation
                                // side (times 1/block), 2 weight side (unscaled)
+    const int32_t* res_S;      // NVFP4 per-token activations: the residual channels of the
+    int res_n;                 // second stage, written at columns K .. K + res_n (0 = none)
 };
+
+// Whether the per-token NVFP4 quantizer can also compute the residual-channel
+// second stage of a row (res_n channels of a K-column row) in the same launch.
+bool nvfp4_token_fuses_residual(int K, int res_n);
 
 struct ResidualArgs {
     const uint16_t* X;

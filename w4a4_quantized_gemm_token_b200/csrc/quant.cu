@@ -52,6 +52,17 @@ __device__ __forceinline__ uint32_t e2m1x8(const float (&v)[8]) {
     return out;
 }
 
+// E2M1 code of one value (the low nibble of a pair conversion with +0).
+__device__ __forceinline__ uint32_t e2m1_one(float v) {
+    uint32_t out;
+    asm("{\n\t.reg .b8 b0;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b0, %2, %1;\n\t"
+        "cvt.u32.u8 %0, b0;\n\t}"
+        : "=r"(out)
+        : "f"(v), "f"(0.0f));
+    return out & 15u;
+}
+
 // Correctly rounded quotient x/d from a correctly rounded reciprocal
 // y = RN(1/d): q = RN(x*y) is within an ulp of x/d, the residual x - q*d is
 // exact in one FMA, and one more FMA rounds q + residual*y to RN(x/d).  This
@@ -705,6 +716,34 @@ __global__ void __launch_bounds__(256) amax_rot_kernel(const uint16_t* X, int M,
     }
 }
 
+// NVFP4 codes (w0: elements 0..7, w1: 8..15) and E4M3 scale of one 16-element
+// block of second-stage residuals R with the row's scale s2: the same rule as
+// the first stage (block scale E4M3(RN(RN(amax / 6) / s2)), codes E2M1 of the
+// correctly rounded quotients), by IEEE division for the scale and by refined
+// division for the codes wherever that is exact.
+__device__ __forceinline__ uint8_t residual_block(const float* R, float s2, uint32_t& w0, uint32_t& w1) {
+    float bmax = 0.0f;
+#pragma unroll
+    for (int i = 0; i < 16; ++i) bmax = fmaxf(bmax, fabsf(R[i]));
+    const uint8_t sb = e4m3_rn_sat(__fdiv_rn(__fdiv_rn(bmax, 6.0f), s2));
+    w0 = 0;
+    w1 = 0;
+    if (sb != 0) {
+        const float d = __fmul_rn(e4m3_value(sb), s2);
+        const float y = __frcp_rn(d);
+        const bool exact = !(d >= 0x1p-100f && d <= 0x1p100f && __fmul_rn(bmax, y) <= 0x1p60f);
+        float q0[8], q1[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+            q0[e] = exact ? __fdiv_rn(R[e], d) : div_refined(R[e], d, y);
+            q1[e] = exact ? __fdiv_rn(R[8 + e], d) : div_refined(R[8 + e], d, y);
+        }
+        w0 = e2m1x8(q0);
+        w1 = e2m1x8(q1);
+    }
+    return sb;
+}
+
 // ---------------------------------------------------------------------------
 // Residual second stage: thread = (row, 16-block of the nS residual channels).
 // ---------------------------------------------------------------------------
@@ -721,7 +760,6 @@ __global__ void __launch_bounds__(128) residual_kernel(ResidualArgs a) {
     if (r < a.M) {
         const float s2 = a.s2[a.mode == 1 ? r : 0];
         float R[16];
-        float bmax = 0.0f;
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
             const int k = checked_channel(a.S, 16 * b + i, a.K);
@@ -733,22 +771,8 @@ __global__ void __launch_bounds__(128) residual_kernel(ResidualArgs a) {
             const float sv = e4m3_value(a.sf[sf_offset(r, k >> 4, a.sf_col_atoms)]);
             const float xhat = __fmul_rn(__fmul_rn(ev, sv), s2);  // ev*sv is exact
             R[i] = __fsub_rn(x, xhat);
-            bmax = fmaxf(bmax, fabsf(R[i]));
         }
-        sb = e4m3_rn_sat(__fdiv_rn(__fdiv_rn(bmax, 6.0f), s2));
-        if (sb != 0) {
-            const float d = __fmul_rn(e4m3_value(sb), s2);
-            const float y = __frcp_rn(d);
-            const bool exact = !(d >= 0x1p-100f && d <= 0x1p100f && __fmul_rn(bmax, y) <= 0x1p60f);
-            float q0[8], q1[8];
-#pragma unroll
-            for (int e = 0; e < 8; ++e) {
-                q0[e] = exact ? __fdiv_rn(R[e], d) : div_refined(R[e], d, y);
-                q1[e] = exact ? __fdiv_rn(R[8 + e], d) : div_refined(R[8 + e], d, y);
-            }
-            w0 = e2m1x8(q0);
-            w1 = e2m1x8(q1);
-        }
+        sb = residual_block(R, s2, w0, w1);
         *reinterpret_cast<uint2*>(a.codes + (size_t)r * a.ldc + (a.K >> 1) + 8 * b) = make_uint2(w0, w1);
     }
     a.sf[sf_offset(r, cblk, a.sf_col_atoms)] = sb;
@@ -829,7 +853,17 @@ __global__ void __launch_bounds__(1024) compact_kernel(const int* selected, int 
 // ROT: every 16-element block rotated first (rotate_item; a block is one
 // item, so no lane exchange; a.rot 1 = activation side, 2 = weight side).
 // TENSOR: one s2 for the whole tensor (see below) instead of one per row.
-template <int J, bool ROT, bool TENSOR>
+// RES: also the residual-channel second stage ("APEX4..." page, para 2:
+// ARCQuant) of every row, written at columns K .. K + res_n.  Each thread
+// keeps its blocks' codes and scales in shared memory as well; after a CTA
+// barrier, residual channel e = S[e] of the row (still in its ring buffer,
+// which is refilled only once the next row has started) is taken by one
+// thread: R = x - x^ with x^ = code value * block scale * s2.  Sixteen
+// consecutive lanes hold one residual block and encode it together with the
+// row's s2: block maximum by lane exchange, then the rule of the separate
+// second-stage kernel (residual_block) per element.  S is cached per CTA; an
+// index outside [0, K) is recorded in the error word and channel 0 taken.
+template <int J, bool ROT, bool TENSOR, bool RES>
 __global__ void __launch_bounds__(J <= 2 ? 1024 : 768) quant_nvfp4_token_kernel(QuantArgs a, int nb) {
     pdl_launch_dependents();
     pdl_wait();  // X and the words to clear may belong to the preceding launch
@@ -843,6 +877,10 @@ __global__ void __launch_bounds__(J <= 2 ? 1024 : 768) quant_nvfp4_token_kernel(
     const int row_bytes = a.K * 2;
     uint64_t* bars = reinterpret_cast<uint64_t*>(qring + (size_t)nb * row_bytes);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + nb);
+    // RES: the residual channels S, and the current row's codes and block scales
+    int32_t* sS = reinterpret_cast<int32_t*>(bars + nb + 2);
+    uint2* scodes = reinterpret_cast<uint2*>(sS + (RES ? a.res_n : 0));
+    uint8_t* sbs = reinterpret_cast<uint8_t*>(scodes + (RES ? items : 0));
     const int G = gridDim.x;
     // rows of this CTA that are loaded: blockIdx.x + i*G < M
     const int nlive = a.M > (int)blockIdx.x ? (a.M - 1 - (int)blockIdx.x) / G + 1 : 0;
@@ -862,6 +900,8 @@ __global__ void __launch_bounds__(J <= 2 ? 1024 : 768) quant_nvfp4_token_kernel(
         fence_mbar_init();
         for (int i = 0; i < nb && i < nlive; ++i) issue(i);
     }
+    if constexpr (RES)
+        for (int k = t; k < a.res_n; k += T) sS[k] = checked_channel(a.res_S, k, a.K);
     __syncthreads();
     for (int i = 0; i < nlive; ++i) {
         const int b = i % nb, r = blockIdx.x + i * G;
@@ -896,7 +936,13 @@ __global__ void __launch_bounds__(J <= 2 ? 1024 : 768) quant_nvfp4_token_kernel(
             if (lane == 0) wmax[i & 1][warp] = m;
         }
         __syncthreads();  // (also: every thread has its row data in registers)
-        if (t == 0 && i + nb < nlive) issue(i + nb);  // the buffer is free again
+        // the buffer is free again: this row's (RES: the previous row's, whose
+        // second stage read it until this barrier)
+        if constexpr (RES) {
+            if (t == 0 && i >= 1 && i - 1 + nb < nlive) issue(i - 1 + nb);
+        } else {
+            if (t == 0 && i + nb < nlive) issue(i + nb);
+        }
         float s2 = ts2;
         if constexpr (!TENSOR) {
             s2 = nvfp4_s2(warp_max_nonneg(lane < nwarps ? wmax[i & 1][lane] : 0.0f));
@@ -939,6 +985,12 @@ __global__ void __launch_bounds__(J <= 2 ? 1024 : 768) quant_nvfp4_token_kernel(
                 w0 = 0;
                 w1 = 0;
             }
+            if constexpr (RES) {
+                if (it < items) {
+                    scodes[it] = make_uint2(w0, w1);
+                    sbs[it] = (uint8_t)sb;
+                }
+            }
             // four consecutive items sit on lanes l .. l+3 (T is a multiple of 32)
             const uint32_t b1 = __shfl_down_sync(0xffffffffu, sb, 1);
             const uint32_t b2 = __shfl_down_sync(0xffffffffu, sb, 2);
@@ -948,6 +1000,58 @@ __global__ void __launch_bounds__(J <= 2 ? 1024 : 768) quant_nvfp4_token_kernel(
                     *reinterpret_cast<uint32_t*>(a.sf + sf_offset(r, it, a.sf_col_atoms)) =
                         sb | (b1 << 8) | (b2 << 16) | (b3 << 24);
                 *reinterpret_cast<uint2*>(a.codes + (size_t)r * a.ldc + 8 * it) = make_uint2(w0, w1);
+            }
+        }
+        if constexpr (RES) {
+            // the second stage of this row (the next row rewrites the codes and
+            // scales in shared memory only after its own barrier)
+            __syncthreads();
+            const uint16_t* xs = reinterpret_cast<const uint16_t*>(xr);
+            const uint8_t* cb = reinterpret_cast<const uint8_t*>(scodes);
+            // T and res_n are multiples of 32 and 16: the 16 lanes of a residual
+            // block are all live or all past res_n, and every lane of a warp
+            // runs the same iterations
+            for (int e0 = 0; e0 < a.res_n; e0 += T) {
+                const int e = e0 + t;
+                const bool live = e < a.res_n;
+                float R = 0.0f;
+                if (live) {
+                    const int k = sS[e];
+                    const float x = __uint_as_float((uint32_t)xs[k] << 16);
+                    const uint32_t nib = (cb[k >> 1] >> (4 * (k & 1))) & 15u;
+                    // x - code value * block scale * s2 (the first product is exact)
+                    R = __fsub_rn(x, __fmul_rn(__fmul_rn(e2m1_decode(nib), e4m3_value(sbs[k >> 4])), s2));
+                }
+                float bmax = fabsf(R);
+#pragma unroll
+                for (int o = 8; o > 0; o >>= 1) bmax = fmaxf(bmax, __shfl_xor_sync(0xffffffffu, bmax, o));
+                // E4M3(RN(RN(bmax / 6) / s2)): by refined divisions in the range
+                // where they are exact, as for the first stage (R is finite
+                // for finite x, so bmax is too)
+                uint8_t sbr;
+                if (fast) {
+                    const float u0 = __fmul_rn(bmax, 0x1.555556p-3f);  // RN(1/6)
+                    const float u = __fmaf_rn(__fmaf_rn(-u0, 6.0f, bmax), 0x1.555556p-3f, u0);
+                    const float v0 = __fmul_rn(u, rinv);
+                    sbr = e4m3_rn_sat(__fmaf_rn(__fmaf_rn(-v0, s2, u), rinv, v0));
+                } else {
+                    sbr = e4m3_rn_sat(__fdiv_rn(__fdiv_rn(bmax, 6.0f), s2));
+                }
+                uint32_t word = 0;
+                if (sbr != 0) {
+                    const float d = __fmul_rn(e4m3_value(sbr), s2);
+                    const float y = __frcp_rn(d);
+                    const bool exact = !(d >= 0x1p-100f && d <= 0x1p100f && __fmul_rn(bmax, y) <= 0x1p60f);
+                    word = e2m1_one(exact ? __fdiv_rn(R, d) : div_refined(R, d, y)) << (4 * (e & 7));
+                }
+#pragma unroll
+                for (int o = 4; o > 0; o >>= 1) word |= __shfl_xor_sync(0xffffffffu, word, o);
+                const uint32_t hi = __shfl_down_sync(0xffffffffu, word, 8);
+                if (live && (e & 15) == 0) {
+                    *reinterpret_cast<uint2*>(a.codes + (size_t)r * a.ldc + (a.K >> 1) + 8 * (e >> 4)) =
+                        make_uint2(word, hi);
+                    a.sf[sf_offset(r, (a.K >> 4) + (e >> 4), a.sf_col_atoms)] = sbr;
+                }
             }
         }
     }
@@ -1003,14 +1107,22 @@ __global__ void __launch_bounds__(1024) quant_nvfp4_tensor_onepass_kernel(QuantA
     if (nlive > 0) mbar_wait(&bar, 0, 2000000000ull, abort_flag);
     // the CTA's amax (block maxima as in the token kernel; NaN ignored)
     const int total = nlive * items;
+    // item f = t + k T of the CTA's rows is (row i, item it); both advance by
+    // (T / items, T % items) per step, so no division inside the loops
+    const int di = T / items, dit = T - di * items, i0 = t / items, it0 = t - i0 * items;
     float m = 0.0f;
     if (!*abort_flag)
-        for (int f = t; f < total; f += T) {
-            const int i = f / items, it = f - i * items;
+        for (int f = t, i = i0, it = it0; f < total; f += T) {
             const uint4* p = reinterpret_cast<const uint4*>(rows + (size_t)i * row_bytes) + 2 * it;
             const uint4 v0 = p[0], v1 = p[1];
             const uint32_t w[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
             m = fmaxf(m, bmax16(w));
+            i += di;
+            it += dit;
+            if (it >= items) {
+                it -= items;
+                ++i;
+            }
         }
     m = warp_max_nonneg(m);
     if (lane == 0) red[warp] = m;
@@ -1044,10 +1156,16 @@ __global__ void __launch_bounds__(1024) quant_nvfp4_tensor_onepass_kernel(QuantA
     const float rinv = __frcp_rn(s2);
     const bool fast = s2 >= 0x1p-100f;  // the same for the whole grid
     const int iters = (total + T - 1) / T;
-    for (int k = 0; k < iters; ++k) {
+    for (int k = 0, fi = i0, fit = it0; k < iters; ++k) {
         const int f = t + k * T;
         const bool valid = f < total;  // uniform over groups of four lanes
-        const int i = valid ? f / items : 0, it = valid ? f - i * items : 0;
+        const int i = valid ? fi : 0, it = valid ? fit : 0;
+        fi += di;
+        fit += dit;
+        if (fit >= items) {
+            fit -= items;
+            ++fi;
+        }
         const int r = (int)blockIdx.x + i * G;
         uint32_t w[8] = {0, 0, 0, 0, 0, 0, 0, 0};
         if (valid) {
@@ -1142,15 +1260,20 @@ static cudaError_t launch_dep(void (*kern)(Args...), dim3 grid, dim3 block, size
 }
 
 template <int J, bool ROT>
-static const void* tok_kernel(bool tensor) {
-    return tensor ? reinterpret_cast<const void*>(quant_nvfp4_token_kernel<J, ROT, true>)
-                  : reinterpret_cast<const void*>(quant_nvfp4_token_kernel<J, ROT, false>);
+static const void* tok_kernel(bool tensor, bool res) {
+    if constexpr (!ROT) {
+        if (res)
+            return tensor ? reinterpret_cast<const void*>(quant_nvfp4_token_kernel<J, false, true, true>)
+                          : reinterpret_cast<const void*>(quant_nvfp4_token_kernel<J, false, false, true>);
+    }
+    return tensor ? reinterpret_cast<const void*>(quant_nvfp4_token_kernel<J, ROT, true, false>)
+                  : reinterpret_cast<const void*>(quant_nvfp4_token_kernel<J, ROT, false, false>);
 }
 
-template <int J, bool ROT, bool TENSOR>
+template <int J, bool ROT, bool TENSOR, bool RES>
 static cudaError_t launch_tok_mode(const QuantArgs& b, int grid, int T, size_t smem, int nb, cudaStream_t st) {
     static SmemAttrCache smem_attr;
-    auto kern = quant_nvfp4_token_kernel<J, ROT, TENSOR>;
+    auto kern = quant_nvfp4_token_kernel<J, ROT, TENSOR, RES>;
     const cudaError_t e = ensure_dynamic_smem(reinterpret_cast<const void*>(kern), smem, smem_attr);
     if (e != cudaSuccess) return e;
     return launch_dep(kern, dim3(grid), dim3(T), smem, st, b, nb);
@@ -1158,8 +1281,17 @@ static cudaError_t launch_tok_mode(const QuantArgs& b, int grid, int T, size_t s
 
 template <int J, bool ROT>
 static cudaError_t launch_tok(const QuantArgs& b, int grid, int T, size_t smem, int nb, cudaStream_t st) {
-    return b.mode == 0 ? launch_tok_mode<J, ROT, true>(b, grid, T, smem, nb, st)
-                       : launch_tok_mode<J, ROT, false>(b, grid, T, smem, nb, st);
+    if constexpr (!ROT) {
+        if (b.res_n > 0)
+            return b.mode == 0 ? launch_tok_mode<J, false, true, true>(b, grid, T, smem, nb, st)
+                               : launch_tok_mode<J, false, false, true>(b, grid, T, smem, nb, st);
+    }
+    return b.mode == 0 ? launch_tok_mode<J, ROT, true, false>(b, grid, T, smem, nb, st)
+                       : launch_tok_mode<J, ROT, false, false>(b, grid, T, smem, nb, st);
+}
+
+bool nvfp4_token_fuses_residual(int K, int res_n) {
+    return res_n > 0 && res_n % 16 == 0 && res_n <= 1024 && K / 16 <= 2048;
 }
 
 static cudaError_t launch_nvfp4_token(const QuantArgs& a, int rows_pad, int num_sms, cudaStream_t st) {
@@ -1176,11 +1308,14 @@ static cudaError_t launch_nvfp4_token(const QuantArgs& a, int rows_pad, int num_
     // memory per SM
     const int row_bytes = a.K * 2;
     const bool tensor = a.mode == 0;
-    const void* kern = J == 1 ? (a.rot ? tok_kernel<1, true>(tensor) : tok_kernel<1, false>(tensor))
-                     : J == 2 ? (a.rot ? tok_kernel<2, true>(tensor) : tok_kernel<2, false>(tensor))
-                              : tok_kernel<4, false>(tensor);
-    static std::atomic<int> regs_seen[3][2][2];  // [J 1/2/4][rot][tensor]: registers per thread
-    std::atomic<int>& rs = regs_seen[J == 1 ? 0 : J == 2 ? 1 : 2][a.rot ? 1 : 0][tensor ? 1 : 0];
+    const bool res = a.res_n > 0;
+    if (res && (a.rot || !nvfp4_token_fuses_residual(a.K, a.res_n))) return cudaErrorInvalidValue;
+    const void* kern = J == 1 ? (a.rot ? tok_kernel<1, true>(tensor, false) : tok_kernel<1, false>(tensor, res))
+                     : J == 2 ? (a.rot ? tok_kernel<2, true>(tensor, false) : tok_kernel<2, false>(tensor, res))
+                              : tok_kernel<4, false>(tensor, res);
+    // [J 1/2/4][rot][tensor][res]: registers per thread
+    static std::atomic<int> regs_seen[3][2][2][2];
+    std::atomic<int>& rs = regs_seen[J == 1 ? 0 : J == 2 ? 1 : 2][a.rot ? 1 : 0][tensor ? 1 : 0][res ? 1 : 0];
     int regs = rs.load(std::memory_order_relaxed);
     if (!regs) {
         cudaFuncAttributes fa{};
@@ -1190,12 +1325,14 @@ static cudaError_t launch_nvfp4_token(const QuantArgs& a, int rows_pad, int num_
     }
     const int warp_regs = (regs * 32 + 255) / 256 * 256;
     int per_sm = 65536 / ((T / 32) * warp_regs);
-    const int by_smem = (200 * 1024) / (3 * row_bytes);
+    // the residual stage's shared arrays: S, and one row's codes and block scales
+    const int res_bytes = res ? (4 * a.res_n + 9 * items + 15) / 16 * 16 : 0;
+    const int by_smem = (200 * 1024) / (3 * row_bytes + res_bytes);
     per_sm = per_sm < by_smem ? per_sm : by_smem;
     per_sm = per_sm < 1 ? 1 : (per_sm > 16 ? 16 : per_sm);
-    int nb = (200 * 1024) / (per_sm * row_bytes);
+    int nb = ((200 * 1024) / per_sm - res_bytes) / row_bytes;
     nb = nb < 2 ? 2 : (nb > 8 ? 8 : nb);
-    const size_t smem = (size_t)nb * row_bytes + 8 * nb + 16;
+    const size_t smem = (size_t)nb * row_bytes + 8 * nb + 16 + res_bytes;
     if (smem > 220 * 1024) return cudaErrorInvalidValue;
     int grid = num_sms * per_sm;
     if (grid > rows_pad) grid = rows_pad;

@@ -232,7 +232,7 @@ def test_augment_parity(orc, mode):
 
 @pytest.mark.parametrize("M,K,nS,order", [(1, 1024, 128, "asc"), (37, 2048, 256, "asc"), (300, 2816, 384, "asc"),
                                            (5, 11008, 256, "asc"), (200, 2048, 256, "desc"),
-                                           (130, 4096, 128, "perm")])
+                                           (130, 4096, 128, "perm"), (70, 4096, 256, "asc")])
 def test_fused_residual_stage_matches_two_calls(orc, M, K, nS, order):
     """The fused linear's residual channels equal the separate second stage
     (w4a4_augment_residual after w4a4_quantize_act) bit for bit: the two

@@ -52,15 +52,15 @@ __device__ __forceinline__ uint32_t e2m1x8(const float (&v)[8]) {
     return out;
 }
 
-// E2M1 code of one value (the low nibble of a pair conversion with +0).
-__device__ __forceinline__ uint32_t e2m1_one(float v) {
+// E2M1 codes of two values in one byte, lo in the low nibble.
+__device__ __forceinline__ uint32_t e2m1x2_byte(float lo, float hi) {
     uint32_t out;
     asm("{\n\t.reg .b8 b0;\n\t"
         "cvt.rn.satfinite.e2m1x2.f32 b0, %2, %1;\n\t"
         "cvt.u32.u8 %0, b0;\n\t}"
         : "=r"(out)
-        : "f"(v), "f"(0.0f));
-    return out & 15u;
+        : "f"(lo), "f"(hi));
+    return out & 0xFFu;
 }
 
 // Correctly rounded quotient x/d from a correctly rounded reciprocal
@@ -832,6 +832,87 @@ __global__ void __launch_bounds__(1024) compact_kernel(const int* selected, int 
 // ---------------------------------------------------------------------------
 // Host launchers
 // ---------------------------------------------------------------------------
+// Second stage of one row in the per-token kernel (RES): residual channel e
+// (e < res_n, in S order) of the row is R = x - x^, with x from the row
+// buffer xs, and its first-stage code and block scale from cb / sbs
+// (x^ = code value * block scale * s2).  Sixteen channels form a residual
+// block; EPL consecutive channels per lane, so 16 / EPL lanes share a block:
+// block maximum by lane exchange, block scale E4M3(RN(RN(max / 6) / s2)) and
+// codes E2M1(RN(R / d)), the rule of residual_block.  The lane holding a
+// block's first channel writes its 8 code bytes to crow + 8 * block and its
+// scale at block column c0 + block.  Every lane of the CTA calls this (the
+// loop bounds are CTA-uniform; T is a multiple of 32, res_n of 16).
+template <int EPL>
+__device__ __forceinline__ void residual_stage(const uint16_t* xs, const uint8_t* cb, const uint8_t* sbs,
+                                               const int32_t* sS, int res_n, float s2, float rinv, bool fast,
+                                               uint8_t* crow, uint8_t* sf, int r, int c0, int sf_col_atoms) {
+    constexpr int LPB = 16 / EPL;  // lanes per residual block
+    constexpr int LPW = 8 / EPL;   // lanes per 32-bit word of codes
+    const int t = threadIdx.x, T = blockDim.x;
+    for (int e0 = 0; e0 < res_n; e0 += EPL * T) {
+        const int e = e0 + EPL * t;  // this lane's first channel
+        const bool live = e < res_n;  // the same for the lanes of a block
+        float R[EPL];
+#pragma unroll
+        for (int j = 0; j < EPL; ++j) R[j] = 0.0f;
+        if (live) {
+            int k[EPL];
+            if constexpr (EPL == 4) {
+                const int4 v = *reinterpret_cast<const int4*>(sS + e);
+                k[0] = v.x; k[1] = v.y; k[2] = v.z; k[3] = v.w;
+            } else if constexpr (EPL == 2) {
+                const int2 v = *reinterpret_cast<const int2*>(sS + e);
+                k[0] = v.x; k[1] = v.y;
+            } else {
+                k[0] = sS[e];
+            }
+#pragma unroll
+            for (int j = 0; j < EPL; ++j) {
+                const float x = __uint_as_float((uint32_t)xs[k[j]] << 16);
+                const uint32_t nib = (cb[k[j] >> 1] >> (4 * (k[j] & 1))) & 15u;
+                // the first product is exact
+                R[j] = __fsub_rn(x, __fmul_rn(__fmul_rn(e2m1_decode(nib), e4m3_value(sbs[k[j] >> 4])), s2));
+            }
+        }
+        float bmax = fabsf(R[0]);
+#pragma unroll
+        for (int j = 1; j < EPL; ++j) bmax = fmaxf(bmax, fabsf(R[j]));
+#pragma unroll
+        for (int o = LPB / 2; o > 0; o >>= 1) bmax = fmaxf(bmax, __shfl_xor_sync(0xffffffffu, bmax, o));
+        // block scale by refined divisions in the range where they are exact,
+        // as for the first stage (R is finite for finite x, so bmax is too)
+        uint8_t sbr;
+        if (fast) {
+            const float u0 = __fmul_rn(bmax, 0x1.555556p-3f);  // RN(1/6)
+            const float u = __fmaf_rn(__fmaf_rn(-u0, 6.0f, bmax), 0x1.555556p-3f, u0);
+            const float v0 = __fmul_rn(u, rinv);
+            sbr = e4m3_rn_sat(__fmaf_rn(__fmaf_rn(-v0, s2, u), rinv, v0));
+        } else {
+            sbr = e4m3_rn_sat(__fdiv_rn(__fdiv_rn(bmax, 6.0f), s2));
+        }
+        uint32_t h = 0;  // this lane's 4 * EPL bits of codes, channel e + j in nibble j
+        if (sbr != 0) {
+            const float d = __fmul_rn(e4m3_value(sbr), s2);
+            const float y = __frcp_rn(d);
+            const bool exact = !(d >= 0x1p-100f && d <= 0x1p100f && __fmul_rn(bmax, y) <= 0x1p60f);
+            float q[EPL];
+#pragma unroll
+            for (int j = 0; j < EPL; ++j) q[j] = exact ? __fdiv_rn(R[j], d) : div_refined(R[j], d, y);
+            if constexpr (EPL == 4) h = e2m1x2_byte(q[0], q[1]) | (e2m1x2_byte(q[2], q[3]) << 8);
+            else if constexpr (EPL == 2) h = e2m1x2_byte(q[0], q[1]);
+            else h = e2m1x2_byte(q[0], 0.0f) & 15u;
+        }
+        uint32_t word = h << (4 * EPL * (t % LPW));
+#pragma unroll
+        for (int o = LPW / 2; o > 0; o >>= 1) word |= __shfl_xor_sync(0xffffffffu, word, o);
+        const uint32_t hi = __shfl_down_sync(0xffffffffu, word, LPW);
+        if (live && t % LPB == 0) {
+            *reinterpret_cast<uint2*>(crow + 8 * (e >> 4)) = make_uint2(word, hi);
+            sf[sf_offset(r, c0 + (e >> 4), sf_col_atoms)] = sbr;
+        }
+    }
+}
+
 // ---------------------------------------------------------------------------
 // NVFP4 with a dynamic per-token scale (the activation hot path), or with the
 // dynamic tensor scale of an amax pass (TENSOR mode).  Persistent
@@ -857,14 +938,14 @@ __global__ void __launch_bounds__(1024) compact_kernel(const int* selected, int 
 // ARCQuant) of every row, written at columns K .. K + res_n.  Each thread
 // keeps its blocks' codes and scales in shared memory as well; after a CTA
 // barrier, residual channel e = S[e] of the row (still in its ring buffer,
-// which is refilled only once the next row has started) is taken by one
-// thread: R = x - x^ with x^ = code value * block scale * s2.  Sixteen
-// consecutive lanes hold one residual block and encode it together with the
-// row's s2: block maximum by lane exchange, then the rule of the separate
-// second-stage kernel (residual_block) per element.  S is cached per CTA; an
-// index outside [0, K) is recorded in the error word and channel 0 taken.
-template <int J, bool ROT, bool TENSOR, bool RES>
+// which is refilled only once the next row has started) gives
+// R = x - x^ with x^ = code value * block scale * s2 (residual_stage: EPL
+// channels per lane, 16 / EPL lanes per residual block; EPL = 0 is the
+// kernel without the second stage).  S is cached per CTA; an index outside
+// [0, K) is recorded in the error word and channel 0 taken.
+template <int J, bool ROT, bool TENSOR, int EPL>
 __global__ void __launch_bounds__(J <= 2 ? 1024 : 768) quant_nvfp4_token_kernel(QuantArgs a, int nb) {
+    constexpr bool RES = EPL > 0;
     pdl_launch_dependents();
     pdl_wait();  // X and the words to clear may belong to the preceding launch
     if (blockIdx.x == 0)
@@ -878,7 +959,8 @@ __global__ void __launch_bounds__(J <= 2 ? 1024 : 768) quant_nvfp4_token_kernel(
     uint64_t* bars = reinterpret_cast<uint64_t*>(qring + (size_t)nb * row_bytes);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + nb);
     // RES: the residual channels S, and the current row's codes and block scales
-    int32_t* sS = reinterpret_cast<int32_t*>(bars + nb + 2);
+    // (16-byte aligned: four channels are read at a time)
+    int32_t* sS = reinterpret_cast<int32_t*>((reinterpret_cast<uintptr_t>(bars + nb + 2) + 15) & ~uintptr_t(15));
     uint2* scodes = reinterpret_cast<uint2*>(sS + (RES ? a.res_n : 0));
     uint8_t* sbs = reinterpret_cast<uint8_t*>(scodes + (RES ? items : 0));
     const int G = gridDim.x;
@@ -991,14 +1073,11 @@ __global__ void __launch_bounds__(J <= 2 ? 1024 : 768) quant_nvfp4_token_kernel(
                     sbs[it] = (uint8_t)sb;
                 }
             }
-            // four consecutive items sit on lanes l .. l+3 (T is a multiple of 32)
-            const uint32_t b1 = __shfl_down_sync(0xffffffffu, sb, 1);
-            const uint32_t b2 = __shfl_down_sync(0xffffffffu, sb, 2);
-            const uint32_t b3 = __shfl_down_sync(0xffffffffu, sb, 3);
+            // one byte per scale: the warp's stores still fill whole 4-byte
+            // groups (items l .. l+3 sit on consecutive lanes), without lane
+            // exchanges to assemble them
             if (it < items) {
-                if ((it & 3) == 0)
-                    *reinterpret_cast<uint32_t*>(a.sf + sf_offset(r, it, a.sf_col_atoms)) =
-                        sb | (b1 << 8) | (b2 << 16) | (b3 << 24);
+                a.sf[sf_offset(r, it, a.sf_col_atoms)] = (uint8_t)sb;
                 *reinterpret_cast<uint2*>(a.codes + (size_t)r * a.ldc + 8 * it) = make_uint2(w0, w1);
             }
         }
@@ -1006,53 +1085,9 @@ __global__ void __launch_bounds__(J <= 2 ? 1024 : 768) quant_nvfp4_token_kernel(
             // the second stage of this row (the next row rewrites the codes and
             // scales in shared memory only after its own barrier)
             __syncthreads();
-            const uint16_t* xs = reinterpret_cast<const uint16_t*>(xr);
-            const uint8_t* cb = reinterpret_cast<const uint8_t*>(scodes);
-            // T and res_n are multiples of 32 and 16: the 16 lanes of a residual
-            // block are all live or all past res_n, and every lane of a warp
-            // runs the same iterations
-            for (int e0 = 0; e0 < a.res_n; e0 += T) {
-                const int e = e0 + t;
-                const bool live = e < a.res_n;
-                float R = 0.0f;
-                if (live) {
-                    const int k = sS[e];
-                    const float x = __uint_as_float((uint32_t)xs[k] << 16);
-                    const uint32_t nib = (cb[k >> 1] >> (4 * (k & 1))) & 15u;
-                    // x - code value * block scale * s2 (the first product is exact)
-                    R = __fsub_rn(x, __fmul_rn(__fmul_rn(e2m1_decode(nib), e4m3_value(sbs[k >> 4])), s2));
-                }
-                float bmax = fabsf(R);
-#pragma unroll
-                for (int o = 8; o > 0; o >>= 1) bmax = fmaxf(bmax, __shfl_xor_sync(0xffffffffu, bmax, o));
-                // E4M3(RN(RN(bmax / 6) / s2)): by refined divisions in the range
-                // where they are exact, as for the first stage (R is finite
-                // for finite x, so bmax is too)
-                uint8_t sbr;
-                if (fast) {
-                    const float u0 = __fmul_rn(bmax, 0x1.555556p-3f);  // RN(1/6)
-                    const float u = __fmaf_rn(__fmaf_rn(-u0, 6.0f, bmax), 0x1.555556p-3f, u0);
-                    const float v0 = __fmul_rn(u, rinv);
-                    sbr = e4m3_rn_sat(__fmaf_rn(__fmaf_rn(-v0, s2, u), rinv, v0));
-                } else {
-                    sbr = e4m3_rn_sat(__fdiv_rn(__fdiv_rn(bmax, 6.0f), s2));
-                }
-                uint32_t word = 0;
-                if (sbr != 0) {
-                    const float d = __fmul_rn(e4m3_value(sbr), s2);
-                    const float y = __frcp_rn(d);
-                    const bool exact = !(d >= 0x1p-100f && d <= 0x1p100f && __fmul_rn(bmax, y) <= 0x1p60f);
-                    word = e2m1_one(exact ? __fdiv_rn(R, d) : div_refined(R, d, y)) << (4 * (e & 7));
-                }
-#pragma unroll
-                for (int o = 4; o > 0; o >>= 1) word |= __shfl_xor_sync(0xffffffffu, word, o);
-                const uint32_t hi = __shfl_down_sync(0xffffffffu, word, 8);
-                if (live && (e & 15) == 0) {
-                    *reinterpret_cast<uint2*>(a.codes + (size_t)r * a.ldc + (a.K >> 1) + 8 * (e >> 4)) =
-                        make_uint2(word, hi);
-                    a.sf[sf_offset(r, (a.K >> 4) + (e >> 4), a.sf_col_atoms)] = sbr;
-                }
-            }
+            residual_stage<EPL>(reinterpret_cast<const uint16_t*>(xr), reinterpret_cast<const uint8_t*>(scodes),
+                                sbs, sS, a.res_n, s2, rinv, fast, a.codes + (size_t)r * a.ldc + (a.K >> 1), a.sf, r,
+                                a.K >> 4, a.sf_col_atoms);
         }
     }
     if (*abort_flag && t == 0)  // wait for the copies still in flight
@@ -1158,7 +1193,7 @@ __global__ void __launch_bounds__(1024) quant_nvfp4_tensor_onepass_kernel(QuantA
     const int iters = (total + T - 1) / T;
     for (int k = 0, fi = i0, fit = it0; k < iters; ++k) {
         const int f = t + k * T;
-        const bool valid = f < total;  // uniform over groups of four lanes
+        const bool valid = f < total;
         const int i = valid ? fi : 0, it = valid ? fit : 0;
         fi += di;
         fit += dit;
@@ -1193,14 +1228,8 @@ __global__ void __launch_bounds__(1024) quant_nvfp4_tensor_onepass_kernel(QuantA
             w0 = 0;
             w1 = 0;
         }
-        // four consecutive items of one row sit on lanes l .. l+3
-        const uint32_t b1 = __shfl_down_sync(0xffffffffu, sb, 1);
-        const uint32_t b2 = __shfl_down_sync(0xffffffffu, sb, 2);
-        const uint32_t b3 = __shfl_down_sync(0xffffffffu, sb, 3);
-        if (valid) {
-            if ((it & 3) == 0)
-                *reinterpret_cast<uint32_t*>(a.sf + sf_offset(r, it, a.sf_col_atoms)) =
-                    sb | (b1 << 8) | (b2 << 16) | (b3 << 24);
+        if (valid) {  // one byte per scale (as in the per-token kernel)
+            a.sf[sf_offset(r, it, a.sf_col_atoms)] = (uint8_t)sb;
             *reinterpret_cast<uint2*>(a.codes + (size_t)r * a.ldc + 8 * it) = make_uint2(w0, w1);
         }
     }
@@ -1259,35 +1288,42 @@ static cudaError_t launch_dep(void (*kern)(Args...), dim3 grid, dim3 block, size
     return cudaLaunchKernelEx(&cfg, kern, args...);
 }
 
+template <int J, bool ROT, int EPL>
+static const void* tok_kernel_e(bool tensor) {
+    return tensor ? reinterpret_cast<const void*>(quant_nvfp4_token_kernel<J, ROT, true, EPL>)
+                  : reinterpret_cast<const void*>(quant_nvfp4_token_kernel<J, ROT, false, EPL>);
+}
 template <int J, bool ROT>
-static const void* tok_kernel(bool tensor, bool res) {
+static const void* tok_kernel(bool tensor, int epl) {
     if constexpr (!ROT) {
-        if (res)
-            return tensor ? reinterpret_cast<const void*>(quant_nvfp4_token_kernel<J, false, true, true>)
-                          : reinterpret_cast<const void*>(quant_nvfp4_token_kernel<J, false, false, true>);
+        if (epl == 4) return tok_kernel_e<J, false, 4>(tensor);
+        if (epl == 2) return tok_kernel_e<J, false, 2>(tensor);
+        if (epl == 1) return tok_kernel_e<J, false, 1>(tensor);
     }
-    return tensor ? reinterpret_cast<const void*>(quant_nvfp4_token_kernel<J, ROT, true, false>)
-                  : reinterpret_cast<const void*>(quant_nvfp4_token_kernel<J, ROT, false, false>);
+    return tok_kernel_e<J, ROT, 0>(tensor);
 }
 
-template <int J, bool ROT, bool TENSOR, bool RES>
+template <int J, bool ROT, bool TENSOR, int EPL>
 static cudaError_t launch_tok_mode(const QuantArgs& b, int grid, int T, size_t smem, int nb, cudaStream_t st) {
     static SmemAttrCache smem_attr;
-    auto kern = quant_nvfp4_token_kernel<J, ROT, TENSOR, RES>;
+    auto kern = quant_nvfp4_token_kernel<J, ROT, TENSOR, EPL>;
     const cudaError_t e = ensure_dynamic_smem(reinterpret_cast<const void*>(kern), smem, smem_attr);
     if (e != cudaSuccess) return e;
     return launch_dep(kern, dim3(grid), dim3(T), smem, st, b, nb);
 }
-
+template <int J, bool ROT, int EPL>
+static cudaError_t launch_tok_e(const QuantArgs& b, int grid, int T, size_t smem, int nb, cudaStream_t st) {
+    return b.mode == 0 ? launch_tok_mode<J, ROT, true, EPL>(b, grid, T, smem, nb, st)
+                       : launch_tok_mode<J, ROT, false, EPL>(b, grid, T, smem, nb, st);
+}
 template <int J, bool ROT>
-static cudaError_t launch_tok(const QuantArgs& b, int grid, int T, size_t smem, int nb, cudaStream_t st) {
+static cudaError_t launch_tok(const QuantArgs& b, int epl, int grid, int T, size_t smem, int nb, cudaStream_t st) {
     if constexpr (!ROT) {
-        if (b.res_n > 0)
-            return b.mode == 0 ? launch_tok_mode<J, false, true, true>(b, grid, T, smem, nb, st)
-                               : launch_tok_mode<J, false, false, true>(b, grid, T, smem, nb, st);
+        if (epl == 4) return launch_tok_e<J, false, 4>(b, grid, T, smem, nb, st);
+        if (epl == 2) return launch_tok_e<J, false, 2>(b, grid, T, smem, nb, st);
+        if (epl == 1) return launch_tok_e<J, false, 1>(b, grid, T, smem, nb, st);
     }
-    return b.mode == 0 ? launch_tok_mode<J, ROT, true, false>(b, grid, T, smem, nb, st)
-                       : launch_tok_mode<J, ROT, false, false>(b, grid, T, smem, nb, st);
+    return launch_tok_e<J, ROT, 0>(b, grid, T, smem, nb, st);
 }
 
 bool nvfp4_token_fuses_residual(int K, int res_n) {
@@ -1310,12 +1346,15 @@ static cudaError_t launch_nvfp4_token(const QuantArgs& a, int rows_pad, int num_
     const bool tensor = a.mode == 0;
     const bool res = a.res_n > 0;
     if (res && (a.rot || !nvfp4_token_fuses_residual(a.K, a.res_n))) return cudaErrorInvalidValue;
-    const void* kern = J == 1 ? (a.rot ? tok_kernel<1, true>(tensor, false) : tok_kernel<1, false>(tensor, res))
-                     : J == 2 ? (a.rot ? tok_kernel<2, true>(tensor, false) : tok_kernel<2, false>(tensor, res))
-                              : tok_kernel<4, false>(tensor, res);
+    // second stage: four residual channels per lane where every thread has at
+    // least four, else fewer, so that more warps share a short stage
+    const int epl = !res ? 0 : 4 * T <= a.res_n ? 4 : 2 * T <= a.res_n ? 2 : 1;
+    const void* kern = J == 1 ? (a.rot ? tok_kernel<1, true>(tensor, 0) : tok_kernel<1, false>(tensor, epl))
+                     : J == 2 ? (a.rot ? tok_kernel<2, true>(tensor, 0) : tok_kernel<2, false>(tensor, epl))
+                              : tok_kernel<4, false>(tensor, epl);
     // [J 1/2/4][rot][tensor][res]: registers per thread
-    static std::atomic<int> regs_seen[3][2][2][2];
-    std::atomic<int>& rs = regs_seen[J == 1 ? 0 : J == 2 ? 1 : 2][a.rot ? 1 : 0][tensor ? 1 : 0][res ? 1 : 0];
+    static std::atomic<int> regs_seen[3][2][2][4];  // [J][rot][tensor][EPL 0, 1, 2, 4]
+    std::atomic<int>& rs = regs_seen[J == 1 ? 0 : J == 2 ? 1 : 2][a.rot ? 1 : 0][tensor ? 1 : 0][epl == 4 ? 3 : epl];
     int regs = rs.load(std::memory_order_relaxed);
     if (!regs) {
         cudaFuncAttributes fa{};
@@ -1326,7 +1365,7 @@ static cudaError_t launch_nvfp4_token(const QuantArgs& a, int rows_pad, int num_
     const int warp_regs = (regs * 32 + 255) / 256 * 256;
     int per_sm = 65536 / ((T / 32) * warp_regs);
     // the residual stage's shared arrays: S, and one row's codes and block scales
-    const int res_bytes = res ? (4 * a.res_n + 9 * items + 15) / 16 * 16 : 0;
+    const int res_bytes = res ? (4 * a.res_n + 9 * items + 15) / 16 * 16 + 16 : 0;  // + alignment of S
     const int by_smem = (200 * 1024) / (3 * row_bytes + res_bytes);
     per_sm = per_sm < by_smem ? per_sm : by_smem;
     per_sm = per_sm < 1 ? 1 : (per_sm > 16 ? 16 : per_sm);
@@ -1343,9 +1382,12 @@ static cudaError_t launch_nvfp4_token(const QuantArgs& a, int rows_pad, int num_
     QuantArgs b = a;
     b.rows_pad = rows_pad;
     cudaError_t e;
-    if (J == 1) e = a.rot ? launch_tok<1, true>(b, grid, T, smem, nb, st) : launch_tok<1, false>(b, grid, T, smem, nb, st);
-    else if (J == 2) e = a.rot ? launch_tok<2, true>(b, grid, T, smem, nb, st) : launch_tok<2, false>(b, grid, T, smem, nb, st);
-    else e = launch_tok<4, false>(b, grid, T, smem, nb, st);
+    if (J == 1)
+        e = a.rot ? launch_tok<1, true>(b, 0, grid, T, smem, nb, st) : launch_tok<1, false>(b, epl, grid, T, smem, nb, st);
+    else if (J == 2)
+        e = a.rot ? launch_tok<2, true>(b, 0, grid, T, smem, nb, st) : launch_tok<2, false>(b, epl, grid, T, smem, nb, st);
+    else
+        e = launch_tok<4, false>(b, epl, grid, T, smem, nb, st);
     return e != cudaSuccess ? e : cudaGetLastError();
 }
 

@@ -38,6 +38,7 @@ PEAKS_FILE = os.path.join(ROOT, "MEASURED_PEAKS.json")
 FP4_PER_BF16 = 4.0        # nominal dense FP4 / BF16 tensor throughput (9 / 2.25 PFLOP/s)
 INT8_PER_BF16 = 2.0       # nominal dense INT8 / BF16 (4.5 / 2.25)
 NOMINAL_FP4_TFLOPS = 9000.0  # B200 dense FP4, nominal
+NOMINAL_INT8_TOPS = 4500.0   # B200 dense INT8, nominal
 # FP4 MMA issue rate per SM: one 128x256x64 NVFP4 MMA (2 * 128 * 256 * 64 FLOP)
 # every 128 cycles, measured back to back on one SM
 MMA_FLOP_PER_CYCLE = 2 * 128 * 256 * 64 // 128
@@ -583,7 +584,8 @@ def extra_rows(args, dev, stream, P):
             tot_ms += ms
             tot_ops += 2.0 * M * N * K
         v = tot_ops / (tot_ms * 1e-3) / 1e12
-        out[f"int4_g{G}_qwen25_7b_m2048"] = {"TOPS": round(v, 1), "frac_int8_peak": round(v / i8_peak, 3)}
+        out[f"int4_g{G}_qwen25_7b_m2048"] = {"TOPS": round(v, 1), "frac_int8_peak": round(v / i8_peak, 3),
+                                             "frac_of_nominal_int8_4p5": round(v / NOMINAL_INT8_TOPS, 3)}
 
     # dual-stage residual augmentation, Qwen2.5-3B shapes at M = 8192
     tot_ms, tot_f, tot_fk = 0.0, 0.0, 0.0

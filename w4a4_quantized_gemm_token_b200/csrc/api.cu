@@ -148,7 +148,7 @@ int cuda_status(cudaError_t e) { return e == cudaSuccess ? W4A4_OK : W4A4_ERR_CU
 int quantize_rows(const uint16_t* X, int M, int K, int ldx, const int32_t* S, int K_src, const float* static_s2,
                   w4a4_qtensor* q, int num_sms, cudaStream_t st, int* zero_words = nullptr, int zero_count = 0,
                   int passes = 1, bool weight_side = false, bool pad_scales = true, const int32_t* res_S = nullptr,
-                  int res_n = 0, bool* res_done = nullptr) {
+                  int res_n = 0, bool* res_done = nullptr, bool chained = false) {
     const int rows_pad = pad_scales ? pad128(M) : M;
     if (res_done) *res_done = false;
     QuantArgs a{};
@@ -178,11 +178,17 @@ int quantize_rows(const uint16_t* X, int M, int K, int ldx, const int32_t* S, in
         // dynamic tensor scale: s2[1] collects the amax (s2[2] counts the CTAs
         // of the one-pass kernel); one cooperative pass when all rows fit in
         // shared memory, else an amax pass and the quantizer
-        cudaError_t e = cudaMemsetAsync(q->s2 + 1, 0, 2 * sizeof(float), st);
+        // Inside the fused linear (chained: a GEMM follows) the two words are
+        // cleared by a kernel that is a programmatic dependent of the
+        // preceding launch, and the one-pass quantizer is one too, so their
+        // launches overlap the preceding GEMM's tail (SwiGLU layer 145 -> 141
+        // us); alone, a memset and a plain cooperative launch cost less.
+        cudaError_t e = chained ? launch_clear_tensor_amax(q->s2 + 1, st)
+                                : cudaMemsetAsync(q->s2 + 1, 0, 2 * sizeof(float), st);
         if (e != cudaSuccess) return W4A4_ERR_CUDA;
         a.tensor_amax = q->s2 + 1;
         if (!S && K == K_src && !a.rot && passes == 1 && !a.int8_codes && nvfp4_tensor_onepass_fits(M, K, num_sms)) {
-            e = launch_nvfp4_tensor_onepass(a, rows_pad, num_sms, reinterpret_cast<unsigned*>(q->s2 + 2), st);
+            e = launch_nvfp4_tensor_onepass(a, rows_pad, num_sms, reinterpret_cast<unsigned*>(q->s2 + 2), chained, st);
             if (e != cudaErrorCooperativeLaunchTooLarge) return cuda_status(e);
             cudaGetLastError();  // fewer SMs available than reported: two passes
         }
@@ -587,7 +593,7 @@ int w4a4_linear(const uint16_t* X, int M, int K, int ldx, const w4a4_qtensor* Wq
     // the quantizer clears the decode GEMM's per-tile counters on its way
     bool res_done = false;
     rc = quantize_rows(X, M, K, ldx, nullptr, K, nullptr, &xq, sms, st, counters, small_m ? (N + kBM - 1) / kBM : 0,
-                       1, false, false, nS ? S : nullptr, nS, &res_done);
+                       1, false, false, nS ? S : nullptr, nS, &res_done, true);
     if (rc != W4A4_OK) return rc;
     if (nS && !res_done) {
         ResidualArgs r{X, M, K, ldx, pad128(M), S, nS, static_cast<uint8_t*>(xq.codes), xq.cols / 2,

@@ -104,7 +104,7 @@ cudaError_t launch_quant(int fmt, bool gather, const QuantArgs& a, int rows_pad,
 // cooperative launch of num_sms CTAs that hold all rows in shared memory:
 // whether M x K fits, and the launch (a.tensor_amax and *arrive zero).
 bool nvfp4_tensor_onepass_fits(int M, int K, int num_sms);
-cudaError_t launch_nvfp4_tensor_onepass(const QuantArgs& a, int rows_pad, int num_sms, unsigned* arrive,
+cudaError_t launch_nvfp4_tensor_onepass(const QuantArgs& a, int rows_pad, int num_sms, unsigned* arrive, bool pdl,
                                         cudaStream_t st);
 // rot: 0 plain amax; 1 / 2 amax of the rotated 16-element blocks (activation / weight side)
 cudaError_t launch_amax(const uint16_t* X, int M, int K, int ldx, float* out, int num_sms, cudaStream_t st,
@@ -112,6 +112,7 @@ cudaError_t launch_amax(const uint16_t* X, int M, int K, int ldx, float* out, in
 cudaError_t launch_residual(const ResidualArgs& a, cudaStream_t st);
 // p[1 .. n) = p[0] (device floats)
 cudaError_t launch_spread_first(float* p, int n, cudaStream_t st);
+cudaError_t launch_clear_tensor_amax(float* p, cudaStream_t st);
 cudaError_t launch_select(const uint16_t* X, int Mc, int K, int ldx, int nS, int32_t* S, float* amax, int* sel,
                           cudaStream_t st);
 

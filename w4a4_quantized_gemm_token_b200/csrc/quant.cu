@@ -1248,7 +1248,7 @@ bool nvfp4_tensor_onepass_fits(int M, int K, int num_sms) {
     return rows * (size_t)K * 2 <= kOnepassSmem;
 }
 
-cudaError_t launch_nvfp4_tensor_onepass(const QuantArgs& a, int rows_pad, int num_sms, unsigned* arrive,
+cudaError_t launch_nvfp4_tensor_onepass(const QuantArgs& a, int rows_pad, int num_sms, unsigned* arrive, bool pdl,
                                         cudaStream_t st) {
     static SmemAttrCache smem_attr;
     const void* kern = reinterpret_cast<const void*>(quant_nvfp4_tensor_onepass_kernel);
@@ -1262,10 +1262,23 @@ cudaError_t launch_nvfp4_tensor_onepass(const QuantArgs& a, int rows_pad, int nu
     cfg.blockDim = dim3(1024);
     cfg.dynamicSmemBytes = smem;
     cfg.stream = st;
-    cudaLaunchAttribute attr[1];
+    // cooperative (every CTA resident: the grid-wide amax wait), and with pdl
+    // a programmatic dependent of the preceding launch where the runtime
+    // allows both; the kernel waits for that launch before touching memory
+    cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeCooperative;
     attr[0].val.cooperative = 1;
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
+    cfg.numAttrs = 2;
+    static std::atomic<int> pdl_refused{0};
+    if (pdl && !pdl_refused.load(std::memory_order_relaxed)) {
+        e = cudaLaunchKernelEx(&cfg, quant_nvfp4_tensor_onepass_kernel, b, arrive);
+        if (e == cudaSuccess || e == cudaErrorCooperativeLaunchTooLarge) return e;
+        cudaGetLastError();  // the combination refused: plain cooperative launches from now on
+        pdl_refused.store(1, std::memory_order_relaxed);
+    }
     cfg.numAttrs = 1;
     return cudaLaunchKernelEx(&cfg, quant_nvfp4_tensor_onepass_kernel, b, arrive);
 }
@@ -1458,10 +1471,24 @@ cudaError_t launch_amax(const uint16_t* X, int M, int K, int ldx, float* out, in
     return cudaGetLastError();
 }
 
+// Zeroes the tensor amax and the one-pass arrival count of an NVFP4 TENSOR
+// activation (p[0], p[1]: s2[1], s2[2]), as a programmatic dependent of the
+// preceding launch, so that the quantizer after it can be one too.
+__global__ void clear_tensor_amax_kernel(float* p) {
+    pdl_launch_dependents();
+    pdl_wait();  // the preceding launch may still read these words
+    if (threadIdx.x < 2) p[threadIdx.x] = 0.0f;
+}
+
 // p[1 .. n) = p[0]: spreads a segment's tensor scale over its rows.
 __global__ void spread_first_kernel(float* p, int n) {
     const float v = p[0];
     for (int i = 1 + blockIdx.x * blockDim.x + threadIdx.x; i < n; i += gridDim.x * blockDim.x) p[i] = v;
+}
+
+cudaError_t launch_clear_tensor_amax(float* p, cudaStream_t st) {
+    const cudaError_t e = launch_dep(clear_tensor_amax_kernel, dim3(1), dim3(32), 0, st, p);
+    return e != cudaSuccess ? e : cudaGetLastError();
 }
 
 cudaError_t launch_spread_first(float* p, int n, cudaStream_t st) {

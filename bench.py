@@ -81,7 +81,7 @@ def peaks():
 # clocks sampled during the timed region
 # ----------------------------------------------------------------------------------------------
 class ClockSampler:
-    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+    QUERY = ("timestamp,index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
@@ -100,7 +100,10 @@ class ClockSampler:
         except Exception:
             self.proc = None
 
-    def stop(self):
+    def stop(self, t0=None, t1=None, t2=None):
+        """Samples taken in the timed region [t0, t1] (host clock); if it was
+        too short to hold one, those of [t1, t2], a window right after it in
+        which the same steps keep running untimed."""
         if self.proc is None:
             return None
         self.proc.terminate()
@@ -111,17 +114,43 @@ class ClockSampler:
         rows = []
         for line in open(self.path):
             f = [x.strip() for x in line.split(",")]
-            if len(f) >= 9:
+            if len(f) >= 10:
                 rows.append(f)
         os.unlink(self.path)
-        if not rows:
-            return None
-        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
-        mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].lower() == "active"})
-        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
-                "reasons": reasons, "samples": len(rows)}
+        return summarize_clocks(rows, t0, t1, t2)
+
+
+def _sample_time(stamp):
+    import datetime
+    try:
+        return datetime.datetime.strptime(stamp, "%Y/%m/%d %H:%M:%S.%f").timestamp()
+    except ValueError:
+        return None
+
+
+def summarize_clocks(rows, t0=None, t1=None, t2=None):
+    """rows: nvidia-smi CSV fields in ClockSampler.QUERY order."""
+    if not rows:
+        return None
+    window = "sampler run"
+    if t0 is not None:
+        ts = [_sample_time(r[0]) for r in rows]
+        inside = [r for r, t in zip(rows, ts) if t is not None and t0 <= t <= t1]
+        after = [r for r, t in zip(rows, ts) if t is not None and t1 < t <= t2]
+        n_in = len(inside)
+        if inside:
+            rows, window = inside, "timed region"
+        elif after:
+            rows, window = after, "the same steps, untimed, right after the timed region (it was shorter than the sampling period)"
+    sm = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+    mx = [float(r[3]) for r in rows if r[3].replace(".", "").isdigit()]
+    names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+    reasons = sorted({names[i] for r in rows for i in range(4) if r[6 + i].lower() == "active"})
+    out = {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+           "reasons": reasons, "samples": len(rows), "window": window}
+    if t0 is not None:
+        out["samples_in_timed_region"] = n_in
+    return out
 
 
 # ----------------------------------------------------------------------------------------------
@@ -332,14 +361,22 @@ def run_ours(args, rank, world):
         dist.barrier()
     torch.cuda.synchronize()
     ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t_clk0 = time.time()
     ev0.record(stream)
     for _ in range(args.steps):
         step()
     ev1.record(stream)
     torch.cuda.synchronize()
+    t_clk1 = time.time()
     if world > 1:
         dist.barrier()
-    clocks = sampler.stop()
+    # the clock window after the timed region: the same steps for 0.4 s,
+    # untimed (used only when the timed region held no clock sample)
+    t_clk2 = time.time() + 0.4
+    while time.time() < t_clk2:
+        step()
+        torch.cuda.synchronize()
+    clocks = sampler.stop(t_clk0, t_clk1, t_clk2)
     ms = ev0.elapsed_time(ev1) / args.steps
     ms = max_over_ranks(ms, dev, world)
     value = flops_step * world / (ms * 1e-3) / 1e12

@@ -262,6 +262,47 @@ def test_fused_residual_stage_matches_two_calls(orc, M, K, nS, order):
         assert not bad.any(), f"{bad.sum()} bad"
 
 
+@pytest.mark.parametrize("bad", [2048 + 5, -3])
+def test_out_of_range_channel_is_channel_zero_and_reported(bad):
+    """A channel index outside [0, K) in a device-side S is taken as channel 0
+    and reported by w4a4_device_status as an invalid argument: the fused
+    linear, the two-call path and the weight gather give exactly the bytes of
+    the list with that index replaced by 0."""
+    M, N, K, nS = 70, 256, 2048, 128
+    Xd = dev(synth.activations("qwen25_3b_aug", M, K, seed=23))
+    Wd = dev(synth.weights("qwen25_3b_aug", N, K, seed=23))
+    S = w4.select_channels(dev(synth.calibration("qwen25_3b_aug", K, rows=512)), nS)
+    S_bad = S.clone()
+    S_bad[37] = bad
+    S_fix = S.clone()
+    S_fix[37] = 0
+    torch.cuda.synchronize()
+    assert w4.device_status() == w4.OK
+    W_bad = w4.quantize_weight(Wd, w4.NVFP4, S=S_bad)
+    torch.cuda.synchronize()
+    assert w4.device_status() == w4.ERR_INVALID_ARG
+    W_fix = w4.quantize_weight(Wd, w4.NVFP4, S=S_fix)
+    torch.cuda.synchronize()
+    assert w4.device_status() == w4.OK
+    assert torch.equal(W_bad.codes, W_fix.codes) and torch.equal(W_bad.scales, W_fix.scales)
+    Y_fix = w4.linear(Xd, W_fix, w4.SCALE_TOKEN, S=S_fix)
+    torch.cuda.synchronize()
+    assert w4.device_status() == w4.OK
+    Y_bad = w4.linear(Xd, W_fix, w4.SCALE_TOKEN, S=S_bad)  # fused second stage
+    torch.cuda.synchronize()
+    assert w4.device_status() == w4.ERR_INVALID_ARG
+    assert torch.equal(Y_bad.view(torch.int16), Y_fix.view(torch.int16))
+    Xq = w4.quantize_act(Xd, w4.NVFP4, w4.SCALE_TOKEN, cols=K + nS)
+    w4.augment_residual(Xd, S_bad, Xq)  # the separate second stage
+    torch.cuda.synchronize()
+    assert w4.device_status() == w4.ERR_INVALID_ARG
+    Xq2 = w4.quantize_act(Xd, w4.NVFP4, w4.SCALE_TOKEN, cols=K + nS)
+    w4.augment_residual(Xd, S_fix, Xq2)
+    torch.cuda.synchronize()
+    assert w4.device_status() == w4.OK
+    assert torch.equal(Xq.codes, Xq2.codes) and torch.equal(Xq.scales, Xq2.scales)
+
+
 def test_determinism_and_poisoned_output(orc):
     """Two runs give identical bytes; every output element is written (NaN poison)."""
     M, N, K = 300, 768, 1024

@@ -698,6 +698,41 @@ def extra_rows(args, dev, stream, P):
                                                   "ms": round(ms, 3)}
         del lay
 
+    # the same layer at M = 4096 as a deployment runs it: gate and up (w1, w3)
+    # read the same normalized input, so they are one module of N = 2 x 28672
+    # with one NVFP4 weight scale per segment, quantized once per call (the
+    # FLOPs are those of the five-linear headline; the headline keeps the five)
+    if want("tokens"):
+        Ms = args.tokens
+        lay = []
+        for li in (0, 1, 4):  # qkv, o, w2
+            name, K, N = LLAMA[li]
+            Wq = w4.quantize_weight(to_dev(synth.weights("llama2_70b", N, K, seed=0, tensor_id=100 + li), dev),
+                                    w4.NVFP4)
+            X = to_dev(synth.activations("llama2_70b", Ms, K, seed=0, tensor_id=200 + li), dev)
+            lay.append((K, N, Wq, X))
+        _, K13, N1 = LLAMA[2]
+        W13 = torch.cat([to_dev(synth.weights("llama2_70b", N1, K13, seed=0, tensor_id=100 + li), dev) for li in (2, 3)])
+        Wq13 = w4.quantize_weight_segments(W13, [0, N1, 2 * N1])
+        del W13
+        X13 = to_dev(synth.activations("llama2_70b", Ms, K13, seed=0, tensor_id=202), dev)
+        lay.insert(2, (K13, 2 * N1, Wq13, X13))
+        lay = [(K, N, Wq, X, torch.empty(Ms, N, dtype=torch.bfloat16, device=dev),
+                torch.empty(w4.linear_workspace(Ms, N, K, w4.NVFP4), dtype=torch.uint8, device=dev))
+               for (K, N, Wq, X) in lay]
+
+        def fused_step():
+            for (K, N, Wq, X, Y, ws) in lay:
+                w4.linear(X, Wq, w4.SCALE_TOKEN, Y=Y, ws=ws)
+        for _ in range(max(3, args.warmup)):
+            fused_step()
+        ms = time_loop(fused_step, max(3, min(args.steps, 10)), stream)
+        fl = sum(2.0 * Ms * N * K for (K, N, *_r) in lay)
+        out[f"linear_nvfp4_llama_layer_gate_up_fused_m{Ms}"] = {
+            "TFLOPS": round(fl / (ms * 1e-3) / 1e12, 1), "ms": round(ms, 3),
+            "linears": "qkv, o, w1|w3 as one module (per-segment weight scales), w2"}
+        del lay
+
     # the 300M SwiGLU decoder layer at M = 4096, NVFP4 with a tensor scale on
     # both sides (the activation scale from an amax pass on every call)
     if want("swiglu"):
